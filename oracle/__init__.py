@@ -1,0 +1,36 @@
+"""CPU oracle for top-p block-sparse self-attention (TEST INFRASTRUCTURE ONLY).
+
+This package is the plain, slow, obviously-correct statement of what the GPU
+path computes.  It exists to check the CUDA library and is used only by
+``tests/``, by ``__graft_entry__.smoke()`` and by the CPU-baseline leg of
+``bench.py``.  Nothing in the product package imports it, and it imports
+nothing from the product package: it shares no code, tables or helpers with
+the CUDA path.  Inputs arrive as numpy arrays; random draws are made by the
+caller.
+
+Sources (cited by page title and section in every function):
+
+* "RECAP: Reciprocal Sparse Attention and Hierarchical Caching for Efficient
+  Video Diffusion" -- full text, sections 1, 3.2, 3.4 (block means, cached
+  dense refinement that corrects the sparse estimate, dense refreshes).
+* the head-wise adaptive top-p abstract (Temporal Mask Reuse / Error-guided
+  Budgeted Calibration) and the GSRS abstract ("Top-p selection for adaptive
+  sparsity control") -- online top-p block selection with per-head p.
+* "Ride the Wave: Precision-Allocated Sparse Attention for Smooth Video
+  Generation" (DFSAttn) abstract -- Hilbert-curve token reordering, block
+  scoring.
+* CalibAtt (calibrated sparse attention), abstract and Fig. 5 -- threshold the
+  top key blocks per query block, skip the unselected blocks.
+
+Modules:
+  hilbert     -- 3-D Hilbert order of the latent grid, perm / inv
+  scoring     -- block mean pooling and per-query-block softmax of block logits
+  topp        -- cumulative top-p block selection, mask and kept lists
+  attention   -- masked softmax attention over the kept blocks (O, LSE)
+  correction  -- dense-minus-sparse refinement and the alpha-scaled correction
+
+Every function carries a "Pinned by" note naming the tests in
+``tests/test_oracle.py`` that tie it to something other than itself.
+"""
+
+from . import hilbert, scoring, topp, attention, correction  # noqa: F401

@@ -1,0 +1,449 @@
+"""Pins of the CPU oracle to things other than itself (CPU only).
+
+Each test ties one oracle function to a closed form, a textbook or library
+routine, a brute-force enumeration or an invariant, so that a dropped term,
+a wrong sign or index or a transposed operand fails at least one of them.
+The last group plants such mistakes in copies of oracle functions and checks
+that the pins catch them.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as oatt
+from oracle import correction as ocor
+from oracle import hilbert as ohil
+from oracle import scoring as osco
+from oracle import topp as otop
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------- Hilbert
+
+def _cube_points(k, n=3):
+    side = 1 << k
+    grids = np.meshgrid(*[np.arange(side)] * n, indexing="ij")
+    return np.stack([g.ravel() for g in grids]).astype(np.int64)
+
+
+@pytest.mark.parametrize("k", [1, 2, 3])
+def test_hilbert_full_cube_is_a_continuous_bijection(k):
+    pts = _cube_points(k)
+    d = ohil.hilbert_index(pts, k)
+    assert sorted(d.tolist()) == list(range(8 ** k))
+    walk = pts[:, np.argsort(d)]
+    steps = np.abs(np.diff(walk, axis=1)).sum(axis=0)
+    assert np.all(steps == 1), "consecutive curve points must be unit neighbours"
+    assert np.all(walk[:, 0] == 0), "curve starts at the origin"
+
+
+@pytest.mark.parametrize("k", [2, 3])
+def test_hilbert_aligned_runs_fill_aligned_subcubes(k):
+    pts = _cube_points(k)
+    d = ohil.hilbert_index(pts, k)
+    walk = pts[:, np.argsort(d)]
+    for m in range(1, k):
+        run = 8 ** m
+        side = 1 << m
+        for start in range(0, 8 ** k, run):
+            seg = walk[:, start:start + run]
+            lo = seg.min(axis=1)
+            assert np.all(lo % side == 0)
+            assert np.all(seg.max(axis=1) - lo == side - 1)
+            assert len({tuple(c) for c in seg.T}) == run
+
+
+def _textbook_d2xy(n, d):
+    """Classic quadrant-rotation Hilbert curve on an n x n square (n = 2^k)."""
+    x = y = 0
+    s = 1
+    t = d
+    while s < n:
+        rx = 1 & (t // 2)
+        ry = 1 & (t ^ rx)
+        if ry == 0:
+            if rx == 1:
+                x, y = s - 1 - x, s - 1 - y
+            x, y = y, x
+        x += s * rx
+        y += s * ry
+        t //= 4
+        s *= 2
+    return x, y
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4])
+def test_hilbert_2d_matches_textbook_curve(k):
+    n = 1 << k
+    pts = _cube_points(k, n=2)
+    d = ohil.hilbert_index(pts, k)
+    table = {_textbook_d2xy(n, i): i for i in range(n * n)}
+    for j in range(n * n):
+        assert table[(int(pts[0, j]), int(pts[1, j]))] == d[j]
+
+
+@pytest.mark.parametrize("grid", [(2, 32, 32), (3, 5, 7), (1, 1, 1), (21, 30, 52)])
+def test_hilbert_perm_bijection_and_inverse(grid):
+    perm, inv = ohil.hilbert_perm(*grid)
+    L = int(np.prod(grid))
+    assert perm.dtype == np.int32 and perm.size == L
+    assert np.array_equal(np.sort(perm), np.arange(L))
+    assert np.array_equal(perm[inv], np.arange(L))
+    x = np.random.default_rng(0).standard_normal((1, 2, L, 3))
+    y = ohil.permute_rows(x, perm)
+    assert np.array_equal(ohil.permute_rows(y, perm, inverse=True), x)
+
+
+def test_hilbert_grid_is_restriction_of_cube_order():
+    T, Hh, W = 3, 5, 6
+    perm, _ = ohil.hilbert_perm(T, Hh, W)
+    k = ohil.bits_for(max(T, Hh, W))
+    cube = _cube_points(k)
+    order = cube[:, np.argsort(ohil.hilbert_index(cube, k))]
+    inside = (order[0] < T) & (order[1] < Hh) & (order[2] < W)
+    flat = (order[0] * Hh + order[1]) * W + order[2]
+    assert np.array_equal(flat[inside], perm)
+
+
+# ------------------------------------------------------------------ scoring
+
+def test_pool_golden_ramps():
+    cases = json.load(open(os.path.join(GOLDEN, "pool_cases.json")))["cases"]
+    for c in cases:
+        L, blk = c["L"], c["blk"]
+        x = np.broadcast_to(np.arange(L, dtype=np.float64)[None, None, :, None], (1, 1, L, 2))
+        got = osco.pool_blocks(x, blk)[0, 0, :, 0]
+        assert np.allclose(got, c["means"], rtol=0, atol=1e-6), c
+
+
+def test_pool_constant_and_linearity():
+    rng = np.random.default_rng(1)
+    x = np.full((1, 2, 70, 8), 3.25)
+    assert np.all(osco.pool_blocks(x, 16) == np.float32(3.25))
+    a = rng.standard_normal((1, 2, 70, 8))
+    b = rng.standard_normal((1, 2, 70, 8))
+    lhs = osco.pool_blocks(2 * a - b, 16)
+    rhs = 2 * osco.pool_blocks(a, 16).astype(np.float64) - osco.pool_blocks(b, 16)
+    assert np.allclose(lhs, rhs, atol=1e-5)
+
+
+def test_block_probs_rows_sum_to_one_and_match_scipy():
+    from scipy.special import softmax
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((1, 3, 300, 16)).astype(np.float32)
+    k = rng.standard_normal((1, 3, 300, 16)).astype(np.float32)
+    qbar, kbar, P = osco.score_blocks(q, k, 64)
+    assert P.shape == (1, 3, 5, 5) and P.dtype == np.float32
+    assert np.allclose(P.sum(-1), 1, atol=1e-6)
+    # logits formed independently: loop over pairs, explicit 1/sqrt(D)
+    S = np.zeros((1, 3, 5, 5))
+    for h in range(3):
+        for i in range(5):
+            for j in range(5):
+                S[0, h, i, j] = float(np.dot(qbar[0, h, i].astype(np.float64),
+                                             kbar[0, h, j].astype(np.float64))) / 4.0
+    assert np.allclose(P, softmax(S, axis=-1), rtol=1e-6, atol=1e-9)
+    # rows are not symmetric in general: the query side is the row
+    assert not np.allclose(P, np.swapaxes(P, -1, -2))
+
+
+def test_block_probs_uniform_for_constant_keys():
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((1, 1, 256, 8))
+    k = np.ones((1, 1, 256, 8)) * 0.7
+    _, _, P = osco.score_blocks(q, k, 32)
+    assert np.allclose(P, 1.0 / 8, atol=1e-7)
+
+
+def test_block_probs_prefers_aligned_key():
+    # one key block aligned with the query mean must get the largest share
+    q = np.zeros((1, 1, 4, 2)); q[..., 0] = 1.0
+    k = np.zeros((1, 1, 4, 2)); k[0, 0, 2:, 0] = 5.0; k[0, 0, :2, 0] = -5.0
+    _, _, P = osco.score_blocks(q, k, 2)
+    expect = np.exp([-5 / math.sqrt(2), 5 / math.sqrt(2)])
+    expect /= expect.sum()
+    assert np.allclose(P[0, 0, 0], expect, rtol=1e-6)
+
+
+# -------------------------------------------------------------------- top-p
+
+def test_topp_golden_rows():
+    cases = json.load(open(os.path.join(GOLDEN, "topp_cases.json")))["cases"]
+    for c in cases:
+        P = np.array([np.nan if v == "nan" else v for v in c["P"]], dtype=np.float32)
+        kept, k = otop.select_row(P, c["p"])
+        assert kept.tolist() == c["kept"], c["name"]
+        assert k == len(c["kept"])
+
+
+def _brute_force_row(P, p):
+    """Smallest subset reaching T; among equal sizes the ordered top-k."""
+    P = otop.clamp_probs(P)
+    nb = P.size
+    u = [int(math.floor(float(x) * 2 ** 40)) for x in P]
+    U = sum(u)
+    T = math.ceil(float(np.float64(np.float32(p)) * np.float64(U)))
+    if np.float32(p) == 1:
+        return list(range(nb))
+    for size in range(1, nb + 1):
+        best = None
+        for sub in itertools.combinations(range(nb), size):
+            if sum(u[j] for j in sub) >= T:
+                key = sorted(sub, key=lambda j: (-float(P[j]), j))
+                if best is None or [(-float(P[j]), j) for j in key] < [(-float(P[j]), j) for j in best]:
+                    best = key
+        if best is not None:
+            return sorted(best)
+    raise AssertionError("unreachable")
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_topp_matches_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    nb = int(rng.integers(1, 11))
+    z = rng.standard_normal(nb) * rng.uniform(0.2, 3)
+    if seed % 3 == 0:
+        z = np.round(z)  # ties
+    P = (np.exp(z) / np.exp(z).sum()).astype(np.float32)
+    for p in (0.3, 0.5, 0.9, 0.97, 1.0):
+        kept, _ = otop.select_row(P, p)
+        assert kept.tolist() == _brute_force_row(P, p), (P, p)
+
+
+def test_topp_mass_and_minimality_on_random_rows():
+    from block_sparse_attention_logits_b200.synthetic import random_probs
+    P = random_probs(1, 2, 37, seed=5, temperature=2.0)
+    p = np.array([0.9, 0.5], dtype=np.float32)
+    mask, idx, cnt = otop.select_topp_mask(P, p)
+    for h in range(2):
+        for i in range(37):
+            row = otop.clamp_probs(P[0, h, i])
+            u = np.floor(row.astype(np.float64) * 2 ** 40)
+            U = u.sum()
+            T = math.ceil(float(p[h]) * U)
+            kept = idx[0, h, i, :cnt[0, h, i]]
+            assert np.array_equal(np.nonzero(mask[0, h, i])[0], kept)
+            assert u[kept].sum() >= T
+            smallest = kept[np.lexsort((-kept, row[kept]))[0]]  # least P, highest index
+            assert u[kept].sum() - u[smallest] < T
+            # every dropped block is ordered after every kept block
+            dropped = np.setdiff1d(np.arange(37), kept)
+            if dropped.size:
+                worst_kept = min((row[j], -j) for j in kept)
+                best_dropped = max((row[j], -j) for j in dropped)
+                assert best_dropped < worst_kept
+
+
+def test_topp_p_one_and_equal_rows():
+    P = np.full((1, 1, 9, 9), 1 / 9, dtype=np.float32)
+    mask, idx, cnt = otop.select_topp_mask(P, [1.0])
+    assert np.all(mask == 1) and np.all(cnt == 9)
+    P = np.full((1, 1, 8, 8), 0.125, dtype=np.float32)
+    mask, idx, cnt = otop.select_topp_mask(P, [0.5])
+    assert np.all(cnt == 4) and np.all(idx[..., :4] == np.arange(4))
+
+
+def test_topp_fast_equals_loop():
+    from block_sparse_attention_logits_b200.synthetic import random_probs
+    for ties in (False, True):
+        P = random_probs(2, 3, 29, seed=9, temperature=1.5, ties=ties)
+        p = np.array([0.9, 0.35, 1.0], dtype=np.float32)
+        a = otop.select_topp_mask(P, p)
+        b = otop.select_topp_mask_fast(P, p)
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
+
+
+def test_topp_rejects_bad_p():
+    P = np.full((1, 1, 2, 2), 0.5, dtype=np.float32)
+    for bad in (0.0, -0.1, 1.5, float("nan")):
+        with pytest.raises(ValueError):
+            otop.select_topp_mask(P, [bad])
+
+
+# ---------------------------------------------------------------- attention
+
+def _naive_attention(q, k, v):
+    L, D = q.shape
+    O = np.zeros((L, D))
+    lse = np.zeros(L)
+    for r in range(L):
+        s = [sum(q[r, d] * k[c, d] for d in range(D)) / math.sqrt(D) for c in range(L)]
+        m = max(s)
+        z = sum(math.exp(x - m) for x in s)
+        lse[r] = m + math.log(z)
+        for c in range(L):
+            w = math.exp(s[c] - lse[r])
+            for d in range(D):
+                O[r, d] += w * v[c, d]
+    return O, lse
+
+
+def test_keep_all_equals_naive_triple_loop():
+    rng = np.random.default_rng(7)
+    L, D, blk = 11, 4, 4
+    q, k, v = (rng.standard_normal((1, 1, L, D)) for _ in range(3))
+    nb = 3
+    idx = np.tile(np.arange(nb, dtype=np.int32), (1, 1, nb, 1))
+    cnt = np.full((1, 1, nb), nb, dtype=np.int32)
+    O, lse = oatt.masked_attention(q, k, v, idx, cnt, blk)
+    On, lsen = _naive_attention(q[0, 0], k[0, 0], v[0, 0])
+    assert np.allclose(O[0, 0], On, atol=1e-12)
+    assert np.allclose(lse[0, 0], lsen, atol=1e-12)
+
+
+def test_keep_all_equals_torch_sdpa_float64():
+    rng = np.random.default_rng(8)
+    B, H, L, D, blk = 1, 2, 200, 16, 64
+    q, k, v = (rng.standard_normal((B, H, L, D)) for _ in range(3))
+    nb = 4
+    idx = np.tile(np.arange(nb, dtype=np.int32), (B, H, nb, 1))
+    cnt = np.full((B, H, nb), nb, dtype=np.int32)
+    O, lse = oatt.masked_attention(q, k, v, idx, cnt, blk)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v)).numpy()
+    assert np.allclose(O, ref, atol=1e-12)
+    Od, lsed = oatt.dense_attention(q, k, v)
+    assert np.allclose(Od, ref, atol=1e-12) and np.allclose(lsed, lse, atol=1e-12)
+    # LSE against torch.logsumexp of independently formed logits
+    s = torch.from_numpy(q) @ torch.from_numpy(k).transpose(-1, -2) / math.sqrt(D)
+    assert np.allclose(lse, torch.logsumexp(s, dim=-1).numpy(), atol=1e-12)
+
+
+def test_masked_attention_weights_sum_to_one_and_respect_mask():
+    rng = np.random.default_rng(9)
+    B, H, L, D, blk = 1, 1, 150, 8, 32
+    q, k, v = (rng.standard_normal((B, H, L, D)) for _ in range(3))
+    kept = np.array([0, 4])  # 4 is the partial last block (22 tokens)
+    o, lse = oatt.masked_attention_block(q, k, v, kept, blk, 0, 0, 1)
+    cols = np.r_[0:32, 128:150]
+    s = q[0, 0, 32:64] @ k[0, 0, cols].T / math.sqrt(D)
+    w = np.exp(s - lse[:, None])
+    assert np.allclose(w.sum(1), 1, atol=1e-12)
+    assert np.allclose(o, w @ v[0, 0, cols], atol=1e-12)
+    # changing a value in a dropped block changes nothing
+    v2 = v.copy(); v2[0, 0, 40] += 100.0
+    o2, _ = oatt.masked_attention_block(q, k, v2, kept, blk, 0, 0, 1)
+    assert np.array_equal(o, o2)
+
+
+def test_single_block_constant_keys_closed_form():
+    rng = np.random.default_rng(10)
+    B, H, L, D, blk = 1, 1, 100, 8, 32
+    q = rng.standard_normal((B, H, L, D))
+    k = np.tile(rng.standard_normal(D), (B, H, L, 1))
+    v = rng.standard_normal((B, H, L, D))
+    for j, n in ((1, 32), (3, 4)):  # a full block and the partial last block
+        o, lse = oatt.masked_attention_block(q, k, v, [j], blk, 0, 0, 0)
+        expect = q[0, 0, :32] @ k[0, 0, 0] / math.sqrt(D) + math.log(n)
+        assert np.allclose(lse, expect, atol=1e-12)
+        assert np.allclose(o, v[0, 0, j * 32:j * 32 + n].mean(0), atol=1e-12)
+
+
+def test_empty_kept_set():
+    z = np.zeros((1, 1, 4, 2))
+    o, lse = oatt.masked_attention_block(z, z, z, [], 4, 0, 0, 0)
+    assert np.all(o == 0) and np.all(np.isneginf(lse))
+
+
+# --------------------------------------------------------------- correction
+
+def test_bf16_round_matches_torch_cast():
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.standard_normal(5000) * 10 ** rng.uniform(-30, 30, 5000),
+                        [0.0, -0.0, np.inf, -np.inf, 3.3895314e38, 1e-40]]).astype(np.float32)
+    ours = ocor.bf16_round(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(ours.view(np.uint32), ref.view(np.uint32))
+
+
+def test_correction_identities():
+    rng = np.random.default_rng(12)
+    to_bf16 = lambda a: torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).float().numpy()
+    od = to_bf16(rng.standard_normal((1, 3, 40, 8)))
+    osp = to_bf16(od + 0.05 * rng.standard_normal(od.shape))
+    R = ocor.refresh_refinement(od, osp)
+    assert np.allclose(ocor.apply_correction(osp, R, np.zeros(3)), osp)
+    full = ocor.apply_correction(osp, R, np.ones(3))
+    # one bf16 rounding of R: |err| <= half an ulp of |R| (2^-9 relative)
+    assert np.all(np.abs(full - od) <= np.abs(od - osp) * 2.0 ** -8 + 1e-30)
+    half = ocor.apply_correction(osp, R, np.array([0.0, 0.5, 1.0]))
+    assert np.allclose(half[:, 1], osp[:, 1] + 0.5 * R[:, 1])
+    assert np.allclose(half[:, 2], full[:, 2]) and np.allclose(half[:, 0], osp[:, 0])
+
+
+# ------------------------------------------------- planted mistakes are caught
+
+def test_planted_mistake_strict_inequality_is_caught(monkeypatch):
+    def strict(P_row, p):
+        P_row = otop.clamp_probs(P_row)
+        nb = P_row.shape[0]
+        if np.float32(p) == 1:
+            return np.arange(nb, dtype=np.int32), nb
+        order = np.lexsort((np.arange(nb), -P_row.astype(np.float64)))
+        u = otop.fixed_point_mass(P_row)
+        T = int(np.ceil(np.float64(np.float32(p)) * float(u.sum())))
+        csum = np.cumsum(u[order])
+        k = int(np.argmax(csum > T)) + 1  # planted: ">" instead of ">="
+        return np.sort(order[:k]).astype(np.int32), k
+    monkeypatch.setattr(otop, "select_row", strict)
+    with pytest.raises(AssertionError):
+        test_topp_golden_rows()
+
+
+def test_planted_mistake_tie_order_is_caught(monkeypatch):
+    orig = otop.select_row
+
+    def highest_index_first(P_row, p):
+        kept, k = orig(np.asarray(P_row)[::-1].copy(), p)
+        return np.sort(len(P_row) - 1 - kept).astype(np.int32), k
+    monkeypatch.setattr(otop, "select_row", highest_index_first)
+    with pytest.raises(AssertionError):
+        test_topp_golden_rows()
+
+
+def test_planted_mistake_pool_divisor_is_caught(monkeypatch):
+    def full_divisor(x, blk):
+        x = np.asarray(x, dtype=np.float64)
+        B, H, L, D = x.shape
+        nb = (L + blk - 1) // blk
+        out = np.zeros((B, H, nb, D))
+        for i in range(nb):
+            out[:, :, i] = x[:, :, i * blk:(i + 1) * blk].sum(2) / blk  # planted
+        return out.astype(np.float32)
+    monkeypatch.setattr(osco, "pool_blocks", full_divisor)
+    with pytest.raises(AssertionError):
+        test_pool_golden_ramps()
+
+
+def test_planted_mistake_transposed_logits_is_caught(monkeypatch):
+    orig = osco.block_logits
+    monkeypatch.setattr(osco, "block_logits", lambda a, b: np.swapaxes(orig(a, b), -1, -2))
+    with pytest.raises(AssertionError):
+        test_block_probs_prefers_aligned_key()
+
+
+def test_planted_mistake_attention_scale_is_caught(monkeypatch):
+    def no_scale(q_rows, k, v, cols):
+        kc = np.asarray(k, dtype=np.float64)[cols]
+        s = np.asarray(q_rows, dtype=np.float64) @ kc.T  # planted: no 1/sqrt(D)
+        m = s.max(1, keepdims=True)
+        lse = m[:, 0] + np.log(np.exp(s - m).sum(1))
+        return np.exp(s - lse[:, None]) @ np.asarray(v, dtype=np.float64)[cols], lse
+    monkeypatch.setattr(oatt, "attend_rows", no_scale)
+    with pytest.raises(AssertionError):
+        test_keep_all_equals_torch_sdpa_float64()
+
+
+def test_planted_mistake_hilbert_axis_order_is_caught(monkeypatch):
+    orig = ohil.hilbert_index
+    monkeypatch.setattr(ohil, "hilbert_index", lambda c, k: orig(np.asarray(c)[::-1], k))
+    with pytest.raises(AssertionError):
+        test_hilbert_2d_matches_textbook_curve(2)
