@@ -1,0 +1,74 @@
+"""ctypes loader for libbsa.so (the C ABI of include/bsa.h).
+
+There is no fallback: if the in-tree library is missing or fails to load,
+every call raises.  Build it with ``python -m block_sparse_attention_logits_b200.build``.
+"""
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbsa.so")
+
+EXPORTS = (
+    "bsa_strerror", "bsa_version", "bsa_score_blocks", "bsa_select_topp_mask",
+    "bsa_reorder_workspace_bytes", "bsa_reorder_tokens", "bsa_permute_tokens",
+    "bsa_sparse_attn_fwd", "bsa_refresh_refinement", "bsa_apply_correction",
+)
+
+BSA_OK, BSA_EINVAL, BSA_ESHAPE, BSA_ENODEV, BSA_ECUDA, BSA_EWORKSPACE = range(6)
+BSA_DEV_TIMEOUT = 1
+BSA_DEV_BAD_INDEX = 2
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("L", ctypes.c_int),
+                ("D", ctypes.c_int), ("blk", ctypes.c_int)]
+
+
+class BsaError(RuntimeError):
+    def __init__(self, fn, code, msg):
+        super().__init__(f"{fn} failed with status {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+
+def load():
+    """Load libbsa.so once and declare every signature."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libbsa.so not found at {LIB_PATH}; build it with "
+                           "`python -m block_sparse_attention_logits_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "bsa_strerror": (ctypes.c_char_p, [_I]),
+        "bsa_version": (_I, []),
+        "bsa_score_blocks": (_I, [Shape, _P, _P, _P, _P, _P, _P]),
+        "bsa_select_topp_mask": (_I, [Shape, _P, ctypes.POINTER(ctypes.c_float), _P, _P, _P, _P]),
+        "bsa_reorder_workspace_bytes": (_SZ, [_I, _I, _I]),
+        "bsa_reorder_tokens": (_I, [_I, _I, _I, _P, _P, _P, _SZ, _P]),
+        "bsa_permute_tokens": (_I, [Shape, _P, _P, _P, _I, _P]),
+        "bsa_sparse_attn_fwd": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "bsa_refresh_refinement": (_I, [Shape, _P, _P, _P, _P]),
+        "bsa_apply_correction": (_I, [Shape, _P, _P, _P, _P, _P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def check(fn, code):
+    if code != BSA_OK:
+        msg = load().bsa_strerror(code).decode()
+        raise BsaError(fn, code, msg)

@@ -1,0 +1,185 @@
+"""Python binding of libbsa: one function per C-ABI call, same names.
+
+Each function only marshals torch tensors (device memory, the current CUDA
+stream) into the C call and raises on a non-zero status; every step of the
+computation runs in libbsa's kernels.  Outputs are allocated with torch when
+not passed in.  All calls are asynchronous on the current stream.
+"""
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import Shape, check
+
+__all__ = [
+    "score_blocks", "select_topp_mask", "reorder_workspace_bytes", "reorder_tokens",
+    "permute_tokens", "sparse_attn_fwd", "refresh_refinement", "apply_correction",
+    "n_blocks", "version",
+]
+
+
+def n_blocks(L, blk):
+    return (L + blk - 1) // blk
+
+
+def version():
+    return _lib.load().bsa_version()
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    return t
+
+
+def _shape(q, blk):
+    B, H, L, D = q.shape
+    return Shape(B, H, L, D, blk)
+
+
+def score_blocks(q, k, blk, q_pool=None, k_pool=None, probs=None):
+    """Block means of Q and K and the per-query-block softmax of their logits.
+
+    q, k: bf16 [B,H,L,D].  Returns (q_pool, k_pool, probs): float32
+    [B,H,NB,D], [B,H,NB,D], [B,H,NB,NB].
+    """
+    B, H, L, D = q.shape
+    nb = n_blocks(L, blk)
+    _need(q, torch.bfloat16, (B, H, L, D), "q")
+    _need(k, torch.bfloat16, (B, H, L, D), "k")
+    dev = q.device
+    q_pool = q_pool if q_pool is not None else torch.empty((B, H, nb, D), dtype=torch.float32, device=dev)
+    k_pool = k_pool if k_pool is not None else torch.empty((B, H, nb, D), dtype=torch.float32, device=dev)
+    probs = probs if probs is not None else torch.empty((B, H, nb, nb), dtype=torch.float32, device=dev)
+    _need(q_pool, torch.float32, (B, H, nb, D), "q_pool")
+    _need(k_pool, torch.float32, (B, H, nb, D), "k_pool")
+    _need(probs, torch.float32, (B, H, nb, nb), "probs")
+    check("bsa_score_blocks", _lib.load().bsa_score_blocks(
+        _shape(q, blk), _ptr(q), _ptr(k), _ptr(q_pool), _ptr(k_pool), _ptr(probs), _stream()))
+    return q_pool, k_pool, probs
+
+
+def select_topp_mask(probs, p, L, blk, D=128, mask=None, kept_idx=None, kept_cnt=None):
+    """Cumulative top-p selection per query block.
+
+    probs: float32 [B,H,NB,NB]; p: per-head thresholds (sequence of H floats
+    in (0,1]) or one float for every head.  Returns (mask uint8, kept_idx
+    int32, kept_cnt int32).
+    """
+    B, H, nb, _ = probs.shape
+    _need(probs, torch.float32, (B, H, nb, nb), "probs")
+    if isinstance(p, (int, float)):
+        p = [float(p)] * H
+    p = [float(x) for x in p]
+    if len(p) != H:
+        raise ValueError("p must have one value per head")
+    dev = probs.device
+    mask = mask if mask is not None else torch.empty((B, H, nb, nb), dtype=torch.uint8, device=dev)
+    kept_idx = kept_idx if kept_idx is not None else torch.empty((B, H, nb, nb), dtype=torch.int32, device=dev)
+    kept_cnt = kept_cnt if kept_cnt is not None else torch.empty((B, H, nb), dtype=torch.int32, device=dev)
+    _need(mask, torch.uint8, (B, H, nb, nb), "mask")
+    _need(kept_idx, torch.int32, (B, H, nb, nb), "kept_idx")
+    _need(kept_cnt, torch.int32, (B, H, nb), "kept_cnt")
+    parr = (ctypes.c_float * H)(*p)
+    check("bsa_select_topp_mask", _lib.load().bsa_select_topp_mask(
+        Shape(B, H, L, D, blk), _ptr(probs), parr, _ptr(mask), _ptr(kept_idx), _ptr(kept_cnt), _stream()))
+    return mask, kept_idx, kept_cnt
+
+
+def reorder_workspace_bytes(T, Hh, W):
+    return int(_lib.load().bsa_reorder_workspace_bytes(T, Hh, W))
+
+
+def reorder_tokens(T, Hh, W, device="cuda", perm=None, inv=None, workspace=None):
+    """Hilbert-curve order of a (T, Hh, W) latent grid: (perm, inv) int32 [L]."""
+    L = T * Hh * W
+    perm = perm if perm is not None else torch.empty(L, dtype=torch.int32, device=device)
+    inv = inv if inv is not None else torch.empty(L, dtype=torch.int32, device=device)
+    nbytes = reorder_workspace_bytes(T, Hh, W)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=perm.device)
+    check("bsa_reorder_tokens", _lib.load().bsa_reorder_tokens(
+        T, Hh, W, _ptr(perm), _ptr(inv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream()))
+    return perm, inv
+
+
+def permute_tokens(x, perm, inverse=False, out=None):
+    """Gather rows into curve order (inverse=False) or scatter them back."""
+    B, H, L, D = x.shape
+    _need(x, torch.bfloat16, (B, H, L, D), "x")
+    _need(perm, torch.int32, (L,), "perm")
+    out = out if out is not None else torch.empty_like(x)
+    _need(out, torch.bfloat16, (B, H, L, D), "out")
+    check("bsa_permute_tokens", _lib.load().bsa_permute_tokens(
+        Shape(B, H, L, D, 0), _ptr(x), _ptr(perm), _ptr(out), 1 if inverse else 0, _stream()))
+    return out
+
+
+def sparse_attn_fwd(q, k, v, blk, kept_idx=None, kept_cnt=None, R=None, alpha=None,
+                    o=None, lse=None, status=None):
+    """Block-sparse attention over the kept blocks (dense when kept_* are None).
+
+    Returns (o bf16 [B,H,L,D], lse float32 [B,H,L]).  With R / alpha the
+    epilogue adds alpha_h * R.  `status` (int32 [1] on the device, zeroed by
+    the caller) receives BSA_DEV_* bits.
+    """
+    B, H, L, D = q.shape
+    nb = n_blocks(L, blk)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, torch.bfloat16, (B, H, L, D), name)
+    if kept_idx is not None:
+        _need(kept_idx, torch.int32, (B, H, nb, nb), "kept_idx")
+        _need(kept_cnt, torch.int32, (B, H, nb), "kept_cnt")
+    if R is not None:
+        _need(R, torch.bfloat16, (B, H, L, D), "R")
+        _need(alpha, torch.float32, (H,), "alpha")
+    o = o if o is not None else torch.empty_like(q)
+    lse = lse if lse is not None else torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    _need(o, torch.bfloat16, (B, H, L, D), "o")
+    _need(lse, torch.float32, (B, H, L), "lse")
+    check("bsa_sparse_attn_fwd", _lib.load().bsa_sparse_attn_fwd(
+        Shape(B, H, L, D, blk), _ptr(q), _ptr(k), _ptr(v), _ptr(kept_idx), _ptr(kept_cnt),
+        _ptr(R), _ptr(alpha), _ptr(o), _ptr(lse), _ptr(status), _stream()))
+    return o, lse
+
+
+def refresh_refinement(o_dense, o_sparse, out=None):
+    """R = bf16(o_dense - o_sparse)."""
+    B, H, L, D = o_dense.shape
+    _need(o_dense, torch.bfloat16, (B, H, L, D), "o_dense")
+    _need(o_sparse, torch.bfloat16, (B, H, L, D), "o_sparse")
+    out = out if out is not None else torch.empty_like(o_dense)
+    check("bsa_refresh_refinement", _lib.load().bsa_refresh_refinement(
+        Shape(B, H, L, D, 0), _ptr(o_dense), _ptr(o_sparse), _ptr(out), _stream()))
+    return out
+
+
+def apply_correction(o_sparse, R, alpha, out=None):
+    """o = bf16(o_sparse + alpha_h * R)."""
+    B, H, L, D = o_sparse.shape
+    _need(o_sparse, torch.bfloat16, (B, H, L, D), "o_sparse")
+    _need(R, torch.bfloat16, (B, H, L, D), "R")
+    _need(alpha, torch.float32, (H,), "alpha")
+    out = out if out is not None else torch.empty_like(o_sparse)
+    check("bsa_apply_correction", _lib.load().bsa_apply_correction(
+        Shape(B, H, L, D, 0), _ptr(o_sparse), _ptr(R), _ptr(alpha), _ptr(out), _stream()))
+    return out

@@ -1,0 +1,169 @@
+// extern "C" entry points of libbsa (declared in include/bsa.h): host-side
+// argument validation, then one or two kernel launches on the caller's
+// stream.  Nothing here allocates, frees or synchronises.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "internal.cuh"
+
+namespace {
+
+using bsa::n_blocks;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ENODEV;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return BSA_ENODEV;
+  return major == 10 ? BSA_OK : BSA_ENODEV;
+}
+
+// Shape rules shared by the block-level calls.
+int check_block_shape(const bsa_shape& s) {
+  if (s.B < 1 || s.H < 1 || s.L < 1) return BSA_ESHAPE;
+  if (s.D != 64 && s.D != 128) return BSA_ESHAPE;
+  if (s.blk != 64 && s.blk != 128) return BSA_ESHAPE;
+  if (n_blocks(s.L, s.blk) > bsa::kMaxNB) return BSA_ESHAPE;
+  if (static_cast<long long>(s.B) * s.H > 65535) return BSA_ESHAPE;
+  const double elems = static_cast<double>(s.B) * s.H * s.L * s.D;
+  if (elems >= 1099511627776.0) return BSA_ESHAPE;  // 2^40
+  return BSA_OK;
+}
+
+// Shape rules of the elementwise calls (any D that is a multiple of 8).
+int check_rows_shape(const bsa_shape& s) {
+  if (s.B < 1 || s.H < 1 || s.L < 1 || s.D < 8 || (s.D % 8) != 0) return BSA_ESHAPE;
+  const double elems = static_cast<double>(s.B) * s.H * s.L * s.D;
+  if (elems >= 1099511627776.0) return BSA_ESHAPE;
+  return BSA_OK;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ECUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* bsa_strerror(int status) {
+  switch (status) {
+    case BSA_OK: return "ok";
+    case BSA_EINVAL: return "invalid argument (null or misaligned pointer, or value out of range)";
+    case BSA_ESHAPE: return "unsupported or inconsistent shape";
+    case BSA_ENODEV: return "no sm_100 CUDA device is current";
+    case BSA_ECUDA: return "CUDA launch or driver call failed";
+    case BSA_EWORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int bsa_version(void) { return 10000; }
+
+int bsa_score_blocks(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, float* q_pool, float* k_pool, float* probs,
+                     bsa_stream stream) {
+  if (!q || !k || !q_pool || !k_pool || !probs) return BSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool) || !aligned16(probs))
+    return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (int r = check_device()) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const auto* qb = reinterpret_cast<const __nv_bfloat16*>(q);
+  const auto* kb = reinterpret_cast<const __nv_bfloat16*>(k);
+  if (cudaError_t e = bsa::launch_pool(s, qb, kb, q_pool, k_pool, st)) return from_cuda(e);
+  return from_cuda(bsa::launch_block_softmax(s, q_pool, k_pool, probs, st));
+}
+
+int bsa_select_topp_mask(bsa_shape s, const float* probs, const float* p_host, uint8_t* mask, int32_t* kept_idx,
+                         int32_t* kept_cnt, bsa_stream stream) {
+  if (!probs || !p_host || !mask || !kept_idx || !kept_cnt) return BSA_EINVAL;
+  if (!aligned16(probs) || !aligned16(mask) || !aligned16(kept_idx) || !aligned16(kept_cnt)) return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (s.H > bsa::kMaxHeadsP) return BSA_ESHAPE;
+  bsa::TopP tp;
+  for (int h = 0; h < bsa::kMaxHeadsP; ++h) tp.p[h] = 1.0f;
+  for (int h = 0; h < s.H; ++h) {
+    const float p = p_host[h];
+    if (!(p > 0.0f) || !(p <= 1.0f)) return BSA_EINVAL;  // rejects NaN too
+    tp.p[h] = p;
+  }
+  if (int r = check_device()) return r;
+  return from_cuda(bsa::launch_select(s, probs, tp, mask, kept_idx, kept_cnt, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t bsa_reorder_workspace_bytes(int T, int Hh, int W) { return bsa::hilbert_workspace_bytes(T, Hh, W); }
+
+int bsa_reorder_tokens(int T, int Hh, int W, int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes,
+                       bsa_stream stream) {
+  if (!perm || !inv) return BSA_EINVAL;
+  const size_t need = bsa::hilbert_workspace_bytes(T, Hh, W);
+  if (need == 0) return BSA_ESHAPE;
+  if (!ws || ws_bytes < need) return BSA_EWORKSPACE;
+  if (!aligned16(perm) || !aligned16(inv) || !aligned16(ws)) return BSA_EINVAL;
+  if (int r = check_device()) return r;
+  return from_cuda(bsa::launch_hilbert(T, Hh, W, perm, inv, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int bsa_permute_tokens(bsa_shape s, const bsa_bf16* x, const int32_t* perm, bsa_bf16* y, int inverse,
+                       bsa_stream stream) {
+  if (!x || !perm || !y) return BSA_EINVAL;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(perm)) return BSA_EINVAL;
+  if (x == y) return BSA_EINVAL;
+  if (int r = check_rows_shape(s)) return r;
+  if (int r = check_device()) return r;
+  return from_cuda(bsa::launch_permute(s, reinterpret_cast<const __nv_bfloat16*>(x), perm,
+                                       reinterpret_cast<__nv_bfloat16*>(y), inverse,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int bsa_sparse_attn_fwd(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v, const int32_t* kept_idx,
+                        const int32_t* kept_cnt, const bsa_bf16* R, const float* alpha, bsa_bf16* o, float* lse,
+                        int32_t* status, bsa_stream stream) {
+  if (!q || !k || !v || !o || !lse) return BSA_EINVAL;
+  if ((kept_idx == nullptr) != (kept_cnt == nullptr)) return BSA_EINVAL;
+  if ((R == nullptr) != (alpha == nullptr)) return BSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return BSA_EINVAL;
+  if ((kept_idx && !aligned16(kept_idx)) || (kept_cnt && !aligned16(kept_cnt)) || (R && !aligned16(R)))
+    return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (int r = check_device()) return r;
+  bsa::AttnArgs a;
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  a.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  a.kept_idx = kept_idx;
+  a.kept_cnt = kept_cnt;
+  a.R = reinterpret_cast<const __nv_bfloat16*>(R);
+  a.alpha = alpha;
+  a.o = reinterpret_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.status = status;
+  return bsa::launch_sparse_attn(s, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bsa_refresh_refinement(bsa_shape s, const bsa_bf16* o_dense, const bsa_bf16* o_sparse, bsa_bf16* R,
+                           bsa_stream stream) {
+  if (!o_dense || !o_sparse || !R) return BSA_EINVAL;
+  if (!aligned16(o_dense) || !aligned16(o_sparse) || !aligned16(R)) return BSA_EINVAL;
+  if (int r = check_rows_shape(s)) return r;
+  if (int r = check_device()) return r;
+  const size_t n = static_cast<size_t>(s.B) * s.H * s.L * s.D;
+  return from_cuda(bsa::launch_refresh(n, reinterpret_cast<const __nv_bfloat16*>(o_dense),
+                                       reinterpret_cast<const __nv_bfloat16*>(o_sparse),
+                                       reinterpret_cast<__nv_bfloat16*>(R), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int bsa_apply_correction(bsa_shape s, const bsa_bf16* o_sparse, const bsa_bf16* R, const float* alpha, bsa_bf16* o,
+                         bsa_stream stream) {
+  if (!o_sparse || !R || !alpha || !o) return BSA_EINVAL;
+  if (!aligned16(o_sparse) || !aligned16(R) || !aligned16(o)) return BSA_EINVAL;
+  if (int r = check_rows_shape(s)) return r;
+  if (int r = check_device()) return r;
+  return from_cuda(bsa::launch_correct(s, reinterpret_cast<const __nv_bfloat16*>(o_sparse),
+                                       reinterpret_cast<const __nv_bfloat16*>(R), alpha,
+                                       reinterpret_cast<__nv_bfloat16*>(o), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,593 @@
+// Block-sparse attention forward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// What it computes (CalibAtt abstract and Fig. 5(b): compute the selected
+// block connections exactly and skip the unselected ones; RECAP section 4.1:
+// block-sparse attention for the selected interactions, dense attention for
+// refreshes; RECAP section 1: a cached dense refinement corrects the sparse
+// output): for every query row r of query block i,
+//     O[r] = softmax over the keys of the kept blocks K(i) of (q_r.k_c/sqrt(D)) . V
+//     LSE[r] = log-sum-exp of those logits,
+// optionally followed by O <- O + alpha_h * R in the epilogue.
+//
+// Work decomposition.  A CTA owns a PAIR of 128-row query tiles of one
+// (batch, head).  The two tiles usually keep overlapping key blocks (their
+// queries are neighbours in token order), so the CTA walks the UNION of the
+// kept lists of its query blocks in ascending key-block order and loads each
+// K/V block once for both tiles; each tile only computes the blocks it keeps.
+// With blk = 64 one 128-row tile spans two query blocks; rows of the half that
+// does not keep a block are masked to -inf for that block.
+//
+// Warp roles (12 warps):
+//   warp 0      TMA producer: Q tiles once, then K/V of every union entry into
+//               an NS-deep ring (128-byte swizzled panels of 64 columns).
+//   warp 1      MMA issuer (one thread): S_t = Q_t K^T (SS form, both operands
+//               in shared memory) into TMEM, then O_t += P_t V with P_t read
+//               from TMEM (TS form).  It serves the two tiles from a polling
+//               state machine so neither tile can block the other.
+//   warp 2      TMEM allocation / release.
+//   warps 4-7   softmax + epilogue of tile 0 (one thread per query row).
+//   warps 8-11  softmax + epilogue of tile 1.
+// TMEM columns: S0 | S1 | O0 | O1.  P_t (bf16, packed in pairs) overwrites the
+// first BN/2 columns of S_t once S_t has been read.
+//
+// Online softmax in the log2 domain in fp32.  The running max used for the
+// exponentials is only raised when the block max exceeds it by more than 8
+// (so P <= 2^8); O in TMEM is rescaled only then, and the final 1/l uses the
+// same reference, so the result is exact up to rounding.
+//
+// Every wait is bounded (2 s of globaltimer); a timeout sets BSA_DEV_TIMEOUT
+// in the caller's status word, aborts the CTA's pipeline, drains what is in
+// flight and releases TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstdio>
+
+#include "internal.cuh"
+#include "sm100.cuh"
+
+namespace bsa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 384;
+constexpr int BM = 128;                        // query rows per tile
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
+constexpr float kRescaleThreshold = 8.0f;      // log2 units
+
+struct Params {
+  const int32_t* kept_idx;
+  const int32_t* kept_cnt;
+  const __nv_bfloat16* R;
+  const float* alpha;
+  __nv_bfloat16* o;
+  float* lse;
+  int32_t* status;
+  int H, L, NB;
+  float scale_log2;
+  int dense;
+};
+
+template <int D, int BN>
+struct Cfg {
+  static constexpr int G = BM / BN;              // query blocks per 128-row tile
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+  static constexpr int UNION_BYTES = kMaxNB * 2;  // uint16 per union entry
+  static constexpr int BITMAP_BYTES = kMaxNB;     // one byte of membership bits per key block
+  static constexpr int MISC_BYTES = 256;          // barriers and scalars
+  static constexpr int FIXED = 2 * Q_BYTES + UNION_BYTES + BITMAP_BYTES + MISC_BYTES;
+  static constexpr int NS_FIT = (227 * 1024 - 1024 - FIXED) / STAGE_BYTES;
+  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+  static_assert(NS >= 2, "shared memory too small for a double-buffered K/V ring");
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_STAGE = 2 * Q_BYTES;
+  static constexpr int OFF_UNION = OFF_STAGE + NS * STAGE_BYTES;
+  static constexpr int OFF_BITMAP = OFF_UNION + UNION_BYTES;
+  static constexpr int OFF_MISC = OFF_BITMAP + BITMAP_BYTES;
+  static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+  static constexpr int COL_S0 = 0, COL_S1 = BN, COL_O0 = 2 * BN, COL_O1 = 2 * BN + D;
+  static constexpr int TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256 : 512;
+  static constexpr int PANELS = D / 64;
+};
+
+struct Shared {
+  // laid out in the MISC region
+  uint64_t full[4];
+  uint64_t empty[4];
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t n_union;
+  uint32_t n_tile[2];
+  volatile int abort_flag;
+};
+static_assert(sizeof(Shared) <= 256, "misc region too small");
+
+__device__ __forceinline__ void flag_status(const Params& prm, int bits) {
+  if (prm.status) atomicOr(prm.status, bits);
+}
+
+// Bounded blocking wait.  Returns false on timeout or when another role has
+// already aborted the CTA.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Shared* sh, const Params& prm) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 15) == 0) {
+      if (sh->abort_flag) return false;
+      if (globaltimer_ns() - t0 > kTimeoutNs) {
+        sh->abort_flag = 1;
+        flag_status(prm, BSA_DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ int next_member(const uint16_t* ulist, int i, int U, uint32_t tile_mask) {
+  while (i < U && ((ulist[i] >> 12) & tile_mask) == 0) ++i;
+  return i;
+}
+
+template <int D, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const Params prm) {
+  using C = Cfg<D, BN>;
+  constexpr int G = C::G;
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint16_t* ulist = reinterpret_cast<uint16_t*>(smem + C::OFF_UNION);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + C::OFF_BITMAP);
+  Shared* sh = reinterpret_cast<Shared*>(smem + C::OFF_MISC);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int pair = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int NB = prm.NB;
+  const int L = prm.L;
+
+  // ---------------------------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->empty[s], 1);
+    }
+    mbar_init(&sh->q_full, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&sh->s_full[t], 1);
+      mbar_init(&sh->p_full[t], 128);
+      mbar_init(&sh->o_full[t], 1);
+    }
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 2) {
+    tmem_alloc(&sh->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  for (int i = threadIdx.x; i < (NB + 3) / 4; i += kThreads) bitmap[i] = 0u;
+  __syncthreads();
+
+  // Membership bits: bit `sub` of key block kb is set when query block
+  // pair*2G + sub keeps kb.
+  for (int sub = 0; sub < 2 * G; ++sub) {
+    const int qb = pair * 2 * G + sub;
+    if (qb >= NB) break;
+    int cnt = NB;
+    const int32_t* row = nullptr;
+    if (!prm.dense) {
+      const size_t r = static_cast<size_t>(bh) * NB + qb;
+      cnt = prm.kept_cnt[r];
+      if (cnt < 0 || cnt > NB) {
+        if (threadIdx.x == 0) flag_status(prm, BSA_DEV_BAD_INDEX);
+        cnt = cnt < 0 ? 0 : NB;
+      }
+      row = prm.kept_idx + r * NB;
+    }
+    for (int n = threadIdx.x; n < cnt; n += kThreads) {
+      const int kb = prm.dense ? n : row[n];
+      if (static_cast<unsigned>(kb) >= static_cast<unsigned>(NB)) {
+        flag_status(prm, BSA_DEV_BAD_INDEX);
+        continue;
+      }
+      atomicOr(&bitmap[kb >> 2], (1u << sub) << ((kb & 3) * 8));
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t m0 = (1u << G) - 1u, m1 = m0 << G;
+    uint32_t U = 0, c0 = 0, c1 = 0;
+    for (int base = 0; base < NB; base += 32) {
+      const int kb = base + lane;
+      const uint32_t m = kb < NB ? (bitmap[kb >> 2] >> ((kb & 3) * 8)) & 0xFu : 0u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, m != 0);
+      if (m) ulist[U + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(kb | (m << 12));
+      U += __popc(bal);
+      c0 += __popc(__ballot_sync(0xffffffffu, (m & m0) != 0));
+      c1 += __popc(__ballot_sync(0xffffffffu, (m & m1) != 0));
+    }
+    if (lane == 0) {
+      sh->n_union = U;
+      sh->n_tile[0] = c0;
+      sh->n_tile[1] = c1;
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  const int U = static_cast<int>(sh->n_union);
+  const int ntile[2] = {static_cast<int>(sh->n_tile[0]), static_cast<int>(sh->n_tile[1])};
+  const uint32_t tile_mask[2] = {(1u << G) - 1u, ((1u << G) - 1u) << G};
+  uint8_t* q_smem = smem + C::OFF_Q;
+  uint8_t* stage_smem = smem + C::OFF_STAGE;
+
+  if (warp == 0) {
+    // --------------------------------------------------------- TMA producer
+    if (lane == 0 && U > 0) {
+      int tiles_here = 0;
+      for (int t = 0; t < 2; ++t)
+        if ((pair * 2 + t) * BM < L) ++tiles_here;
+      mbar_arrive_expect_tx(&sh->q_full, tiles_here * C::Q_BYTES);
+      for (int t = 0; t < 2; ++t) {
+        const int row0 = (pair * 2 + t) * BM;
+        if (row0 >= L) continue;
+        for (int pnl = 0; pnl < C::PANELS; ++pnl)
+          tma_load_3d(q_smem + t * C::Q_BYTES + pnl * BM * 128, &tmQ, &sh->q_full, pnl * 64, row0, bh);
+      }
+      int issued = 0;
+      for (int u = 0; u < U; ++u) {
+        const int slot = u % NS;
+        if (u >= NS && !wait_bounded(&sh->empty[slot], ((u / NS) - 1) & 1, sh, prm)) break;
+        const int kb = ulist[u] & 0xFFF;
+        uint8_t* st = stage_smem + slot * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(&sh->full[slot], 2 * C::KV_BYTES);
+        for (int pnl = 0; pnl < C::PANELS; ++pnl) {
+          tma_load_3d(st + pnl * BN * 128, &tmK, &sh->full[slot], pnl * 64, kb * BN, bh);
+          tma_load_3d(st + C::KV_BYTES + pnl * BN * 128, &tmV, &sh->full[slot], pnl * 64, kb * BN, bh);
+        }
+        issued = u + 1;
+      }
+      if (sh->abort_flag) {
+        // drain: wait (bounded) for the loads of the last NS issues to land
+        for (int u = issued - NS < 0 ? 0 : issued - NS; u < issued; ++u) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try(&sh->full[u % NS], (u / NS) & 1) && globaltimer_ns() - t0 < kTimeoutNs / 4) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issuer
+    if (lane == 0 && U > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(BM, D, false, true);
+      const uint32_t colS[2] = {C::COL_S0, C::COL_S1};
+      const uint32_t colO[2] = {C::COL_O0, C::COL_O1};
+      bool ok = wait_bounded(&sh->q_full, 0, sh, prm);
+      tc_fence_after();
+      enum { NEED_S = 0, NEED_P = 1, DONE = 2 };
+      int st[2], cur[2], n[2];
+      for (int t = 0; t < 2; ++t) {
+        n[t] = 0;
+        cur[t] = next_member(ulist, 0, U, tile_mask[t]);
+        st[t] = (ntile[t] > 0) ? NEED_S : DONE;
+      }
+      const uint32_t q_base = smem_u32(q_smem);
+      const uint32_t stage_base = smem_u32(stage_smem);
+      uint64_t t_idle = 0;
+      uint32_t spins = 0;
+      while (ok && (st[0] != DONE || st[1] != DONE)) {
+        bool progress = false;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (st[t] == NEED_S) {
+            const int u = cur[t];
+            const int slot = u % NS;
+            if (mbar_test(&sh->full[slot], (u / NS) & 1)) {
+              tc_fence_after();
+              const uint32_t qa = q_base + t * C::Q_BYTES;
+              const uint32_t ka = stage_base + slot * C::STAGE_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off_q = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+                mma_ss(tmem + colS[t], sdesc_sw128(qa + off_q, 16, 1024), sdesc_sw128(ka + off_k, 16, 1024), idS,
+                       kk > 0 ? 1u : 0u);
+              }
+              tc_commit(&sh->s_full[t]);
+              st[t] = NEED_P;
+              progress = true;
+            }
+          }
+          if (st[t] == NEED_P) {
+            if (mbar_test(&sh->p_full[t], n[t] & 1)) {
+              tc_fence_after();
+              const int u = cur[t];
+              const int slot = u % NS;
+              const uint32_t va = stage_base + slot * C::STAGE_BYTES + C::KV_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < BN / 16; ++kk) {
+                mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, sdesc_sw128(va + kk * 2048, BN * 128, 1024), idPV,
+                       (n[t] > 0 || kk > 0) ? 1u : 0u);
+              }
+              const int o = 1 - t;
+              const bool other_member = ((ulist[u] >> 12) & tile_mask[o]) != 0;
+              if (!other_member || st[o] == DONE || cur[o] > u) tc_commit(&sh->empty[slot]);
+              ++n[t];
+              cur[t] = next_member(ulist, u + 1, U, tile_mask[t]);
+              if (n[t] == ntile[t]) {
+                tc_commit(&sh->o_full[t]);
+                st[t] = DONE;
+              } else {
+                st[t] = NEED_S;
+              }
+              progress = true;
+            }
+          }
+        }
+        if (progress) {
+          spins = 0;
+          t_idle = 0;
+        } else if ((++spins & 63) == 0) {
+          const uint64_t now = globaltimer_ns();
+          if (t_idle == 0) t_idle = now;
+          if (sh->abort_flag) ok = false;
+          if (now - t_idle > kTimeoutNs) {
+            sh->abort_flag = 1;
+            flag_status(prm, BSA_DEV_TIMEOUT);
+            ok = false;
+          }
+        }
+      }
+      if (!ok) {
+        // make sure no MMA is still writing TMEM before it is released
+        tc_commit(&sh->drain);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try(&sh->drain, 0) && globaltimer_ns() - t0 < kTimeoutNs / 4) {
+        }
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------ softmax + epilogue
+    const int t = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (t == 0 ? C::COL_S0 : C::COL_S1);
+    const uint32_t tO = tmem + lane_off + (t == 0 ? C::COL_O0 : C::COL_O1);
+    const int grow = (pair * 2 + t) * BM + r;
+    const uint32_t my_bit = 1u << (t * G + r / BN);
+    const float sl2 = prm.scale_log2;
+    float m_ref = -INFINITY;
+    float l = 0.f;
+    bool ok = true;
+    int u = next_member(ulist, 0, U, tile_mask[t]);
+    for (int n = 0; n < ntile[t]; ++n) {
+      const uint32_t e = ulist[u];
+      const int kb = e & 0xFFF;
+      const bool row_ok = ((e >> 12) & my_bit) != 0;
+      const int valid = (kb == NB - 1) ? (L - kb * BN) : BN;
+      ok = wait_bounded(&sh->s_full[t], n & 1, sh, prm);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t regs[32];
+        tmem_ld32(tS + c * 32, regs);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(regs[i]);
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < BN; ++j) {
+        float x = s[j] * sl2;
+        if (!row_ok || j >= valid) x = -INFINITY;
+        s[j] = x;
+        mx = fmaxf(mx, x);
+      }
+      const float m_new = fmaxf(m_ref, mx);
+      const bool resc = m_new > m_ref + kRescaleThreshold;
+      float factor = 1.f;
+      if (resc) {
+        factor = ex2_approx(m_ref - m_new);  // 0 when m_ref is -inf
+        l *= factor;
+        m_ref = m_new;
+      }
+      if (n > 0 && __any_sync(0xffffffffu, resc)) {
+        // O of this tile is final for block n-1: s_full of block n is
+        // committed after the PV MMA of block n-1.
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t regs[32];
+          tmem_ld32(tO + c * 32, regs);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) regs[i] = __float_as_uint(__uint_as_float(regs[i]) * factor);
+          tmem_st32(tO + c * 32, regs);
+        }
+        tmem_wait_st();
+      }
+      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < BN / 64; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2_approx(s[c * 64 + 2 * i] - mu);
+          const float p1 = ex2_approx(s[c * 64 + 2 * i + 1] - mu);
+          rs += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + c * 32, pk);
+      }
+      l += rs;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sh->p_full[t]);
+      u = next_member(ulist, u + 1, U, tile_mask[t]);
+    }
+    // ----------------------------------------------------------- epilogue
+    bool have_o = ok && ntile[t] > 0;
+    if (have_o) {
+      have_o = wait_bounded(&sh->o_full[t], 0, sh, prm);
+      have_o = __all_sync(0xffffffffu, have_o);
+      tc_fence_after();
+    }
+    if (ok) {
+      const bool store = grow < L;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float lse_v = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const size_t row_elem = (static_cast<size_t>(bh) * L + (store ? grow : 0)) * D;
+      const int h = bh % prm.H;
+      const float a = prm.R ? prm.alpha[h] : 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t regs[32];
+        if (have_o) {
+          tmem_ld32(tO + c * 32, regs);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) regs[i] = 0u;
+        }
+        if (store) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(regs[i]) * inv_l;
+          if (prm.R) {
+            const uint4* rp = reinterpret_cast<const uint4*>(prm.R + row_elem + c * 32);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const uint4 rv = __ldg(rp + w);
+              const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                v[w * 8 + 2 * i] += a * __uint_as_float(rw[i] << 16);
+                v[w * 8 + 2 * i + 1] += a * __uint_as_float(rw[i] & 0xFFFF0000u);
+              }
+            }
+          }
+          uint4* op = reinterpret_cast<uint4*>(prm.o + row_elem + c * 32);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            uint4 ov;
+            ov.x = pack_bf16x2(v[w * 8 + 0], v[w * 8 + 1]);
+            ov.y = pack_bf16x2(v[w * 8 + 2], v[w * 8 + 3]);
+            ov.z = pack_bf16x2(v[w * 8 + 4], v[w * 8 + 5]);
+            ov.w = pack_bf16x2(v[w * 8 + 6], v[w * 8 + 7]);
+            op[w] = ov;
+          }
+        }
+      }
+      if (store) prm.lse[static_cast<size_t>(bh) * L + grow] = lse_v;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [BH, L, D] bf16 viewed as a 3-D tensor; box = 64 columns x rows x 1.
+bool make_map(CUtensorMap* m, const void* base, int D, int L, int BH, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int BN>
+int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
+  using C = Cfg<D, BN>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(sparse_attn_kernel<D, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return BSA_ECUDA;
+    configured = true;
+  }
+  const int BH = s.B * s.H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, D, s.L, BH, BM) || !make_map(&mk, a.k, D, s.L, BH, BN) ||
+      !make_map(&mv, a.v, D, s.L, BH, BN))
+    return BSA_ECUDA;
+  Params prm;
+  prm.kept_idx = a.kept_idx;
+  prm.kept_cnt = a.kept_cnt;
+  prm.R = a.R;
+  prm.alpha = a.alpha;
+  prm.o = a.o;
+  prm.lse = a.lse;
+  prm.status = a.status;
+  prm.H = s.H;
+  prm.L = s.L;
+  prm.NB = n_blocks(s.L, s.blk);
+  prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  prm.dense = a.kept_idx == nullptr;
+  const int n_tiles = (s.L + BM - 1) / BM;
+  dim3 grid((n_tiles + 1) / 2, BH);
+  sparse_attn_kernel<D, BN><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ECUDA;
+}
+
+}  // namespace
+
+int launch_sparse_attn(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
+  if (s.D == 128 && s.blk == 128) return run<128, 128>(s, a, st);
+  if (s.D == 128 && s.blk == 64) return run<128, 64>(s, a, st);
+  if (s.D == 64 && s.blk == 128) return run<64, 128>(s, a, st);
+  if (s.D == 64 && s.blk == 64) return run<64, 64>(s, a, st);
+  return BSA_ESHAPE;
+}
+
+}  // namespace bsa

@@ -1,0 +1,53 @@
+// Private declarations shared by the libbsa translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/bsa.h"
+
+namespace bsa {
+
+constexpr int kMaxNB = 4096;     // key/query blocks per sequence
+constexpr int kMaxHeadsP = 512;  // heads whose top-p threshold travels as a kernel argument
+
+struct TopP {
+  float p[kMaxHeadsP];
+};
+
+inline int n_blocks(int L, int blk) { return (L + blk - 1) / blk; }
+
+// launchers (return cudaSuccess or the launch error)
+cudaError_t launch_pool(const bsa_shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, float* qp, float* kp,
+                        cudaStream_t st);
+cudaError_t launch_block_softmax(const bsa_shape& s, const float* qp, const float* kp, float* probs,
+                                 cudaStream_t st);
+cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p, uint8_t* mask, int32_t* idx,
+                          int32_t* cnt, cudaStream_t st);
+size_t hilbert_workspace_bytes(int T, int Hh, int W);
+cudaError_t launch_hilbert(int T, int Hh, int W, int32_t* perm, int32_t* inv, void* ws, cudaStream_t st);
+cudaError_t launch_permute(const bsa_shape& s, const __nv_bfloat16* x, const int32_t* perm, __nv_bfloat16* y,
+                           int inverse, cudaStream_t st);
+cudaError_t launch_refresh(size_t n, const __nv_bfloat16* od, const __nv_bfloat16* os, __nv_bfloat16* R,
+                           cudaStream_t st);
+cudaError_t launch_correct(const bsa_shape& s, const __nv_bfloat16* os, const __nv_bfloat16* R, const float* alpha,
+                           __nv_bfloat16* o, cudaStream_t st);
+
+struct AttnArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const int32_t* kept_idx;
+  const int32_t* kept_cnt;
+  const __nv_bfloat16* R;
+  const float* alpha;
+  __nv_bfloat16* o;
+  float* lse;
+  int32_t* status;
+};
+// Returns BSA_OK / BSA_ECUDA (tensor-map encoding or launch failure).
+int launch_sparse_attn(const bsa_shape& s, const AttnArgs& a, cudaStream_t st);
+
+}  // namespace bsa

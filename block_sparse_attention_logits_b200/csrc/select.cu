@@ -1,0 +1,176 @@
+// Cumulative top-p block selection (head-wise top-p abstract: per-head top-p
+// thresholds; GSRS abstract: top-p selection for adaptive sparsity; CalibAtt
+// Fig. 5: threshold the top key blocks per query block).
+//
+// Per row: key_j = float32 bits of clamp(P_j, 0, 1) (order-preserving for
+// non-negative floats), u_j = floor(P_j * 2^40) computed exactly from the
+// exponent and mantissa, T = ceil(p * sum u) in IEEE double.  The kept set is
+// the shortest prefix of the (P desc, index asc) order whose u-sum is >= T.
+//
+// No sort is needed.  One warp per row finds, by a 31-step bitwise search,
+// the largest key threshold tau with  sum_{key >= tau} u >= T.  Every block
+// with key > tau is kept; blocks with key == tau are kept in ascending index
+// order while the running mass is still below T (a warp prefix scan).  All
+// sums are exact uint64 integer sums, so the result does not depend on the
+// order of summation and equals the sequential definition bit for bit.
+#include "internal.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr uint32_t kSelected = 0xFFFFFFFFu;  // marker: above every real key
+
+__device__ __forceinline__ uint32_t prob_key(float p) {
+  // NaN and p <= 0 (incl. -0) -> 0; p > 1 (incl. inf) -> bits of 1.0f
+  if (!(p > 0.f)) return 0u;
+  if (p > 1.f) p = 1.f;
+  return __float_as_uint(p);
+}
+
+// floor(P * 2^40) for P given by its (non-negative, <= 1.0) float32 bits.
+__device__ __forceinline__ uint64_t fixed_mass(uint32_t key) {
+  const int e = static_cast<int>(key >> 23);  // biased exponent
+  if (e == 0) return 0ull;                    // zero or subnormal (< 2^-126)
+  const uint64_t m = (key & 0x7FFFFFu) | 0x800000u;  // 24-bit significand
+  // P * 2^40 = m * 2^(e - 127 - 23 + 40) = m * 2^(e - 110)
+  const int sh = e - 110;
+  if (sh >= 0) return m << sh;  // e <= 127 -> sh <= 17: fits
+  return (-sh >= 24) ? 0ull : (m >> (-sh));
+}
+
+__device__ __forceinline__ uint64_t warp_sum(uint64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ probs, const __grid_constant__ TopP tp,
+                                                     uint8_t* __restrict__ mask, int32_t* __restrict__ kept_idx,
+                                                     int32_t* __restrict__ kept_cnt, int H, int NB, long long rows,
+                                                     int nbp) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int warps = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint64_t* us = reinterpret_cast<uint64_t*>(smem) + static_cast<size_t>(w) * nbp;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + static_cast<size_t>(warps) * nbp * 8) + static_cast<size_t>(w) * nbp;
+  const long long row = static_cast<long long>(blockIdx.x) * warps + w;
+  if (row >= rows) return;
+  const int h = static_cast<int>((row / NB) % H);
+  const float p = tp.p[h];
+  const float* P = probs + row * NB;
+  uint8_t* mrow = mask + row * NB;
+  int32_t* irow = kept_idx + row * NB;
+
+  if (p == 1.0f) {
+    for (int j = lane; j < NB; j += 32) {
+      mrow[j] = 1;
+      irow[j] = j;
+    }
+    if (lane == 0) kept_cnt[row] = NB;
+    return;
+  }
+
+  uint64_t total = 0;
+  for (int j = lane; j < NB; j += 32) {
+    const uint32_t key = prob_key(__ldg(P + j));
+    const uint64_t u = fixed_mass(key);
+    keys[j] = key;
+    us[j] = u;
+    total += u;
+  }
+  total = warp_sum(total);
+  __syncwarp();
+  const uint64_t T = static_cast<uint64_t>(ceil(static_cast<double>(p) * static_cast<double>(total)));
+
+  uint32_t tau;
+  if (T == 0) {
+    // nothing to reach: keep the first block of the order (max key, lowest index)
+    uint32_t best_key = 0;
+    int best_j = 0x7FFFFFFF;
+    for (int j = lane; j < NB; j += 32) {
+      const uint32_t kj = keys[j];
+      if (kj > best_key || (kj == best_key && j < best_j)) {
+        best_key = kj;
+        best_j = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint32_t ok = __shfl_xor_sync(0xffffffffu, best_key, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, best_j, o);
+      if (ok > best_key || (ok == best_key && oj < best_j)) {
+        best_key = ok;
+        best_j = oj;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) keys[best_j] = kSelected;
+    tau = kSelected - 1u;
+  } else {
+    // largest tau with sum_{key >= tau} u >= T (bit 31 is never set in a key)
+    tau = 0;
+    for (int b = 30; b >= 0; --b) {
+      const uint32_t cand = tau | (1u << b);
+      uint64_t g = 0;
+      for (int j = lane; j < NB; j += 32) g += keys[j] >= cand ? us[j] : 0ull;
+      if (warp_sum(g) >= T) tau = cand;
+    }
+    uint64_t above = 0;
+    for (int j = lane; j < NB; j += 32) above += keys[j] > tau ? us[j] : 0ull;
+    const uint64_t need = T - warp_sum(above);  // > 0 by maximality of tau
+    // blocks equal to tau, in ascending index order, while mass is short
+    uint64_t carry = 0;
+    for (int base = 0; base < NB && carry < need; base += 32) {
+      const int j = base + lane;
+      const bool tie = j < NB && keys[j] == tau;
+      const uint64_t val = tie ? us[j] : 0ull;
+      uint64_t incl = val;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (tie && carry + (incl - val) < need) keys[j] = kSelected;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  __syncwarp();
+  // emit mask and the ascending kept list
+  int count = 0;
+  for (int base = 0; base < NB; base += 32) {
+    const int j = base + lane;
+    const bool sel = j < NB && keys[j] > tau;
+    if (j < NB) mrow[j] = sel ? 1 : 0;
+    const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+    if (sel) irow[count + __popc(bal & ((1u << lane) - 1u))] = j;
+    count += __popc(bal);
+  }
+  if (lane == 0) kept_cnt[row] = count;
+}
+
+}  // namespace
+
+cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p, uint8_t* mask, int32_t* idx,
+                          int32_t* cnt, cudaStream_t st) {
+  const int NB = n_blocks(s.L, s.blk);
+  const int nbp = (NB + 1) & ~1;
+  const size_t per_warp = static_cast<size_t>(nbp) * 12;
+  int warps = static_cast<int>((160 * 1024) / per_warp);
+  if (warps > 8) warps = 8;
+  if (warps < 1) warps = 1;
+  const size_t smem = per_warp * warps;
+  static size_t configured = 0;
+  if (smem > 48 * 1024 && smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  const long long rows = static_cast<long long>(s.B) * s.H * NB;
+  const long long grid = (rows + warps - 1) / warps;
+  select_kernel<<<static_cast<unsigned>(grid), warps * 32, smem, st>>>(probs, p, mask, idx, cnt, s.H, NB, rows, nbp);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

@@ -1,0 +1,201 @@
+/*
+ * bsa.h -- C ABI of libbsa: top-p block-sparse self-attention for video
+ * diffusion transformers on NVIDIA B200 (sm_100a).
+ *
+ * The method (sources named per call below):
+ *   1. reorder the latent tokens along a 3-D Hilbert curve (optional),
+ *   2. score key blocks per query block from block means and select, per
+ *      query block, the smallest set of key blocks whose softmax mass reaches
+ *      the head's top-p threshold,
+ *   3. run exact softmax attention over the kept blocks only (O and LSE),
+ *   4. correct the sparse output with a cached dense-minus-sparse refinement
+ *      scaled per head: O + alpha_h * R.
+ *
+ * Conventions shared by every call
+ *   - Tensors are dense, contiguous, row-major.  Q, K, V, O, R are bf16
+ *     [B, H, L, D] (bsa_bf16 = raw bfloat16 bits).  NB = ceil(L / blk) blocks
+ *     per sequence; the last block holds L - (NB-1)*blk tokens.
+ *   - Every pointer argument is a DEVICE pointer unless its comment says
+ *     "host".  Device pointers must be 16-byte aligned.  The caller owns and
+ *     allocates every buffer (inputs, outputs, workspaces); the library never
+ *     allocates, frees or synchronises.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream)
+ *     and returns a bsa_status.  Arguments are validated on the host before
+ *     anything is launched: a call that returns an error launched nothing.
+ *     BSA_ECUDA means a launch failed; the CUDA error is not cleared.
+ *   - Device-side faults of the input data (a kept index out of range, a
+ *     timed-out internal wait) are reported through the optional device
+ *     `status` word of bsa_sparse_attn_fwd, never by trapping.
+ *   - Supported: D in {64, 128}; blk in {64, 128}; 1 <= NB <= 4096;
+ *     B*H*L*D < 2^40; H <= 512 for bsa_select_topp_mask.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BSA_API __attribute__((visibility("default")))
+#else
+#define BSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t bsa_bf16;             /* bfloat16 bit pattern */
+typedef struct CUstream_st* bsa_stream; /* same type as cudaStream_t */
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_EINVAL = 1,     /* null required pointer, misaligned pointer, p or alpha out of range */
+  BSA_ESHAPE = 2,     /* unsupported or inconsistent sizes */
+  BSA_ENODEV = 3,     /* no sm_100 device current */
+  BSA_ECUDA = 4,      /* a kernel launch or a driver call failed */
+  BSA_EWORKSPACE = 5  /* workspace missing or too small */
+} bsa_status;
+
+/* Bits a kernel may OR into a device status word. */
+#define BSA_DEV_TIMEOUT 1   /* an internal pipeline wait exceeded its time limit */
+#define BSA_DEV_BAD_INDEX 2 /* a kept index or count was out of range and was skipped */
+
+typedef struct {
+  int B;   /* batch */
+  int H;   /* heads */
+  int L;   /* tokens per sequence */
+  int D;   /* head dimension */
+  int blk; /* tokens per query / key block */
+} bsa_shape;
+
+/* Human-readable name of a status code (static storage). */
+BSA_API const char* bsa_strerror(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+BSA_API int bsa_version(void);
+
+/*
+ * bsa_score_blocks -- block importance scores.
+ * Defines: block means as coarse attention estimates (RECAP, section 3.2),
+ * block scoring for block importance (DFSAttn abstract), a per-query-block
+ * distribution over key blocks for top-p selection (head-wise top-p and GSRS
+ * abstracts).
+ *   q_pool[b,h,i,:] = mean of Q[b,h,t,:] over the tokens t of block i
+ *   k_pool[b,h,j,:] = same for K   (partial last block: its own count)
+ *   probs[b,h,i,:]  = softmax_j( q_pool_i . k_pool_j / sqrt(D) )
+ * Arguments: q, k bf16 [B,H,L,D]; outputs q_pool, k_pool float32 [B,H,NB,D]
+ * and probs float32 [B,H,NB,NB].  Accumulation is float32.
+ * Errors: BSA_EINVAL on a null or misaligned pointer; BSA_ESHAPE on an
+ * unsupported shape.
+ */
+BSA_API int bsa_score_blocks(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, float* q_pool, float* k_pool,
+                     float* probs, bsa_stream stream);
+
+/*
+ * bsa_select_topp_mask -- cumulative top-p block selection.
+ * Defines: online top-p sparse attention with per-head thresholds (head-wise
+ * top-p abstract); top-p selection for adaptive sparsity (GSRS abstract);
+ * thresholding the top key blocks per query block (CalibAtt, Fig. 5).
+ * Per row (b,h,i): clamp P to [0,1] (NaN -> 0); order key blocks by
+ * (P desc, index asc); u_j = floor(P_j * 2^40) (exact integers);
+ * T = ceil(p_h * sum_j u_j) in IEEE double; keep the shortest ordered prefix
+ * whose u-sum is >= T (at least one block); p_h == 1 keeps every block.
+ * The result is a pure function of the float32 probs: bit-identical on any
+ * thread count or summation order.
+ * Arguments: probs float32 [B,H,NB,NB]; p_host: HOST array of H floats,
+ * each in (0, 1] (read before the call returns); outputs mask uint8
+ * [B,H,NB,NB] (1 = kept), kept_idx int32 [B,H,NB,NB] (first kept_cnt entries
+ * of each row: kept key-block indices ascending; the rest unspecified),
+ * kept_cnt int32 [B,H,NB].
+ * Errors: BSA_EINVAL on a null pointer or a p outside (0,1]; BSA_ESHAPE.
+ */
+BSA_API int bsa_select_topp_mask(bsa_shape s, const float* probs, const float* p_host, uint8_t* mask,
+                         int32_t* kept_idx, int32_t* kept_cnt, bsa_stream stream);
+
+/*
+ * bsa_reorder_workspace_bytes -- device scratch needed by bsa_reorder_tokens
+ * for a (T, Hh, W) grid (0 on an unsupported grid).
+ */
+BSA_API size_t bsa_reorder_workspace_bytes(int T, int Hh, int W);
+
+/*
+ * bsa_reorder_tokens -- 3-D Hilbert-curve token order of a latent grid.
+ * Defines: Hilbert curve-based token reordering that makes spatially close
+ * tokens contiguous (DFSAttn abstract).  Curve: Skilling's n-dimensional
+ * Hilbert curve on the smallest 2^k cube holding the grid, axis order
+ * (t, y, x) with t most significant; grid tokens are row-major
+ * n = (t*Hh + y)*W + x; cube points outside the grid are skipped.
+ * Outputs int32 perm[L] (perm[i] = grid token at Hilbert rank i) and
+ * inv[L] (inv[perm[i]] = i).  Computed once per grid shape.
+ * ws: device scratch of bsa_reorder_workspace_bytes(T,Hh,W) bytes, contents
+ * ignored on entry and clobbered.
+ * Errors: BSA_EINVAL on null pointers; BSA_ESHAPE if any extent is < 1 or
+ * > 256; BSA_EWORKSPACE if ws is NULL or ws_bytes too small.
+ */
+BSA_API int bsa_reorder_tokens(int T, int Hh, int W, int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes,
+                       bsa_stream stream);
+
+/*
+ * bsa_permute_tokens -- apply a token permutation to [B,H,L,D] bf16 rows.
+ *   inverse == 0:  y[b,h,i,:]       = x[b,h,perm[i],:]   (into curve order)
+ *   inverse != 0:  y[b,h,perm[i],:] = x[b,h,i,:]         (back to grid order)
+ * s.blk is ignored; D must be a multiple of 8.  x and y must not overlap.
+ * perm must be a permutation of [0, L) (not checked on the device).
+ */
+BSA_API int bsa_permute_tokens(bsa_shape s, const bsa_bf16* x, const int32_t* perm, bsa_bf16* y, int inverse,
+                       bsa_stream stream);
+
+/*
+ * bsa_sparse_attn_fwd -- block-sparse attention forward with an optional
+ * fused correction epilogue.
+ * Defines: computing the selected connections densely and skipping the
+ * unselected blocks (CalibAtt abstract, Fig. 5(b)); block-sparse attention
+ * for selected interactions and dense attention for refreshes (RECAP,
+ * section 4.1); cached dense refinement correcting the sparse estimate
+ * (RECAP, section 1 and abstract).
+ * For every query token r of query block i with kept key blocks K(i):
+ *   LSE[r] = log sum_{c in K(i), c < L} exp(q_r . k_c / sqrt(D))
+ *   O[r]   = sum_c exp(q_r . k_c / sqrt(D) - LSE[r]) v_c       (+ alpha_h R[r])
+ * Arguments: q, k, v bf16 [B,H,L,D]; kept_idx/kept_cnt as produced by
+ * bsa_select_topp_mask, or both NULL for dense attention (every block kept);
+ * R bf16 [B,H,L,D] and alpha float32 [H] (device), both NULL for no
+ * correction; with R the epilogue writes bf16(O_fp32 + alpha_h * R) and LSE
+ * stays the sparse LSE.  Outputs o bf16 [B,H,L,D], lse float32 [B,H,L]
+ * (natural log; -inf and O = 0 for a row with no kept key).
+ * status: optional device int32 that receives BSA_DEV_* bits (OR-ed; the
+ * caller zeroes it); NULL to skip.  Kept indices outside [0, NB) and counts
+ * outside [0, NB] are skipped/clamped and flagged, never dereferenced.
+ * Errors: BSA_EINVAL on null/misaligned pointers or exactly one of
+ * kept_idx/kept_cnt (or R/alpha) NULL; BSA_ESHAPE; BSA_ENODEV; BSA_ECUDA.
+ */
+BSA_API int bsa_sparse_attn_fwd(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
+                        const int32_t* kept_idx, const int32_t* kept_cnt, const bsa_bf16* R,
+                        const float* alpha, bsa_bf16* o, float* lse, int32_t* status, bsa_stream stream);
+
+/*
+ * bsa_refresh_refinement -- renew the cached refinement at a dense refresh.
+ * Defines: the refinement cached at a dense refresh and renewed only there
+ * (RECAP, sections 1, 3.4 and 4.3).
+ *   R = bf16( float(o_dense) - float(o_sparse) )   elementwise, [B,H,L,D]
+ * s.blk is ignored; D must be a multiple of 8.
+ */
+BSA_API int bsa_refresh_refinement(bsa_shape s, const bsa_bf16* o_dense, const bsa_bf16* o_sparse, bsa_bf16* R,
+                           bsa_stream stream);
+
+/*
+ * bsa_apply_correction -- standalone form of the fused correction.
+ * Defines: fresh sparse statistics regulating how strongly the aging cached
+ * refinement is applied (RECAP, section 1 and abstract), here as a
+ * caller-supplied per-head strength alpha_h.
+ *   o[b,h,:,:] = bf16( float(o_sparse[b,h,:,:]) + alpha[h] * float(R[b,h,:,:]) )
+ * alpha: device float32 [H].  o may alias o_sparse.  D multiple of 8.
+ */
+BSA_API int bsa_apply_correction(bsa_shape s, const bsa_bf16* o_sparse, const bsa_bf16* R, const float* alpha,
+                         bsa_bf16* o, bsa_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

@@ -1,0 +1,113 @@
+"""The C-ABI library loads, exports every symbol include/bsa.h declares, and
+rejects bad arguments on the host before touching the device (CPU only)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_logits_b200 import _lib
+from block_sparse_attention_logits_b200._lib import Shape
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from block_sparse_attention_logits_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"BSA_API\s+[\w\s\*]+?\b(bsa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("bsa_score_blocks", "bsa_select_topp_mask", "bsa_reorder_tokens", "bsa_permute_tokens",
+                 "bsa_sparse_attn_fwd", "bsa_refresh_refinement", "bsa_apply_correction", "bsa_strerror"):
+        assert name in syms
+    assert set(syms) == set(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    exported = set(re.findall(r" T (bsa_\w+)", out))
+    assert exported == set(declared_symbols())
+
+
+def test_strerror_and_version(lib):
+    assert lib.bsa_version() >= 10000
+    for code in range(6):
+        assert len(lib.bsa_strerror(code)) > 0
+    assert lib.bsa_strerror(99) == b"unknown status"
+
+
+NULL = ctypes.c_void_p(0)
+FAKE = ctypes.c_void_p(1 << 20)     # aligned, never dereferenced on the host
+MISALIGNED = ctypes.c_void_p((1 << 20) + 4)
+
+
+def test_score_blocks_validation(lib):
+    good = Shape(1, 2, 256, 128, 128)
+    assert lib.bsa_score_blocks(good, NULL, FAKE, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_score_blocks(good, MISALIGNED, FAKE, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+    for bad in (Shape(1, 2, 256, 96, 128), Shape(1, 2, 256, 128, 32), Shape(0, 2, 256, 128, 128),
+                Shape(1, 2, 0, 128, 128), Shape(1, 1, 4097 * 64, 64, 64)):
+        assert lib.bsa_score_blocks(bad, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == _lib.BSA_ESHAPE
+    # valid arguments, no GPU in this process: the device check answers
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.bsa_score_blocks(good, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == _lib.BSA_ENODEV
+
+
+def test_select_validation(lib):
+    good = Shape(1, 3, 256, 128, 128)
+    p_ok = (ctypes.c_float * 3)(0.9, 0.5, 1.0)
+    for bad_p in ((0.0, 0.5, 0.5), (0.5, 1.5, 0.5), (0.5, float("nan"), 0.5), (-1.0, 0.5, 0.5)):
+        arr = (ctypes.c_float * 3)(*bad_p)
+        assert lib.bsa_select_topp_mask(good, FAKE, arr, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_select_topp_mask(good, FAKE, None, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_select_topp_mask(good, FAKE, p_ok, NULL, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+    many = Shape(1, 513, 256, 128, 128)
+    arr = (ctypes.c_float * 513)(*([0.9] * 513))
+    assert lib.bsa_select_topp_mask(many, FAKE, arr, FAKE, FAKE, FAKE, NULL) == _lib.BSA_ESHAPE
+
+
+def test_reorder_validation(lib):
+    assert lib.bsa_reorder_workspace_bytes(21, 45, 80) == 512 * 4      # 128^3 cells / 4096 per chunk
+    assert lib.bsa_reorder_workspace_bytes(2, 32, 32) == 8 * 4         # 32^3 / 4096
+    assert lib.bsa_reorder_workspace_bytes(257, 1, 1) == 0
+    assert lib.bsa_reorder_workspace_bytes(0, 4, 4) == 0
+    assert lib.bsa_reorder_tokens(257, 2, 2, FAKE, FAKE, FAKE, 1 << 20, NULL) == _lib.BSA_ESHAPE
+    assert lib.bsa_reorder_tokens(21, 45, 80, FAKE, FAKE, FAKE, 100, NULL) == _lib.BSA_EWORKSPACE
+    assert lib.bsa_reorder_tokens(21, 45, 80, FAKE, FAKE, NULL, 4096, NULL) == _lib.BSA_EWORKSPACE
+    assert lib.bsa_reorder_tokens(21, 45, 80, NULL, FAKE, FAKE, 4096, NULL) == _lib.BSA_EINVAL
+
+
+def test_attention_validation(lib):
+    s = Shape(1, 2, 1000, 128, 128)
+    args = [FAKE] * 3
+    # exactly one of kept_idx / kept_cnt
+    assert lib.bsa_sparse_attn_fwd(s, *args, FAKE, NULL, NULL, NULL, FAKE, FAKE, NULL, NULL) == _lib.BSA_EINVAL
+    # R without alpha
+    assert lib.bsa_sparse_attn_fwd(s, *args, NULL, NULL, FAKE, NULL, FAKE, FAKE, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd(s, *args, NULL, NULL, NULL, NULL, NULL, FAKE, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd(Shape(1, 2, 1000, 80, 128), *args, NULL, NULL, NULL, NULL, FAKE, FAKE,
+                                   NULL, NULL) == _lib.BSA_ESHAPE
+    assert lib.bsa_sparse_attn_fwd(Shape(70000, 1, 10, 64, 64), *args, NULL, NULL, NULL, NULL, FAKE, FAKE,
+                                   NULL, NULL) == _lib.BSA_ESHAPE
+
+
+def test_elementwise_validation(lib):
+    assert lib.bsa_refresh_refinement(Shape(1, 1, 10, 12, 0), FAKE, FAKE, FAKE, NULL) == _lib.BSA_ESHAPE
+    assert lib.bsa_refresh_refinement(Shape(1, 1, 10, 16, 0), FAKE, NULL, FAKE, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_apply_correction(Shape(1, 1, 10, 16, 0), FAKE, FAKE, NULL, FAKE, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_permute_tokens(Shape(1, 1, 10, 16, 0), FAKE, FAKE, FAKE, 0, NULL) == _lib.BSA_EINVAL  # x == y
