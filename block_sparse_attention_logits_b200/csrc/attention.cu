@@ -266,10 +266,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = u + 1;
       }
       if (sh->abort_flag) {
-        // drain: wait (bounded) for the loads of the last NS issues to land
+        // Drain before the CTA exits: wait (bounded) for the newest load of
+        // every slot.  Load k of a slot is issued only after the release of
+        // load k-1, which the MMA thread commits after observing its landing,
+        // so the parity of load k is unambiguous here.
         for (int u = issued - NS < 0 ? 0 : issued - NS; u < issued; ++u) {
           const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try(&sh->full[u % NS], (u / NS) & 1) && globaltimer_ns() - t0 < kTimeoutNs / 4) {
+          while (!mbar_try(&sh->full[u % NS], (u / NS) & 1) && globaltimer_ns() - t0 < kTimeoutNs) {
           }
         }
       }
@@ -292,6 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint32_t q_base = smem_u32(q_smem);
       const uint32_t stage_base = smem_u32(stage_smem);
+      // Landing of the K/V stages is observed strictly in union order, for
+      // every entry, whichever tile keeps it.  A tile skips entries it does not
+      // keep, so testing only its own entry could confuse phase k of a slot
+      // with phase k-2 (a parity wait cannot tell them apart); observing in
+      // order guarantees phase k-1 completed before phase k is tested.
+      int seen = 0;
       uint64_t t_idle = 0;
       uint32_t spins = 0;
       while (ok && (st[0] != DONE || st[1] != DONE)) {
@@ -301,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (st[t] == NEED_S) {
             const int u = cur[t];
             const int slot = u % NS;
-            if (mbar_test(&sh->full[slot], (u / NS) & 1)) {
+            while (seen <= u && mbar_test(&sh->full[seen % NS], (seen / NS) & 1)) ++seen;
+            if (seen > u) {
               tc_fence_after();
               const uint32_t qa = q_base + t * C::Q_BYTES;
               const uint32_t ka = stage_base + slot * C::STAGE_BYTES;
