@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the top-p block-sparse attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one pass of the whole hot path over one batch of the Wan2.1-14B
+720P workload (B=1, H=40, D=128, 21x45x80 latent tokens, blk 128, Hilbert
+order, top-p tuned to ~90% block sparsity) with inputs resident in HBM:
+  gather Q, K, V into Hilbert order -> block means + block softmax -> top-p
+  selection -> block-sparse attention with the fused O + alpha*R epilogue ->
+  scatter O back to grid order.
+value = kept-block TFLOP per step x ranks / device-timed step time (max over
+ranks).  Under torchrun every rank runs its own copy of the workload (heads
+are independent problems, no collective on the data path): weak scaling.
+
+--impl reference times the CPU oracle (the plain float64 statement of the
+same computation) on a bounded sample of the same workload, on the host
+cores; under torchrun only rank 0 runs it.
+Prints one JSON line on rank 0.
+"""
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_logits_b200 import configs  # noqa: E402
+from block_sparse_attention_logits_b200.synthetic import make_qkv, random_bf16  # noqa: E402
+
+METRIC = "block-sparse attn ms/call & TFLOP/s on kept blocks vs bf16 TC peak at 90% sparsity"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 8  # 3 gathers, pooling, block softmax, selection, attention, scatter
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="wan2.1-14b-720p", choices=sorted(configs.ALL))
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only the first N heads of the workload (small profiling captures)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- plumbing
+
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash():
+    p = os.path.join(ROOT, "block_sparse_attention_logits_b200", "csrc", "attention.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu summary, only if
+    it was taken on the current attention source."""
+    p = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(workload)
+    if not d or d.get("attention_cu_sha256_16") != source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.sel = str(device_index)
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = [r.split(", ") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        os.unlink(self.path)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def kept_flops(mask, L, blk, D):
+    """4*D*sum over kept (i, j) of rows_i * cols_j, real tokens only."""
+    nb = mask.shape[-1]
+    sizes = torch.full((nb,), float(blk), dtype=torch.float64, device=mask.device)
+    sizes[-1] = L - (nb - 1) * blk
+    per_row = (mask.double() * sizes).sum(-1)  # kept key tokens per query block
+    return float(4.0 * D * (per_row * sizes).sum().item())
+
+
+# ---------------------------------------------------------- oracle sample
+
+def oracle_sample(w, p, seconds, max_blocks=None):
+    """Time the oracle on head 0 of the workload: Hilbert order, block scores,
+    top-p selection, then masked attention of as many query blocks as fit in
+    `seconds` (at least 4).  Returns (kept_flops, seconds, n_blocks, detail)."""
+    from oracle import attention as oatt
+    from oracle import hilbert as ohil
+    from oracle import scoring as osco
+    from oracle import topp as otop
+
+    t = make_qkv(1, 1, w.grid, w.D, w.fp)
+    q, k, v = (t[n].float().numpy() for n in ("q", "k", "v"))
+    t0 = time.perf_counter()
+    if w.hilbert:
+        perm, _ = ohil.hilbert_perm(*w.grid)
+        q, k, v = (ohil.permute_rows(x, perm) for x in (q, k, v))
+    _, _, P = osco.score_blocks(q, k, w.blk)
+    _, idx, cnt = otop.select_topp_mask_fast(P, np.array([p], np.float32))
+    t_score = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    order = rng.permutation(w.NB)
+    sizes = np.full(w.NB, w.blk)
+    sizes[-1] = w.L - (w.NB - 1) * w.blk
+    flops, done, t_att = 0.0, 0, 0.0
+    for i in order:
+        if (t_att >= seconds and done >= 4) or (max_blocks and done >= max_blocks):
+            break
+        t1 = time.perf_counter()
+        kb = idx[0, 0, i, :cnt[0, 0, i]]
+        oatt.masked_attention_block(q, k, v, kb, w.blk, 0, 0, int(i))
+        t_att += time.perf_counter() - t1
+        flops += 4.0 * w.D * sizes[i] * sizes[kb].sum()
+        done += 1
+    # charge the scoring of the head in proportion to the blocks sampled
+    total = t_att + t_score * done / w.NB
+    return flops, total, done, f"head 0, {done} of {w.NB} query blocks (float64 numpy), scoring charged pro rata"
+
+
+# ------------------------------------------------------------------- ours
+
+def run_ours(args, w, world, rank, local):
+    from block_sparse_attention_logits_b200 import api, _lib
+    from block_sparse_attention_logits_b200 import build as bsa_build
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    bsa_build.build()
+    _lib.load()
+
+    B, H, L, D, blk = w.B, w.H, w.L, w.D, w.blk
+    p = float(w.p[0])
+    pin = torch.cuda.is_available()
+    host = {n: torch.empty((B, H, L, D), dtype=torch.bfloat16, pin_memory=pin) for n in ("q", "k", "v")}
+    make_qkv(B, H, w.grid, D, w.fp, out=host)
+    q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+    R_h = random_bf16((B, H, L, D), 99, scale=0.05).to(dev)  # cached refinement (curve order)
+    alpha = torch.tensor(w.alpha(), dtype=torch.float32, device=dev)
+
+    if w.hilbert:
+        perm, inv = api.reorder_tokens(*w.grid, device=dev)
+    nb = api.n_blocks(L, blk)
+    bufs = dict(
+        qh=torch.empty_like(q), kh=torch.empty_like(k), vh=torch.empty_like(v),
+        qp=torch.empty((B, H, nb, D), dtype=torch.float32, device=dev),
+        kp=torch.empty((B, H, nb, D), dtype=torch.float32, device=dev),
+        probs=torch.empty((B, H, nb, nb), dtype=torch.float32, device=dev),
+        mask=torch.empty((B, H, nb, nb), dtype=torch.uint8, device=dev),
+        idx=torch.empty((B, H, nb, nb), dtype=torch.int32, device=dev),
+        cnt=torch.empty((B, H, nb), dtype=torch.int32, device=dev),
+        oh=torch.empty_like(q), lse=torch.empty((B, H, L), dtype=torch.float32, device=dev),
+        o=torch.empty_like(q),
+    )
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ev = None
+
+    def step(qi, ki, vi, events=None):
+        b = bufs
+        if w.hilbert:
+            api.permute_tokens(qi, perm, out=b["qh"])
+            api.permute_tokens(ki, perm, out=b["kh"])
+            api.permute_tokens(vi, perm, out=b["vh"])
+            qs, ks, vs = b["qh"], b["kh"], b["vh"]
+        else:
+            qs, ks, vs = qi, ki, vi
+        if events:
+            events[0].record()
+        api.score_blocks(qs, ks, blk, b["qp"], b["kp"], b["probs"])
+        api.select_topp_mask(b["probs"], p, L, blk, D, b["mask"], b["idx"], b["cnt"])
+        if events:
+            events[1].record()
+        api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h, alpha, b["oh"], b["lse"], status=status)
+        if events:
+            events[2].record()
+        if w.hilbert:
+            api.permute_tokens(b["oh"], perm, inverse=True, out=b["o"])
+            return b["o"], b["lse"]
+        return b["oh"], b["lse"]
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    # warm-up
+    for _ in range(max(args.warmup, 3)):
+        step(q, k, v)
+    torch.cuda.synchronize()
+    if status.item() != 0:
+        raise RuntimeError(f"attention kernel reported status {status.item()}")
+    flops = kept_flops(bufs["mask"], L, blk, D)
+    sparsity = 1.0 - bufs["cnt"].double().sum().item() / (B * H * nb * nb)
+
+    # timed region: K steps, events per stage
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    start.record()
+    for i in range(K):
+        step(q, k, v, evs[i])
+    stop.record()
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = start.elapsed_time(stop)
+    attn_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(K)]
+    sel_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_step = elapsed_ms / K
+    value = flops * world / (ms_step * 1e-3) / 1e12
+
+    # e2e: host buffers in, result out, through the same API calls
+    e2e = None
+    if not args.no_e2e:
+        o_host = torch.empty((B, H, L, D), dtype=torch.bfloat16, pin_memory=pin)
+        lse_host = torch.empty((B, H, L), dtype=torch.float32, pin_memory=pin)
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            qd.copy_(host["q"], non_blocking=True)
+            kd.copy_(host["k"], non_blocking=True)
+            vd.copy_(host["v"], non_blocking=True)
+            o, lse = step(qd, kd, vd)
+            o_host.copy_(o, non_blocking=True)
+            lse_host.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        Ke = max(3, min(K, 20))
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for _ in range(Ke):
+            e2e_step()
+        e2.record()
+        barrier()
+        e_ms = s2.elapsed_time(e2)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": round(flops * world / (e_ms / Ke * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "ms_per_step": round(e_ms / Ke, 3), "steps": Ke,
+               "h2d_bytes_per_step": 3 * B * H * L * D * 2, "d2h_bytes_per_step": B * H * L * D * 2 + B * H * L * 4}
+
+    if status.item() != 0:
+        raise RuntimeError(f"attention kernel reported status {status.item()}")
+
+    peaks, peak_src = load_peaks()
+    attn_avg_ms = float(np.mean(attn_ms))
+    achieved = flops / (attn_avg_ms * 1e-3) / 1e12
+    traffic = profiled_traffic(w.name)
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2),
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                "traffic": traffic, "kernel": "sparse_attn_kernel<128,128>",
+                "peak_kind": f"{peak_src} sustained (kernel timed inside a long step)",
+                "peak_burst": peaks["bf16_tflops"], "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        f, s, n, what = oracle_sample(w, p, args.cpu_seconds)
+        cpu = {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": what, "seconds": round(s, 2)}
+
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "H": H, "L": L, "D": D, "blk": blk, "grid": list(w.grid),
+                   "hilbert": w.hilbert, "top_p": p, "block_sparsity": round(sparsity, 4),
+                   "fused_correction": True, "kept_tflop_per_step": round(flops / 1e12, 4),
+                   "l2": "inputs larger than L2 (Q/K/V 2.3 GB per step), no flush",
+                   "parallelism": f"independent replicas x{world} (heads shard with no collective)"},
+        "attn": {"ms_per_call": round(attn_avg_ms, 4), "ms_p10": round(float(np.percentile(attn_ms, 10)), 4),
+                 "ms_p90": round(float(np.percentile(attn_ms, 90)), 4), "kept_tflops": round(achieved, 2),
+                 "dense_equiv_tflops": round(4.0 * B * H * L * L * D / (attn_avg_ms * 1e-3) / 1e12, 2)},
+        "stages_ms": {"score_and_select": round(float(np.mean(sel_ms)), 4), "attention": round(attn_avg_ms, 4),
+                      "gather_scatter_and_rest": round(ms_step - attn_avg_ms - float(np.mean(sel_ms)), 4)},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": LAUNCHES_PER_STEP * K if w.hilbert else (LAUNCHES_PER_STEP - 4) * K,
+        "clocks": clk,
+    }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# -------------------------------------------------------------- reference
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    p = float(w.p[0])
+    blocks = 12  # query blocks of head 0 per step
+    times, flops = [], []
+    for i in range(max(args.warmup, 3) + args.steps):
+        f, s, n, what = oracle_sample(w, p, seconds=1e9, max_blocks=blocks)
+        if i >= max(args.warmup, 3):
+            times.append(s)
+            flops.append(f)
+    sec = float(np.sum(times))
+    value = float(np.sum(flops)) / sec / 1e12
+    cores = blas_threads()
+    out = {
+        "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(sec / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "D": w.D, "blk": w.blk,
+                   "grid": list(w.grid), "hilbert": w.hilbert, "top_p": p,
+                   "parallelism": "CPU oracle on rank 0"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {what}"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_info()
+    if world != args.gpus and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    w = configs.ALL[args.workload]
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, H=min(args.heads, w.H))
+    if args.impl == "reference":
+        run_reference(args, w, world, rank)
+    else:
+        run_ours(args, w, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()
