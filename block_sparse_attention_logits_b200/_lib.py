@@ -12,7 +12,7 @@ LIB_PATH = os.path.join(_PKG, "libbsa.so")
 
 EXPORTS = (
     "bsa_strerror", "bsa_version", "bsa_score_blocks", "bsa_select_topp_mask",
-    "bsa_reorder_workspace_bytes", "bsa_reorder_tokens", "bsa_permute_tokens",
+    "bsa_reorder_workspace_bytes", "bsa_reorder_tokens", "bsa_reorder_tokens_noalloc", "bsa_permute_tokens",
     "bsa_sparse_attn_fwd", "bsa_refresh_refinement", "bsa_apply_correction",
 )
 
@@ -55,6 +55,7 @@ def load():
         "bsa_select_topp_mask": (_I, [Shape, _P, ctypes.POINTER(ctypes.c_float), _P, _P, _P, _P]),
         "bsa_reorder_workspace_bytes": (_SZ, [_I, _I, _I]),
         "bsa_reorder_tokens": (_I, [_I, _I, _I, _P, _P, _P, _SZ, _P]),
+        "bsa_reorder_tokens_noalloc": (_I, [_I, _I, _I, _P, _P, _P]),
         "bsa_permute_tokens": (_I, [Shape, _P, _P, _P, _I, _P]),
         "bsa_sparse_attn_fwd": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_refresh_refinement": (_I, [Shape, _P, _P, _P, _P]),

@@ -10,6 +10,8 @@
 // Ranks come from a two-pass stream compaction over chunks of the index
 // range: pass 1 counts grid points per chunk into the caller's workspace,
 // pass 2 adds up the counts of the preceding chunks and writes perm / inv.
+#include <mutex>
+
 #include "internal.cuh"
 
 namespace bsa {
@@ -217,4 +219,62 @@ cudaError_t launch_permute(const bsa_shape& s, const __nv_bfloat16* x, const int
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant (bsa_reorder_tokens_noalloc).
+//
+// Some callers cannot allocate device memory for the two-pass scratch: a host
+// framework that owns all device memory through its own allocator and hands
+// this library only its input and output buffers, with no way to ask for more;
+// a process whose caching allocator has already reserved nearly all of HBM, so
+// a fresh cudaMalloc can fail; or a latency-critical loop that cannot afford
+// cudaMalloc's implicit device synchronisation.  For them the per-chunk counts
+// live in a file-scope device array instead of a caller workspace.
+//
+// Limit: kNoAllocChunks counts (16 KB), which covers every grid this call
+// accepts (extents <= 256, so at most 2^24 cube cells = 4096 chunks).  Every
+// GPU that loads the library holds the array until the process exits.
+// Nothing in it has to start at zero: pass 1 writes every count pass 2 reads.
+// All calls share the array and it keeps the last call's counts, so calls
+// that overlap on the GPU (two streams, two host threads) race: serialise them.
+constexpr int kNoAllocChunks = 4096;
+static __device__ __align__(256) int g_reorder_counts[kNoAllocChunks];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_counts_mu;
+void* g_counts_addr[kMaxDevices] = {};
+
+// Device address of g_reorder_counts on the current device, looked up once per
+// device (the first call on a device does it; make that call before any stream
+// capture).  In host code the array's name is only a host-side stand-in.
+int counts_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ENODEV;
+  std::lock_guard<std::mutex> lock(g_counts_mu);
+  if (g_counts_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_reorder_counts) != cudaSuccess || p == nullptr) return BSA_ECUDA;
+    g_counts_addr[dev] = p;
+  }
+  *out = g_counts_addr[dev];
+  return BSA_OK;
+}
+}  // namespace
+
 }  // namespace bsa
+
+extern "C" int bsa_reorder_tokens_noalloc(int T, int Hh, int W, int32_t* perm, int32_t* inv, bsa_stream stream) {
+  if (!perm || !inv) return BSA_EINVAL;
+  const size_t need = bsa::hilbert_workspace_bytes(T, Hh, W);
+  if (need == 0 || need > sizeof(int) * static_cast<size_t>(bsa::kNoAllocChunks)) return BSA_ESHAPE;
+  if ((reinterpret_cast<uintptr_t>(perm) & 15u) || (reinterpret_cast<uintptr_t>(inv) & 15u)) return BSA_EINVAL;
+  int major = 0, dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10)
+    return BSA_ENODEV;
+  void* counts = nullptr;
+  if (int r = bsa::counts_address(&counts)) return r;
+  return bsa::launch_hilbert(T, Hh, W, perm, inv, counts, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? BSA_OK
+             : BSA_ECUDA;
+}

@@ -137,6 +137,23 @@ BSA_API int bsa_reorder_tokens(int T, int Hh, int W, int32_t* perm, int32_t* inv
                        bsa_stream stream);
 
 /*
+ * bsa_reorder_tokens_noalloc -- bsa_reorder_tokens for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a library
+ * convenience.  Same result as bsa_reorder_tokens; the scratch it needs lives
+ * in a 16 KB array inside the library (every GPU that loads the library holds
+ * it until exit), which covers every grid the call accepts (extents <= 256).
+ * For callers whose device memory is owned by a host framework's allocator
+ * that passes only input/output buffers, whose HBM is already reserved, or
+ * that cannot take cudaMalloc's implicit synchronisation.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the array: calls that overlap on the GPU race, so
+ * serialise them.  Allocates nothing, frees nothing.
+ * Errors: as bsa_reorder_tokens, with BSA_ESHAPE for a grid beyond the limit.
+ */
+BSA_API int bsa_reorder_tokens_noalloc(int T, int Hh, int W, int32_t* perm, int32_t* inv, bsa_stream stream);
+
+/*
  * bsa_permute_tokens -- apply a token permutation to [B,H,L,D] bf16 rows.
  *   inverse == 0:  y[b,h,i,:]       = x[b,h,perm[i],:]   (into curve order)
  *   inverse != 0:  y[b,h,perm[i],:] = x[b,h,i,:]         (back to grid order)
