@@ -18,17 +18,26 @@
 // does not keep a block are masked to -inf for that block.
 //
 // Warp roles (12 warps):
-//   warp 0      TMA producer: Q tiles once, then K/V of every union entry into
-//               an NS-deep ring (128-byte swizzled panels of 64 columns).
-//   warp 1      MMA issuer (one thread): S_t = Q_t K^T (SS form, both operands
-//               in shared memory) into TMEM, then O_t += P_t V with P_t read
-//               from TMEM (TS form).  It serves the two tiles from a polling
-//               state machine so neither tile can block the other.
-//   warp 2      TMEM allocation / release.
-//   warps 4-7   softmax + epilogue of tile 0 (one thread per query row).
-//   warps 8-11  softmax + epilogue of tile 1.
+//   warp 0      TMA producer of Q (once) and of K for every union entry
+//   warp 3      TMA producer of V for every union entry; TMEM allocation
+//   warp 1 / 2  MMA issuer of tile 0 / tile 1: S_t = Q_t K^T (both operands
+//               in shared memory, K-major) into TMEM, then O_t += P_t V with
+//               P_t read from TMEM and V MN-major in shared memory
+//   warps 4-7   softmax + epilogue of tile 0 (one thread per query row)
+//   warps 8-11  softmax + epilogue of tile 1
+// K and V have separate rings, so a K slot is refilled as soon as the S
+// MMAs that read it are done, without waiting for the PV MMAs.
 // TMEM columns: S0 | S1 | O0 | O1.  P_t (bf16, packed in pairs) overwrites the
-// first BN/2 columns of S_t once S_t has been read.
+// first BN/2 columns of S_t once S_t has been read; the next S_t is issued by
+// the same thread after the PV that reads P_t, so the tensor pipe's issue
+// order protects P_t.
+//
+// Every role walks the union in order and waits on every entry, member or
+// not: a parity wait cannot tell phase k of a barrier from phase k-2, so a
+// thread that skipped entries could take an older phase for the one it wants.
+// An MMA warp that does not compute an entry still observes its landing and
+// releases its slot with a plain arrive, so each release barrier always gets
+// exactly one arrival per MMA warp and entry.
 //
 // Online softmax in the log2 domain in fp32.  The running max used for the
 // exponentials is only raised when the block max exceeds it by more than 8
@@ -53,9 +62,13 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 384;
-constexpr int BM = 128;                        // query rows per tile
+constexpr int BM = 128;                         // query rows per tile
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
-constexpr float kRescaleThreshold = 8.0f;      // log2 units
+constexpr float kRescaleThreshold = 8.0f;       // log2 units
+constexpr int kRegsLaunch = 168;                // 65536 / 384, rounded down to a multiple of 8
+constexpr int kRegsCtl = 72;
+constexpr int kRegsSoftmax = 216;
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split exceeds launch");
 
 struct Params {
   const int32_t* kept_idx;
@@ -72,22 +85,21 @@ struct Params {
 
 template <int D, int BN>
 struct Cfg {
-  static constexpr int G = BM / BN;              // query blocks per 128-row tile
+  static constexpr int G = BM / BN;               // query blocks per 128-row tile
   static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+  static constexpr int KV_BYTES = BN * D * 2;     // one K or one V tile
   static constexpr int UNION_BYTES = kMaxNB * 2;  // uint16 per union entry
-  static constexpr int BITMAP_BYTES = kMaxNB;     // one byte of membership bits per key block
   static constexpr int MISC_BYTES = 256;          // barriers and scalars
-  static constexpr int FIXED = 2 * Q_BYTES + UNION_BYTES + BITMAP_BYTES + MISC_BYTES;
-  static constexpr int NS_FIT = (227 * 1024 - 1024 - FIXED) / STAGE_BYTES;
-  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
-  static_assert(NS >= 2, "shared memory too small for a double-buffered K/V ring");
+  static constexpr int SLOTS = (227 * 1024 - 1024 - 2 * Q_BYTES - UNION_BYTES - MISC_BYTES) / KV_BYTES;
+  static constexpr int NSK = ((SLOTS + 1) / 2) > 4 ? 4 : (SLOTS + 1) / 2;
+  static constexpr int NSV = (SLOTS / 2) > 4 ? 4 : SLOTS / 2;
+  static_assert(NSK >= 2 && NSV >= 2, "shared memory too small for double-buffered K and V");
+  static_assert(KV_BYTES >= kMaxNB, "the set-up bitmap is staged in the first K slot");
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_STAGE = 2 * Q_BYTES;
-  static constexpr int OFF_UNION = OFF_STAGE + NS * STAGE_BYTES;
-  static constexpr int OFF_BITMAP = OFF_UNION + UNION_BYTES;
-  static constexpr int OFF_MISC = OFF_BITMAP + BITMAP_BYTES;
+  static constexpr int OFF_K = 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
+  static constexpr int OFF_UNION = OFF_V + NSV * KV_BYTES;
+  static constexpr int OFF_MISC = OFF_UNION + UNION_BYTES;
   static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
   static constexpr int COL_S0 = 0, COL_S1 = BN, COL_O0 = 2 * BN, COL_O1 = 2 * BN + D;
   static constexpr int TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256 : 512;
@@ -96,13 +108,15 @@ struct Cfg {
 
 struct Shared {
   // laid out in the MISC region
-  uint64_t full[4];
-  uint64_t empty[4];
+  uint64_t full_k[4];
+  uint64_t empty_k[4];
+  uint64_t full_v[4];
+  uint64_t empty_v[4];
   uint64_t q_full;
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
   uint32_t n_union;
   uint32_t n_tile[2];
@@ -132,9 +146,50 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Sha
   }
 }
 
+// Warp-uniform bounded wait (every lane waits; all must succeed).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Shared* sh, const Params& prm) {
+  const bool ok = wait_bounded(bar, parity, sh, prm);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait used only while draining after an abort.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try(bar, parity) && globaltimer_ns() - t0 < kTimeoutNs) {
+  }
+}
+
 __device__ __forceinline__ int next_member(const uint16_t* ulist, int i, int U, uint32_t tile_mask) {
   while (i < U && ((ulist[i] >> 12) & tile_mask) == 0) ++i;
   return i;
+}
+
+// TMA producer of one operand ring (K or V): entry u goes to slot u % NS once
+// both MMA warps released the slot's previous entry.
+template <int D, int BN, int NS>
+__device__ __forceinline__ void produce_ring(const CUtensorMap* map, uint8_t* ring, uint64_t* full, uint64_t* empty,
+                                             const uint16_t* ulist, int U, int bh, int lane, Shared* sh,
+                                             const Params& prm) {
+  using C = Cfg<D, BN>;
+  int issued = 0;
+  for (int u = 0; u < U; ++u) {
+    const int slot = u % NS;
+    if (u >= NS && !warp_wait(&empty[slot], ((u / NS) - 1) & 1, sh, prm)) break;
+    if (lane == 0) {
+      const int kb = ulist[u] & 0xFFF;
+      uint8_t* dst = ring + slot * C::KV_BYTES;
+      mbar_arrive_expect_tx(&full[slot], C::KV_BYTES);
+      for (int pnl = 0; pnl < C::PANELS; ++pnl)
+        tma_load_3d(dst + pnl * BN * 128, map, &full[slot], pnl * 64, kb * BN, bh);
+    }
+    __syncwarp();
+    issued = u + 1;
+  }
+  if (sh->abort_flag && lane == 0) {
+    // load k of a slot is issued only after release k-1, which follows the
+    // consumers' observation of landing k-1: the parity below is exact
+    for (int u = issued - NS < 0 ? 0 : issued - NS; u < issued; ++u) drain_wait(&full[u % NS], (u / NS) & 1);
+  }
 }
 
 template <int D, int BN>
@@ -143,12 +198,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmV, const Params prm) {
   using C = Cfg<D, BN>;
   constexpr int G = C::G;
-  constexpr int NS = C::NS;
+  constexpr int NSK = C::NSK;
+  constexpr int NSV = C::NSV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint16_t* ulist = reinterpret_cast<uint16_t*>(smem + C::OFF_UNION);
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + C::OFF_BITMAP);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + C::OFF_K);  // set-up only
   Shared* sh = reinterpret_cast<Shared*>(smem + C::OFF_MISC);
+  uint8_t* q_smem = smem + C::OFF_Q;
+  uint8_t* k_ring = smem + C::OFF_K;
+  uint8_t* v_ring = smem + C::OFF_V;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -159,17 +218,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&sh->full[s], 1);
-      mbar_init(&sh->empty[s], 1);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&sh->full_k[s], 1);
+      mbar_init(&sh->empty_k[s], 2);
+      mbar_init(&sh->full_v[s], 1);
+      mbar_init(&sh->empty_v[s], 2);
     }
     mbar_init(&sh->q_full, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sh->s_full[t], 1);
       mbar_init(&sh->p_full[t], 128);
       mbar_init(&sh->o_full[t], 1);
+      mbar_init(&sh->drain[t], 1);
     }
-    mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     fence_mbar_init();
   }
@@ -178,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  if (warp == 2) {
+  if (warp == 3) {
     tmem_alloc(&sh->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
     tc_fence_before();
@@ -230,153 +291,101 @@ __global__ void __launch_bounds__(kThreads, 1)
       sh->n_tile[1] = c1;
     }
   }
-  __syncthreads();
+  __syncthreads();  // union list complete; the bitmap's K slot may now be overwritten
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
   const int U = static_cast<int>(sh->n_union);
   const int ntile[2] = {static_cast<int>(sh->n_tile[0]), static_cast<int>(sh->n_tile[1])};
   const uint32_t tile_mask[2] = {(1u << G) - 1u, ((1u << G) - 1u) << G};
-  uint8_t* q_smem = smem + C::OFF_Q;
-  uint8_t* stage_smem = smem + C::OFF_STAGE;
 
-  if (warp == 0) {
-    // --------------------------------------------------------- TMA producer
-    if (lane == 0 && U > 0) {
-      int tiles_here = 0;
-      for (int t = 0; t < 2; ++t)
-        if ((pair * 2 + t) * BM < L) ++tiles_here;
-      mbar_arrive_expect_tx(&sh->q_full, tiles_here * C::Q_BYTES);
-      for (int t = 0; t < 2; ++t) {
-        const int row0 = (pair * 2 + t) * BM;
-        if (row0 >= L) continue;
-        for (int pnl = 0; pnl < C::PANELS; ++pnl)
-          tma_load_3d(q_smem + t * C::Q_BYTES + pnl * BM * 128, &tmQ, &sh->q_full, pnl * 64, row0, bh);
-      }
-      int issued = 0;
-      for (int u = 0; u < U; ++u) {
-        const int slot = u % NS;
-        if (u >= NS && !wait_bounded(&sh->empty[slot], ((u / NS) - 1) & 1, sh, prm)) break;
-        const int kb = ulist[u] & 0xFFF;
-        uint8_t* st = stage_smem + slot * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(&sh->full[slot], 2 * C::KV_BYTES);
-        for (int pnl = 0; pnl < C::PANELS; ++pnl) {
-          tma_load_3d(st + pnl * BN * 128, &tmK, &sh->full[slot], pnl * 64, kb * BN, bh);
-          tma_load_3d(st + C::KV_BYTES + pnl * BN * 128, &tmV, &sh->full[slot], pnl * 64, kb * BN, bh);
-        }
-        issued = u + 1;
-      }
-      if (sh->abort_flag) {
-        // Drain before the CTA exits: wait (bounded) for the newest load of
-        // every slot.  Load k of a slot is issued only after the release of
-        // load k-1, which the MMA thread commits after observing its landing,
-        // so the parity of load k is unambiguous here.
-        for (int u = issued - NS < 0 ? 0 : issued - NS; u < issued; ++u) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try(&sh->full[u % NS], (u / NS) & 1) && globaltimer_ns() - t0 < kTimeoutNs) {
-          }
+  if (warp < 4) {
+    // Registers: warpgroup 0 (TMA, MMA issue, TMEM allocation) needs few; the
+    // two softmax warpgroups hold a whole score row each.
+    setmaxnreg_dec<kRegsCtl>();
+    if (warp == 0 && U > 0) {
+      // ------------------------------------------------ TMA: Q, then K ring
+      if (lane == 0) {
+        int tiles_here = 0;
+        for (int t = 0; t < 2; ++t)
+          if ((pair * 2 + t) * BM < L) ++tiles_here;
+        mbar_arrive_expect_tx(&sh->q_full, tiles_here * C::Q_BYTES);
+        for (int t = 0; t < 2; ++t) {
+          const int row0 = (pair * 2 + t) * BM;
+          if (row0 >= L) continue;
+          for (int pnl = 0; pnl < C::PANELS; ++pnl)
+            tma_load_3d(q_smem + t * C::Q_BYTES + pnl * BM * 128, &tmQ, &sh->q_full, pnl * 64, row0, bh);
         }
       }
-    }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------- MMA issuer
-    if (lane == 0 && U > 0) {
+      __syncwarp();
+      produce_ring<D, BN, NSK>(&tmK, k_ring, sh->full_k, sh->empty_k, ulist, U, bh, lane, sh, prm);
+    } else if (warp == 3 && U > 0) {
+      // ------------------------------------------------------ TMA: V ring
+      produce_ring<D, BN, NSV>(&tmV, v_ring, sh->full_v, sh->empty_v, ulist, U, bh, lane, sh, prm);
+    } else if ((warp == 1 || warp == 2) && U > 0) {
+      // ----------------------------------------- MMA issue, one tile each
+      const int t = warp - 1;
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(BM, D, false, true);
-      const uint32_t colS[2] = {C::COL_S0, C::COL_S1};
-      const uint32_t colO[2] = {C::COL_O0, C::COL_O1};
-      bool ok = wait_bounded(&sh->q_full, 0, sh, prm);
+      const uint32_t colS = t == 0 ? C::COL_S0 : C::COL_S1;
+      const uint32_t colO = t == 0 ? C::COL_O0 : C::COL_O1;
+      const uint32_t qa = smem_u32(q_smem) + t * C::Q_BYTES;
+      const uint32_t k_base = smem_u32(k_ring);
+      const uint32_t v_base = smem_u32(v_ring);
+      bool ok = ntile[t] == 0 || warp_wait(&sh->q_full, 0, sh, prm);
       tc_fence_after();
-      enum { NEED_S = 0, NEED_P = 1, DONE = 2 };
-      int st[2], cur[2], n[2];
-      for (int t = 0; t < 2; ++t) {
-        n[t] = 0;
-        cur[t] = next_member(ulist, 0, U, tile_mask[t]);
-        st[t] = (ntile[t] > 0) ? NEED_S : DONE;
-      }
-      const uint32_t q_base = smem_u32(q_smem);
-      const uint32_t stage_base = smem_u32(stage_smem);
-      // Landing of the K/V stages is observed strictly in union order, for
-      // every entry, whichever tile keeps it.  A tile skips entries it does not
-      // keep, so testing only its own entry could confuse phase k of a slot
-      // with phase k-2 (a parity wait cannot tell them apart); observing in
-      // order guarantees phase k-1 completed before phase k is tested.
-      int seen = 0;
-      uint64_t t_idle = 0;
-      uint32_t spins = 0;
-      while (ok && (st[0] != DONE || st[1] != DONE)) {
-        bool progress = false;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (st[t] == NEED_S) {
-            const int u = cur[t];
-            const int slot = u % NS;
-            while (seen <= u && mbar_test(&sh->full[seen % NS], (seen / NS) & 1)) ++seen;
-            if (seen > u) {
-              tc_fence_after();
-              const uint32_t qa = q_base + t * C::Q_BYTES;
-              const uint32_t ka = stage_base + slot * C::STAGE_BYTES;
-#pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off_q = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-                mma_ss(tmem + colS[t], sdesc_sw128(qa + off_q, 16, 1024), sdesc_sw128(ka + off_k, 16, 1024), idS,
-                       kk > 0 ? 1u : 0u);
-              }
-              tc_commit(&sh->s_full[t]);
-              st[t] = NEED_P;
-              progress = true;
-            }
-          }
-          if (st[t] == NEED_P) {
-            if (mbar_test(&sh->p_full[t], n[t] & 1)) {
-              tc_fence_after();
-              const int u = cur[t];
-              const int slot = u % NS;
-              const uint32_t va = stage_base + slot * C::STAGE_BYTES + C::KV_BYTES;
-#pragma unroll
-              for (int kk = 0; kk < BN / 16; ++kk) {
-                mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, sdesc_sw128(va + kk * 2048, BN * 128, 1024), idPV,
-                       (n[t] > 0 || kk > 0) ? 1u : 0u);
-              }
-              const int o = 1 - t;
-              const bool other_member = ((ulist[u] >> 12) & tile_mask[o]) != 0;
-              if (!other_member || st[o] == DONE || cur[o] > u) tc_commit(&sh->empty[slot]);
-              ++n[t];
-              cur[t] = next_member(ulist, u + 1, U, tile_mask[t]);
-              if (n[t] == ntile[t]) {
-                tc_commit(&sh->o_full[t]);
-                st[t] = DONE;
-              } else {
-                st[t] = NEED_S;
-              }
-              progress = true;
-            }
-          }
+      int n = 0;
+      for (int u = 0; ok && u < U; ++u) {
+        const bool member = ((ulist[u] >> 12) & tile_mask[t]) != 0;
+        const int sk = u % NSK, sv = u % NSV;
+        if (!(ok = warp_wait(&sh->full_k[sk], (u / NSK) & 1, sh, prm))) break;
+        if (!member) {
+          // not this tile's block: observe both landings, release both slots
+          if (lane == 0) mbar_arrive(&sh->empty_k[sk]);
+          if (!(ok = warp_wait(&sh->full_v[sv], (u / NSV) & 1, sh, prm))) break;
+          if (lane == 0) mbar_arrive(&sh->empty_v[sv]);
+          continue;
         }
-        if (progress) {
-          spins = 0;
-          t_idle = 0;
-        } else if ((++spins & 63) == 0) {
-          const uint64_t now = globaltimer_ns();
-          if (t_idle == 0) t_idle = now;
-          if (sh->abort_flag) ok = false;
-          if (now - t_idle > kTimeoutNs) {
-            sh->abort_flag = 1;
-            flag_status(prm, BSA_DEV_TIMEOUT);
-            ok = false;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t ka = k_base + sk * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off_q = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+            const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+            mma_ss(tmem + colS, sdesc_sw128(qa + off_q, 16, 1024), sdesc_sw128(ka + off_k, 16, 1024), idS,
+                   kk > 0 ? 1u : 0u);
           }
+          tc_commit(&sh->s_full[t]);
+          tc_commit(&sh->empty_k[sk]);
+        }
+        __syncwarp();
+        if (!(ok = warp_wait(&sh->p_full[t], n & 1, sh, prm))) break;
+        if (!(ok = warp_wait(&sh->full_v[sv], (u / NSV) & 1, sh, prm))) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t va = v_base + sv * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ts(tmem + colO, tmem + colS + kk * 8, sdesc_sw128(va + kk * 2048, BN * 128, 1024), idPV,
+                   (n > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&sh->empty_v[sv]);
+        }
+        __syncwarp();
+        ++n;
+      }
+      if (lane == 0) {
+        if (ok && n > 0) tc_commit(&sh->o_full[t]);
+        if (!ok) {
+          // no MMA of this thread may still write TMEM when it is released
+          tc_commit(&sh->drain[t]);
+          drain_wait(&sh->drain[t], 0);
         }
       }
-      if (!ok) {
-        // make sure no MMA is still writing TMEM before it is released
-        tc_commit(&sh->drain);
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try(&sh->drain, 0) && globaltimer_ns() - t0 < kTimeoutNs / 4) {
-        }
-      }
+      __syncwarp();
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------ softmax + epilogue
+    setmaxnreg_inc<kRegsSoftmax>();
     const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
@@ -395,30 +404,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kb = e & 0xFFF;
       const bool row_ok = ((e >> 12) & my_bit) != 0;
       const int valid = (kb == NB - 1) ? (L - kb * BN) : BN;
-      ok = wait_bounded(&sh->s_full[t], n & 1, sh, prm);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
+      if (!(ok = warp_wait(&sh->s_full[t], n & 1, sh, prm))) break;
       tc_fence_after();
-      float s[BN];
+      // the whole score row of this thread: BN/32 loads, one wait
+      uint32_t sr[BN / 32][32];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t regs[32];
-        tmem_ld32(tS + c * 32, regs);
-        tmem_wait_ld();
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, sr[c]);
+      tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(regs[i]);
+      for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) reg_fence(sr[c][i]);
+      // masked blocks only: the ragged last key block, or a row half that
+      // does not keep this block (blk = 64)
+      if (!row_ok || valid < BN) {
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (!row_ok || c * 32 + i >= valid) sr[c][i] = __float_as_uint(-INFINITY);
       }
+      // raw row max (the scale is positive, so it commutes with max)
       float mx = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < BN; ++j) {
-        float x = s[j] * sl2;
-        if (!row_ok || j >= valid) x = -INFINITY;
-        s[j] = x;
-        mx = fmaxf(mx, x);
-      }
-      const float m_new = fmaxf(m_ref, mx);
+      for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) mx = max3(mx, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+      const float m_new = fmaxf(m_ref, mx * sl2);
       const bool resc = m_new > m_ref + kRescaleThreshold;
       float factor = 1.f;
       if (resc) {
@@ -430,31 +442,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O of this tile is final for block n-1: s_full of block n is
         // committed after the PV MMA of block n-1.
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t regs[32];
-          tmem_ld32(tO + c * 32, regs);
+        for (int h2 = 0; h2 < D / 64; ++h2) {
+          uint32_t o0[32], o1[32];
+          tmem_ld32(tO + h2 * 64, o0);
+          tmem_ld32(tO + h2 * 64 + 32, o1);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) regs[i] = __float_as_uint(__uint_as_float(regs[i]) * factor);
-          tmem_st32(tO + c * 32, regs);
+          for (int i = 0; i < 32; ++i) {
+            reg_fence(o0[i]);
+            reg_fence(o1[i]);
+            o0[i] = __float_as_uint(__uint_as_float(o0[i]) * factor);
+            o1[i] = __float_as_uint(__uint_as_float(o1[i]) * factor);
+          }
+          tmem_st32(tO + h2 * 64, o0);
+          tmem_st32(tO + h2 * 64 + 32, o1);
         }
         tmem_wait_st();
       }
+      // p = 2^(s*scale - m): one packed FMA per pair, ex2 on the MUFU unit,
+      // packed row sums, bf16 pairs written over the first half of S
       const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float rs = 0.f;
+      const uint64_t scale2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-mu, -mu);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(s[c * 64 + 2 * i] - mu);
-          const float p1 = ex2_approx(s[c * 64 + 2 * i + 1] - mu);
-          rs += p0 + p1;
+          const int col = c * 64 + 2 * i;
+          const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[col >> 5][col & 31]),
+                                            __uint_as_float(sr[col >> 5][(col & 31) + 1])),
+                                    scale2, negm2);
+          float x0, x1;
+          f2_unpack(x, x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st32(tS + c * 32, pk);
       }
-      l += rs;
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+        f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
+        l += (a0 + a1) + (b0 + b1);
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sh->p_full[t]);
@@ -463,8 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ----------------------------------------------------------- epilogue
     bool have_o = ok && ntile[t] > 0;
     if (have_o) {
-      have_o = wait_bounded(&sh->o_full[t], 0, sh, prm);
-      have_o = __all_sync(0xffffffffu, have_o);
+      have_o = warp_wait(&sh->o_full[t], 0, sh, prm);
       tc_fence_after();
     }
     if (ok) {
@@ -480,6 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (have_o) {
           tmem_ld32(tO + c * 32, regs);
           tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) reg_fence(regs[i]);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) regs[i] = 0u;
@@ -518,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 3) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
