@@ -17,32 +17,37 @@
 // With blk = 64 one 128-row tile spans two query blocks; rows of the half that
 // does not keep a block are masked to -inf for that block.
 //
-// Warp roles (12 warps):
-//   warp 0      TMA producer of Q (once) and of K for every union entry
-//   warp 3      TMA producer of V for every union entry; TMEM allocation
-//   warp 1 / 2  MMA issuer of tile 0 / tile 1: S_t = Q_t K^T (both operands
-//               in shared memory, K-major) into TMEM, then O_t += P_t V with
-//               P_t read from TMEM and V MN-major in shared memory
-//   warps 4-7   softmax + epilogue of tile 0 (one thread per query row)
-//   warps 8-11  softmax + epilogue of tile 1
-// K and V have separate rings, so a K slot is refilled as soon as the S
-// MMAs that read it are done, without waiting for the PV MMAs.
-// TMEM columns: S0 | S1 | O0 | O1.  P_t (bf16, packed in pairs) overwrites the
-// first BN/2 columns of S_t once S_t has been read; the next S_t is issued by
-// the same thread after the PV that reads P_t, so the tensor pipe's issue
-// order protects P_t.
+// Half blocks.  Scores are produced and consumed in 64-key halves, and every
+// tile has two S buffers in TMEM, so the tensor core computes S for half h+1
+// (and h+2) while the softmax works on half h: a tile never waits for its own
+// PV -> S round trip.  P of half h (bf16 pairs) overwrites the first 32
+// columns of its S buffer; S of half h+2 reuses the buffer only after the PV
+// of half h has completed.
 //
-// Every role walks the union in order and waits on every entry, member or
-// not: a parity wait cannot tell phase k of a barrier from phase k-2, so a
-// thread that skipped entries could take an older phase for the one it wants.
-// An MMA warp that does not compute an entry still observes its landing and
-// releases its slot with a plain arrive, so each release barrier always gets
-// exactly one arrival per MMA warp and entry.
+// Warp roles (16 warps):
+//   warp 0        TMA: Q (once), then K of every union entry (ring of NSK)
+//   warp 1        TMA: V of every union entry (ring of NSV)
+//   warp 2 / 12   S issuer of tile 0 / 1: S_h = Q K_h^T, K-major operands in
+//                 shared memory, fp32 accumulator in TMEM
+//   warp 3 / 13   PV issuer of tile 0 / 1: O += P_h V_h, P from TMEM, V
+//                 MN-major in shared memory
+//   warp 14       TMEM allocation
+//   warps 4-7     softmax + epilogue of tile 0 (one thread per query row)
+//   warps 8-11    softmax + epilogue of tile 1
+// TMEM columns: S0a S0b | S1a S1b | O0 | O1.
+//
+// Every issuer walks the union in order and waits on every entry's landing,
+// member or not: a parity wait cannot tell phase k of a barrier from phase
+// k-2, so a thread that skipped entries could take an older phase for the one
+// it wants.  For an entry its tile does not keep, an issuer releases the slot
+// with a plain arrive, so each release barrier gets exactly one arrival per
+// issuer of that ring (two) and entry.
 //
 // Online softmax in the log2 domain in fp32.  The running max used for the
-// exponentials is only raised when the block max exceeds it by more than 8
-// (so P <= 2^8); O in TMEM is rescaled only then, and the final 1/l uses the
-// same reference, so the result is exact up to rounding.
+// exponentials is only raised when a half-block max exceeds it by more than 8
+// (so P <= 2^8); O in TMEM is rescaled only then (after the previous PV has
+// completed), and the final 1/l uses the same reference, so the result is
+// exact up to rounding.
 //
 // Every wait is bounded (2 s of globaltimer); a timeout sets BSA_DEV_TIMEOUT
 // in the caller's status word, aborts the CTA's pipeline, drains what is in
@@ -61,14 +66,15 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int BM = 128;                         // query rows per tile
+constexpr int SN = 64;                          // keys per half block (S buffer width)
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
 constexpr float kRescaleThreshold = 8.0f;       // log2 units
-constexpr int kRegsLaunch = 168;                // 65536 / 384, rounded down to a multiple of 8
-constexpr int kRegsCtl = 72;
-constexpr int kRegsSoftmax = 216;
-static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split exceeds launch");
+constexpr int kRegsLaunch = 128;                // 65536 / 512
+constexpr int kRegsCtl = 56;
+constexpr int kRegsSoftmax = 200;
+static_assert(256 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split exceeds launch");
 
 struct Params {
   const int32_t* kept_idx;
@@ -86,10 +92,11 @@ struct Params {
 template <int D, int BN>
 struct Cfg {
   static constexpr int G = BM / BN;               // query blocks per 128-row tile
+  static constexpr int HB = BN / SN;              // halves per key block
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;     // one K or one V tile
   static constexpr int UNION_BYTES = kMaxNB * 2;  // uint16 per union entry
-  static constexpr int MISC_BYTES = 256;          // barriers and scalars
+  static constexpr int MISC_BYTES = 512;          // barriers and scalars
   static constexpr int SLOTS = (227 * 1024 - 1024 - 2 * Q_BYTES - UNION_BYTES - MISC_BYTES) / KV_BYTES;
   static constexpr int NSK = ((SLOTS + 1) / 2) > 4 ? 4 : (SLOTS + 1) / 2;
   static constexpr int NSV = (SLOTS / 2) > 4 ? 4 : SLOTS / 2;
@@ -101,8 +108,8 @@ struct Cfg {
   static constexpr int OFF_UNION = OFF_V + NSV * KV_BYTES;
   static constexpr int OFF_MISC = OFF_UNION + UNION_BYTES;
   static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
-  static constexpr int COL_S0 = 0, COL_S1 = BN, COL_O0 = 2 * BN, COL_O1 = 2 * BN + D;
-  static constexpr int TMEM_COLS = (2 * BN + 2 * D) <= 256 ? 256 : 512;
+  static constexpr int COL_O = 4 * SN;                            // O_t at COL_O + t*D
+  static constexpr int TMEM_COLS = 512;
   static constexpr int PANELS = D / 64;
 };
 
@@ -113,16 +120,17 @@ struct Shared {
   uint64_t full_v[4];
   uint64_t empty_v[4];
   uint64_t q_full;
-  uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t s_full[2][2];   // [tile][buffer]
+  uint64_t p_full[2][2];
+  uint64_t pv_done[2][2];
   uint64_t o_full[2];
-  uint64_t drain[2];
+  uint64_t drain[4];
   uint32_t tmem_base;
   uint32_t n_union;
   uint32_t n_tile[2];
   volatile int abort_flag;
 };
-static_assert(sizeof(Shared) <= 256, "misc region too small");
+static_assert(sizeof(Shared) <= 512, "misc region too small");
 
 __device__ __forceinline__ void flag_status(const Params& prm, int bits) {
   if (prm.status) atomicOr(prm.status, bits);
@@ -165,7 +173,7 @@ __device__ __forceinline__ int next_member(const uint16_t* ulist, int i, int U, 
 }
 
 // TMA producer of one operand ring (K or V): entry u goes to slot u % NS once
-// both MMA warps released the slot's previous entry.
+// both issuers of the ring released the slot's previous entry.
 template <int D, int BN, int NS>
 __device__ __forceinline__ void produce_ring(const CUtensorMap* map, uint8_t* ring, uint64_t* full, uint64_t* empty,
                                              const uint16_t* ulist, int U, int bh, int lane, Shared* sh,
@@ -187,7 +195,7 @@ __device__ __forceinline__ void produce_ring(const CUtensorMap* map, uint8_t* ri
   }
   if (sh->abort_flag && lane == 0) {
     // load k of a slot is issued only after release k-1, which follows the
-    // consumers' observation of landing k-1: the parity below is exact
+    // issuers' observation of landing k-1: the parity below is exact
     for (int u = issued - NS < 0 ? 0 : issued - NS; u < issued; ++u) drain_wait(&full[u % NS], (u / NS) & 1);
   }
 }
@@ -198,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmV, const Params prm) {
   using C = Cfg<D, BN>;
   constexpr int G = C::G;
+  constexpr int HB = C::HB;
   constexpr int NSK = C::NSK;
   constexpr int NSV = C::NSV;
   extern __shared__ uint8_t smem_raw[];
@@ -223,13 +232,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh->empty_k[s], 2);
       mbar_init(&sh->full_v[s], 1);
       mbar_init(&sh->empty_v[s], 2);
+      mbar_init(&sh->drain[s], 1);
     }
     mbar_init(&sh->q_full, 1);
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&sh->s_full[t], 1);
-      mbar_init(&sh->p_full[t], 128);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&sh->s_full[t][b], 1);
+        mbar_init(&sh->p_full[t][b], 128);
+        mbar_init(&sh->pv_done[t][b], 1);
+      }
       mbar_init(&sh->o_full[t], 1);
-      mbar_init(&sh->drain[t], 1);
     }
     sh->abort_flag = 0;
     fence_mbar_init();
@@ -239,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  if (warp == 3) {
+  if (warp == 14) {
     tmem_alloc(&sh->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
     tc_fence_before();
@@ -298,9 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntile[2] = {static_cast<int>(sh->n_tile[0]), static_cast<int>(sh->n_tile[1])};
   const uint32_t tile_mask[2] = {(1u << G) - 1u, ((1u << G) - 1u) << G};
 
-  if (warp < 4) {
-    // Registers: warpgroup 0 (TMA, MMA issue, TMEM allocation) needs few; the
-    // two softmax warpgroups hold a whole score row each.
+  if (warp < 4 || warp >= 12) {
+    // Registers: the control warpgroups (TMA, MMA issue, TMEM allocation)
+    // need few; the two softmax warpgroups hold score rows.
     setmaxnreg_dec<kRegsCtl>();
     if (warp == 0 && U > 0) {
       // ------------------------------------------------ TMA: Q, then K ring
@@ -318,67 +330,90 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       produce_ring<D, BN, NSK>(&tmK, k_ring, sh->full_k, sh->empty_k, ulist, U, bh, lane, sh, prm);
-    } else if (warp == 3 && U > 0) {
+    } else if (warp == 1 && U > 0) {
       // ------------------------------------------------------ TMA: V ring
       produce_ring<D, BN, NSV>(&tmV, v_ring, sh->full_v, sh->empty_v, ulist, U, bh, lane, sh, prm);
-    } else if ((warp == 1 || warp == 2) && U > 0) {
-      // ----------------------------------------- MMA issue, one tile each
-      const int t = warp - 1;
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
-      constexpr uint32_t idPV = idesc_bf16_f32(BM, D, false, true);
-      const uint32_t colS = t == 0 ? C::COL_S0 : C::COL_S1;
-      const uint32_t colO = t == 0 ? C::COL_O0 : C::COL_O1;
+    } else if ((warp == 2 || warp == 12) && U > 0) {
+      // ------------------------------------------- S issuer of one tile
+      const int t = warp == 2 ? 0 : 1;
+      constexpr uint32_t idS = idesc_bf16_f32(BM, SN, false, false);
       const uint32_t qa = smem_u32(q_smem) + t * C::Q_BYTES;
       const uint32_t k_base = smem_u32(k_ring);
-      const uint32_t v_base = smem_u32(v_ring);
       bool ok = ntile[t] == 0 || warp_wait(&sh->q_full, 0, sh, prm);
       tc_fence_after();
-      int n = 0;
+      int h = 0;
       for (int u = 0; ok && u < U; ++u) {
-        const bool member = ((ulist[u] >> 12) & tile_mask[t]) != 0;
-        const int sk = u % NSK, sv = u % NSV;
+        const int sk = u % NSK;
         if (!(ok = warp_wait(&sh->full_k[sk], (u / NSK) & 1, sh, prm))) break;
-        if (!member) {
-          // not this tile's block: observe both landings, release both slots
-          if (lane == 0) mbar_arrive(&sh->empty_k[sk]);
-          if (!(ok = warp_wait(&sh->full_v[sv], (u / NSV) & 1, sh, prm))) break;
-          if (lane == 0) mbar_arrive(&sh->empty_v[sv]);
+        if (((ulist[u] >> 12) & tile_mask[t]) == 0) {
+          if (lane == 0) mbar_arrive(&sh->empty_k[sk]);  // not this tile's block
           continue;
         }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t ka = k_base + sk * C::KV_BYTES;
+        for (int j = 0; j < HB; ++j, ++h) {
+          const int b = h & 1;
+          // S_h reuses buffer b: P_{h-2} in it must have been consumed
+          if (h >= 2 && !(ok = warp_wait(&sh->pv_done[t][b], ((h - 2) >> 1) & 1, sh, prm))) break;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t ka = k_base + sk * C::KV_BYTES + j * (SN * 128);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off_q = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-            const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-            mma_ss(tmem + colS, sdesc_sw128(qa + off_q, 16, 1024), sdesc_sw128(ka + off_k, 16, 1024), idS,
-                   kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off_q = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+              const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+              mma_ss(tmem + t * 2 * SN + b * SN, sdesc_sw128(qa + off_q, 16, 1024),
+                     sdesc_sw128(ka + off_k, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&sh->s_full[t][b]);
           }
-          tc_commit(&sh->s_full[t]);
-          tc_commit(&sh->empty_k[sk]);
+          __syncwarp();
         }
+        if (!ok) break;
+        if (lane == 0) tc_commit(&sh->empty_k[sk]);
         __syncwarp();
-        if (!(ok = warp_wait(&sh->p_full[t], n & 1, sh, prm))) break;
+      }
+      if (lane == 0 && !ok) {
+        tc_commit(&sh->drain[t]);
+        drain_wait(&sh->drain[t], 0);
+      }
+      __syncwarp();
+    } else if ((warp == 3 || warp == 13) && U > 0) {
+      // ------------------------------------------ PV issuer of one tile
+      const int t = warp == 3 ? 0 : 1;
+      constexpr uint32_t idPV = idesc_bf16_f32(BM, D, false, true);
+      const uint32_t v_base = smem_u32(v_ring);
+      const uint32_t colO = C::COL_O + t * D;
+      bool ok = true;
+      int h = 0;
+      for (int u = 0; ok && u < U; ++u) {
+        const int sv = u % NSV;
         if (!(ok = warp_wait(&sh->full_v[sv], (u / NSV) & 1, sh, prm))) break;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t va = v_base + sv * C::KV_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            mma_ts(tmem + colO, tmem + colS + kk * 8, sdesc_sw128(va + kk * 2048, BN * 128, 1024), idPV,
-                   (n > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(&sh->empty_v[sv]);
+        if (((ulist[u] >> 12) & tile_mask[t]) == 0) {
+          if (lane == 0) mbar_arrive(&sh->empty_v[sv]);  // not this tile's block
+          continue;
         }
+        for (int j = 0; j < HB; ++j, ++h) {
+          const int b = h & 1;
+          if (!(ok = warp_wait(&sh->p_full[t][b], (h >> 1) & 1, sh, prm))) break;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t va = v_base + sv * C::KV_BYTES + j * (SN * 128);
+#pragma unroll
+            for (int kk = 0; kk < SN / 16; ++kk)
+              mma_ts(tmem + colO, tmem + t * 2 * SN + b * SN + kk * 8,
+                     sdesc_sw128(va + kk * 2048, BN * 128, 1024), idPV, (h > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&sh->pv_done[t][b]);
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (lane == 0) tc_commit(&sh->empty_v[sv]);
         __syncwarp();
-        ++n;
       }
       if (lane == 0) {
-        if (ok && n > 0) tc_commit(&sh->o_full[t]);
+        if (ok && h > 0) tc_commit(&sh->o_full[t]);
         if (!ok) {
-          // no MMA of this thread may still write TMEM when it is released
-          tc_commit(&sh->drain[t]);
-          drain_wait(&sh->drain[t], 0);
+          tc_commit(&sh->drain[2 + t]);
+          drain_wait(&sh->drain[2 + t], 0);
         }
       }
       __syncwarp();
@@ -390,8 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + (t == 0 ? C::COL_S0 : C::COL_S1);
-    const uint32_t tO = tmem + lane_off + (t == 0 ? C::COL_O0 : C::COL_O1);
+    const uint32_t tS = tmem + lane_off + t * 2 * SN;  // + b * SN
+    const uint32_t tO = tmem + lane_off + C::COL_O + t * D;
     const int grow = (pair * 2 + t) * BM + r;
     const uint32_t my_bit = 1u << (t * G + r / BN);
     const float sl2 = prm.scale_log2;
@@ -399,78 +434,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l = 0.f;
     bool ok = true;
     int u = next_member(ulist, 0, U, tile_mask[t]);
-    for (int n = 0; n < ntile[t]; ++n) {
+    int h = 0;
+    for (int n = 0; ok && n < ntile[t]; ++n) {
       const uint32_t e = ulist[u];
       const int kb = e & 0xFFF;
       const bool row_ok = ((e >> 12) & my_bit) != 0;
       const int valid = (kb == NB - 1) ? (L - kb * BN) : BN;
-      if (!(ok = warp_wait(&sh->s_full[t], n & 1, sh, prm))) break;
-      tc_fence_after();
-      // the whole score row of this thread: BN/32 loads, one wait
-      uint32_t sr[BN / 32][32];
+      for (int j = 0; j < HB; ++j, ++h) {
+        const int b = h & 1;
+        const int valid_h = valid - j * SN;  // may be <= 0: the whole half is padding
+        if (!(ok = warp_wait(&sh->s_full[t][b], (h >> 1) & 1, sh, prm))) break;
+        tc_fence_after();
+        uint32_t sr[2][32];
+        tmem_ld32(tS + b * SN, sr[0]);
+        tmem_ld32(tS + b * SN + 32, sr[1]);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, sr[c]);
-      tmem_wait_ld();
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
+          for (int i = 0; i < 32; ++i) reg_fence(sr[c][i]);
+        // masked halves only: the ragged last key block, or a row half that
+        // does not keep this block (blk = 64)
+        if (!row_ok || valid_h < SN) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) reg_fence(sr[c][i]);
-      // masked blocks only: the ragged last key block, or a row half that
-      // does not keep this block (blk = 64)
-      if (!row_ok || valid < BN) {
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (!row_ok || c * 32 + i >= valid) sr[c][i] = __float_as_uint(-INFINITY);
-      }
-      // raw row max (the scale is positive, so it commutes with max)
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) mx = max3(mx, __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
-      const float m_new = fmaxf(m_ref, mx * sl2);
-      const bool resc = m_new > m_ref + kRescaleThreshold;
-      float factor = 1.f;
-      if (resc) {
-        factor = ex2_approx(m_ref - m_new);  // 0 when m_ref is -inf
-        l *= factor;
-        m_ref = m_new;
-      }
-      if (n > 0 && __any_sync(0xffffffffu, resc)) {
-        // O of this tile is final for block n-1: s_full of block n is
-        // committed after the PV MMA of block n-1.
-#pragma unroll
-        for (int h2 = 0; h2 < D / 64; ++h2) {
-          uint32_t o0[32], o1[32];
-          tmem_ld32(tO + h2 * 64, o0);
-          tmem_ld32(tO + h2 * 64 + 32, o1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            reg_fence(o0[i]);
-            reg_fence(o1[i]);
-            o0[i] = __float_as_uint(__uint_as_float(o0[i]) * factor);
-            o1[i] = __float_as_uint(__uint_as_float(o1[i]) * factor);
-          }
-          tmem_st32(tO + h2 * 64, o0);
-          tmem_st32(tO + h2 * 64 + 32, o1);
+            for (int i = 0; i < 32; ++i)
+              if (!row_ok || c * 32 + i >= valid_h) sr[c][i] = __float_as_uint(-INFINITY);
         }
-        tmem_wait_st();
-      }
-      // p = 2^(s*scale - m): one packed FMA per pair, ex2 on the MUFU unit,
-      // packed row sums, bf16 pairs written over the first half of S
-      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-      const uint64_t scale2 = f2_pack(sl2, sl2);
-      const uint64_t negm2 = f2_pack(-mu, -mu);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        // raw max (the scale is positive, so it commutes with max), 4 chains
+        float mxa = -INFINITY, mxb = -INFINITY, mxc = -INFINITY, mxd = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) {
+        for (int i = 0; i < 32; i += 4) {
+          mxa = max3(mxa, __uint_as_float(sr[0][i]), __uint_as_float(sr[0][i + 1]));
+          mxb = max3(mxb, __uint_as_float(sr[0][i + 2]), __uint_as_float(sr[0][i + 3]));
+          mxc = max3(mxc, __uint_as_float(sr[1][i]), __uint_as_float(sr[1][i + 1]));
+          mxd = max3(mxd, __uint_as_float(sr[1][i + 2]), __uint_as_float(sr[1][i + 3]));
+        }
+        const float mx = fmaxf(max3(mxa, mxb, mxc), mxd);
+        const float m_new = fmaxf(m_ref, mx * sl2);
+        const bool resc = m_new > m_ref + kRescaleThreshold;
+        float factor = 1.f;
+        if (resc) {
+          factor = ex2_approx(m_ref - m_new);  // 0 when m_ref is -inf
+          l *= factor;
+          m_ref = m_new;
+        }
+        if (h > 0 && __any_sync(0xffffffffu, resc)) {
+          // O must be final for half h-1 before it is rescaled (PV_h waits
+          // for this half's P, so nothing newer can touch O meanwhile)
+          if (!(ok = warp_wait(&sh->pv_done[t][(h - 1) & 1], ((h - 1) >> 1) & 1, sh, prm))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int h2 = 0; h2 < D / 64; ++h2) {
+            uint32_t o0[32], o1[32];
+            tmem_ld32(tO + h2 * 64, o0);
+            tmem_ld32(tO + h2 * 64 + 32, o1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              reg_fence(o0[i]);
+              reg_fence(o1[i]);
+              o0[i] = __float_as_uint(__uint_as_float(o0[i]) * factor);
+              o1[i] = __float_as_uint(__uint_as_float(o1[i]) * factor);
+            }
+            tmem_st32(tO + h2 * 64, o0);
+            tmem_st32(tO + h2 * 64 + 32, o1);
+          }
+          tmem_wait_st();
+        }
+        // p = 2^(s*scale - m): one packed FMA per pair, ex2 on the MUFU unit,
+        // packed row sums, bf16 pairs written over the first half of S
+        const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const uint64_t scale2 = f2_pack(sl2, sl2);
+        const uint64_t negm2 = f2_pack(-mu, -mu);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int col = c * 64 + 2 * i;
+          const int col = 2 * i;
           const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[col >> 5][col & 31]),
                                             __uint_as_float(sr[col >> 5][(col & 31) + 1])),
                                     scale2, negm2);
@@ -481,17 +523,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(tS + c * 32, pk);
+        tmem_st32(tS + b * SN, pk);
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+          f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
+          l += (a0 + a1) + (b0 + b1);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sh->p_full[t][b]);
       }
-      {
-        float a0, a1, b0, b1;
-        f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
-        f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
-        l += (a0 + a1) + (b0 + b1);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&sh->p_full[t]);
       u = next_member(ulist, u + 1, U, tile_mask[t]);
     }
     // ----------------------------------------------------------- epilogue
@@ -505,8 +547,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const float lse_v = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       const size_t row_elem = (static_cast<size_t>(bh) * L + (store ? grow : 0)) * D;
-      const int h = bh % prm.H;
-      const float a = prm.R ? prm.alpha[h] : 0.f;
+      const int hh = bh % prm.H;
+      const float a = prm.R ? prm.alpha[hh] : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t regs[32];
@@ -553,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncthreads();
-  if (warp == 3) {
+  if (warp == 14) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
