@@ -669,12 +669,17 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-int launch_sparse_attn(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
+int launch_sparse_attn_pair(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   if (s.D == 128 && s.blk == 128) return run<128, 128>(s, a, st);
   if (s.D == 128 && s.blk == 64) return run<128, 64>(s, a, st);
   if (s.D == 64 && s.blk == 128) return run<64, 128>(s, a, st);
   if (s.D == 64 && s.blk == 64) return run<64, 64>(s, a, st);
   return BSA_ESHAPE;
+}
+
+int launch_sparse_attn(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
+  if (s.blk == 128) return launch_sparse_attn_tile(s, a, st);
+  return launch_sparse_attn_pair(s, a, st);
 }
 
 }  // namespace bsa

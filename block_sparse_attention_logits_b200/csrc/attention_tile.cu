@@ -1,0 +1,757 @@
+// Block-sparse attention forward for sm_100a, 128-token key blocks:
+// persistent, one 128-row query tile at a time per CTA (one CTA per SM).
+//
+// What it computes (CalibAtt abstract and Fig. 5(b): compute the selected
+// block connections exactly and skip the unselected ones; RECAP section 4.1:
+// block-sparse attention for the selected interactions, dense attention for
+// refreshes; RECAP section 1: a cached dense refinement corrects the sparse
+// output): for every query row r of query block i,
+//     O[r] = softmax over the keys of the kept blocks K(i) of (q_r.k_c/sqrt(D)) . V
+//     LSE[r] = log-sum-exp of those logits,
+// optionally followed by O <- O + alpha_h * R in the epilogue.
+//
+// Schedule.  Work item w = (b*H + h) * NT + query block.  CTAs take items
+// from one atomic counter, in order, so the items in flight at any time are
+// neighbouring query blocks of the same head (its K/V stays in L2) and uneven
+// kept lists do not unbalance the SMs.  The TMA-Q/K warp fetches the next item
+// and passes it to the other roles through a 4-deep queue in shared memory.
+// The counter lives in a slot of a small in-library ring (one slot per launch,
+// round robin); the last CTA of a launch resets its slot, so each launch finds
+// its slot at zero as long as fewer than kSchedSlots launches overlap.
+//
+// Tensor memory (512 columns): S0 | S1 | O0 | O1.  S is double buffered, so
+// the tensor core computes S for block n+1 while the softmax works on block
+// n; O is double buffered across work items, so the epilogue of one item
+// overlaps the next.  All MMAs are M=128, N=128 (or N=D), K=16: full-rate
+// shapes.  P of block n (bf16 pairs) overwrites the first 64 columns of its S
+// buffer; S of block n+2 reuses the buffer only after the PV of block n has
+// completed.
+//
+// Warp roles (16 warps):
+//   warp 0       item queue; TMA: Q of every item (double buffered), K ring
+//   warp 1       TMA: V ring; TMEM allocation
+//   warp 2       S issuer:  S_n = Q K_n^T into S[n%2]
+//   warp 3       PV issuer: O[item%2] += P_n V_n, P read from TMEM
+//   warps 4-7    softmax of rows 32q+0..15 of every TMEM quarter q
+//   warps 8-11   softmax of rows 32q+16..31
+//   warps 12-15  epilogue: O/l (+ alpha*R) -> bf16, LSE
+// The softmax reads S with 16-lane TMEM loads: a thread holds two rows and,
+// per 8-key chunk, one adjacent key pair of each, which is exactly the bf16
+// pair of one P column; 4 threads share a row and combine maxima and sums with
+// two shuffles.  The two softmax warpgroups own disjoint rows and never wait
+// for each other, so one can exponentiate while the other loads.
+//
+// Online softmax in the log2 domain in fp32.  The reference max is only
+// raised when a block max exceeds it by more than 8 (so P <= 2^8); O is then
+// rescaled in TMEM (after the previous PV completed), and the final 1/l uses
+// the same reference.
+//
+// Every wait is bounded (2 s of globaltimer); a timeout sets BSA_DEV_TIMEOUT
+// in the caller's status word and makes every role give up; the MMA issuers
+// and TMA producers wait (bounded) for their operations in flight before TMEM
+// is released.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <atomic>
+#include <cmath>
+
+#include "internal.cuh"
+#include "sm100.cuh"
+
+namespace bsa {
+namespace tile_attn {
+
+using namespace sm100;
+
+constexpr int kThreads = 512;
+constexpr int BM = 128;                         // query rows per work item
+constexpr int BN = 128;                         // keys per block
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
+constexpr float kRescaleThreshold = 8.0f;       // log2 units
+constexpr int kQueue = 4;                       // item queue depth
+constexpr int kItemReaders = 32 * 3 + 256 + 128;  // threads of the roles that read the queue
+// registers per thread: launch 65536 / 512 = 128, then re-balanced per warpgroup
+constexpr int kRegsCtl = 56;        // TMA producers, MMA issuers
+constexpr int kRegsSoftmax = 168;   // two warpgroups
+constexpr int kRegsEpilogue = 120;
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax + 128 * kRegsEpilogue <= 512 * 128, "register split exceeds launch");
+
+// Work counters, one per launch in flight (round robin).  Zero at module
+// load; every launch leaves its slot at zero again.
+constexpr int kSchedSlots = 64;
+struct SchedSlot {
+  unsigned int next;
+  unsigned int done;
+  unsigned int pad[30];
+};
+__device__ SchedSlot g_sched[kSchedSlots];
+
+struct Params {
+  const int32_t* kept_idx;
+  const int32_t* kept_cnt;
+  const __nv_bfloat16* R;
+  const float* alpha;
+  __nv_bfloat16* o;
+  float* lse;
+  int32_t* status;
+  int H, L, NB, NT, n_work;
+  float scale_log2;
+  int dense;
+  int sched_slot;
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int STATS_BYTES = 2 * 2 * BM * 4;  // [item parity][l, m][row]
+  static constexpr int MISC_BYTES = 512;
+  static constexpr int SLOTS = (227 * 1024 - 1024 - 2 * Q_BYTES - STATS_BYTES - MISC_BYTES) / KV_BYTES;
+  static constexpr int NSK = ((SLOTS + 1) / 2) > 4 ? 4 : (SLOTS + 1) / 2;
+  static constexpr int NSV = (SLOTS / 2) > 4 ? 4 : SLOTS / 2;
+  static_assert(NSK >= 2 && NSV >= 2, "shared memory too small for double-buffered K and V");
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
+  static constexpr int OFF_STATS = OFF_V + NSV * KV_BYTES;
+  static constexpr int OFF_MISC = OFF_STATS + STATS_BYTES;
+  static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
+  static constexpr int COL_S = 0;        // S[b] at b*BN
+  static constexpr int COL_O = 2 * BN;   // O[j] at COL_O + j*D
+  static constexpr int PANELS = D / 64;
+};
+
+struct Shared {
+  uint64_t full_k[4], empty_k[4], full_v[4], empty_v[4];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t o_full[2], o_empty[2];
+  uint64_t stats_full[2], stats_free[2];
+  uint64_t drain[2];
+  uint64_t item_full[kQueue], item_empty[kQueue];
+  int items[kQueue];
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+static_assert(sizeof(Shared) <= 512, "misc region too small");
+
+__device__ __forceinline__ void flag_status(const Params& prm, int bits) {
+  if (prm.status) atomicOr(prm.status, bits);
+}
+
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Shared* sh, const Params& prm) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 15) == 0) {
+      if (sh->abort_flag) return false;
+      if (globaltimer_ns() - t0 > kTimeoutNs) {
+        sh->abort_flag = 1;
+        flag_status(prm, BSA_DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Shared* sh, const Params& prm) {
+  const bool ok = wait_bounded(bar, parity, sh, prm);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try(bar, parity) && globaltimer_ns() - t0 < kTimeoutNs) {
+  }
+}
+
+// Next work item of this CTA (queue position i), or -1 at the end / on abort.
+// Every reading thread releases its queue slot right after reading it.
+__device__ __forceinline__ int next_item(int i, Shared* sh, const Params& prm) {
+  const int qs = i % kQueue;
+  if (!warp_wait(&sh->item_full[qs], (i / kQueue) & 1, sh, prm)) return -1;
+  const int w = sh->items[qs];
+  mbar_arrive(&sh->item_empty[qs]);
+  return w;
+}
+
+// One work item: a 128-row query block of one (batch, head) and its key list.
+struct Item {
+  int bh, qb, cnt;
+  const int32_t* list;  // null in dense mode
+  bool bad_cnt;         // the count was outside [0, NB] and was clamped
+};
+
+__device__ __forceinline__ Item item_of(int w, const Params& prm) {
+  Item it;
+  it.bh = w / prm.NT;
+  it.qb = w - it.bh * prm.NT;
+  it.bad_cnt = false;
+  if (prm.dense) {
+    it.cnt = prm.NB;
+    it.list = nullptr;
+  } else {
+    const size_t r = static_cast<size_t>(it.bh) * prm.NB + it.qb;
+    const int c = __ldg(prm.kept_cnt + r);
+    it.bad_cnt = c < 0 || c > prm.NB;
+    it.cnt = c < 0 ? 0 : (c > prm.NB ? prm.NB : c);
+    it.list = prm.kept_idx + r * prm.NB;
+  }
+  return it;
+}
+
+// Key block of entry n, or -1 for an out-of-range entry (skipped by every role).
+__device__ __forceinline__ int entry_kb(const Item& it, int n, int NB) {
+  const int kb = it.list ? __ldg(it.list + n) : n;
+  return static_cast<unsigned>(kb) < static_cast<unsigned>(NB) ? kb : -1;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const Params prm) {
+  using C = Cfg<D>;
+  constexpr int NSK = C::NSK;
+  constexpr int NSV = C::NSV;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Shared* sh = reinterpret_cast<Shared*>(smem + C::OFF_MISC);
+  float* stats = reinterpret_cast<float*>(smem + C::OFF_STATS);
+  uint8_t* q_smem = smem + C::OFF_Q;
+  uint8_t* k_ring = smem + C::OFF_K;
+  uint8_t* v_ring = smem + C::OFF_V;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int NB = prm.NB;
+  const int L = prm.L;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&sh->full_k[s], 1);
+      mbar_init(&sh->empty_k[s], 1);
+      mbar_init(&sh->full_v[s], 1);
+      mbar_init(&sh->empty_v[s], 1);
+      mbar_init(&sh->item_full[s], 1);
+      mbar_init(&sh->item_empty[s], kItemReaders);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&sh->q_full[j], 1);
+      mbar_init(&sh->q_empty[j], 1);
+      mbar_init(&sh->s_full[j], 1);
+      mbar_init(&sh->p_full[j], 256);
+      mbar_init(&sh->pv_done[j], 1);
+      mbar_init(&sh->o_full[j], 1);
+      mbar_init(&sh->o_empty[j], 128);
+      mbar_init(&sh->stats_full[j], 256);
+      mbar_init(&sh->stats_free[j], 128);
+      mbar_init(&sh->drain[j], 1);
+    }
+    sh->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsCtl>();
+    if (warp == 0) {
+      // ---------------------------------- item queue, TMA: Q and the K ring
+      SchedSlot* sched = &g_sched[prm.sched_slot];
+      int u = 0;
+      bool ok = true;
+      for (int i = 0;; ++i) {
+        const int qs = i % kQueue;
+        if (i >= kQueue && !(ok = warp_wait(&sh->item_empty[qs], ((i / kQueue) - 1) & 1, sh, prm))) break;
+        int w = 0;
+        if (lane == 0) {
+          w = static_cast<int>(atomicAdd(&sched->next, 1u));
+          if (w >= prm.n_work) w = -1;
+          sh->items[qs] = w;
+          mbar_arrive(&sh->item_full[qs]);
+        }
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (w < 0) break;
+        const Item it = item_of(w, prm);
+        if (it.bad_cnt && lane == 0) flag_status(prm, BSA_DEV_BAD_INDEX);
+        const int qb = i & 1;
+        if (i >= 2 && !(ok = warp_wait(&sh->q_empty[qb], ((i - 2) >> 1) & 1, sh, prm))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sh->q_full[qb], C::Q_BYTES);
+          for (int pnl = 0; pnl < C::PANELS; ++pnl)
+            tma_load_3d(q_smem + qb * C::Q_BYTES + pnl * BM * 128, &tmQ, &sh->q_full[qb], pnl * 64, it.qb * BM,
+                        it.bh);
+        }
+        __syncwarp();
+        for (int n = 0; ok && n < it.cnt; ++n) {
+          const int kb = entry_kb(it, n, NB);
+          if (kb < 0) {
+            if (lane == 0) flag_status(prm, BSA_DEV_BAD_INDEX);
+            continue;
+          }
+          const int slot = u % NSK;
+          if (u >= NSK && !(ok = warp_wait(&sh->empty_k[slot], ((u / NSK) - 1) & 1, sh, prm))) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&sh->full_k[slot], C::KV_BYTES);
+            for (int pnl = 0; pnl < C::PANELS; ++pnl)
+              tma_load_3d(k_ring + slot * C::KV_BYTES + pnl * BN * 128, &tmK, &sh->full_k[slot], pnl * 64, kb * BN,
+                          it.bh);
+          }
+          __syncwarp();
+          ++u;
+        }
+        if (!ok) break;
+      }
+      if (!ok && lane == 0) {
+        for (int v = u - NSK < 0 ? 0 : u - NSK; v < u; ++v) drain_wait(&sh->full_k[v % NSK], (v / NSK) & 1);
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------ TMA: V ring
+      int u = 0;
+      bool ok = true;
+      for (int i = 0; ok; ++i) {
+        const int w = next_item(i, sh, prm);
+        if (w < 0) break;
+        const Item it = item_of(w, prm);
+        for (int n = 0; n < it.cnt; ++n) {
+          const int kb = entry_kb(it, n, NB);
+          if (kb < 0) continue;
+          const int slot = u % NSV;
+          if (u >= NSV && !(ok = warp_wait(&sh->empty_v[slot], ((u / NSV) - 1) & 1, sh, prm))) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&sh->full_v[slot], C::KV_BYTES);
+            for (int pnl = 0; pnl < C::PANELS; ++pnl)
+              tma_load_3d(v_ring + slot * C::KV_BYTES + pnl * BN * 128, &tmV, &sh->full_v[slot], pnl * 64, kb * BN,
+                          it.bh);
+          }
+          __syncwarp();
+          ++u;
+        }
+      }
+      if (!ok && lane == 0)
+        for (int v = u - NSV < 0 ? 0 : u - NSV; v < u; ++v) drain_wait(&sh->full_v[v % NSV], (v / NSV) & 1);
+      __syncwarp();
+    } else if (warp == 2) {
+      // ---------------------------------------------------------- S issuer
+      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
+      const uint32_t q_base = smem_u32(q_smem);
+      const uint32_t k_base = smem_u32(k_ring);
+      int u = 0;
+      bool ok = true;
+      for (int i = 0; ok; ++i) {
+        const int w = next_item(i, sh, prm);
+        if (w < 0) break;
+        const Item it = item_of(w, prm);
+        const int qb = i & 1;
+        if (!(ok = warp_wait(&sh->q_full[qb], (i >> 1) & 1, sh, prm))) break;
+        const uint32_t qa = q_base + qb * C::Q_BYTES;
+        for (int n = 0; n < it.cnt; ++n) {
+          if (entry_kb(it, n, NB) < 0) continue;
+          const int sk = u % NSK;
+          const int b = u & 1;
+          if (!(ok = warp_wait(&sh->full_k[sk], (u / NSK) & 1, sh, prm))) break;
+          if (u >= 2 && !(ok = warp_wait(&sh->pv_done[b], ((u - 2) >> 1) & 1, sh, prm))) break;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t ka = k_base + sk * C::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off_q = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+              const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+              mma_ss(tmem + C::COL_S + b * BN, sdesc_sw128(qa + off_q, 16, 1024), sdesc_sw128(ka + off_k, 16, 1024),
+                     idS, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&sh->s_full[b]);
+            tc_commit(&sh->empty_k[sk]);
+          }
+          __syncwarp();
+          ++u;
+        }
+        if (!ok) break;
+        if (lane == 0) tc_commit(&sh->q_empty[qb]);
+        __syncwarp();
+      }
+      if (!ok && lane == 0) {
+        tc_commit(&sh->drain[0]);
+        drain_wait(&sh->drain[0], 0);
+      }
+      __syncwarp();
+    } else {
+      // --------------------------------------------------------- PV issuer
+      constexpr uint32_t idPV = idesc_bf16_f32(BM, D, false, true);
+      const uint32_t v_base = smem_u32(v_ring);
+      int u = 0;
+      bool ok = true;
+      for (int i = 0; ok; ++i) {
+        const int w = next_item(i, sh, prm);
+        if (w < 0) break;
+        const Item it = item_of(w, prm);
+        const int ob = i & 1;
+        if (i >= 2 && !(ok = warp_wait(&sh->o_empty[ob], ((i - 2) >> 1) & 1, sh, prm))) break;
+        bool first = true;
+        for (int n = 0; n < it.cnt; ++n) {
+          if (entry_kb(it, n, NB) < 0) continue;
+          const int sv = u % NSV;
+          const int b = u & 1;
+          if (!(ok = warp_wait(&sh->p_full[b], (u >> 1) & 1, sh, prm))) break;
+          if (!(ok = warp_wait(&sh->full_v[sv], (u / NSV) & 1, sh, prm))) break;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t va = v_base + sv * C::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+              mma_ts(tmem + C::COL_O + ob * D, tmem + C::COL_S + b * BN + kk * 8,
+                     sdesc_sw128(va + kk * 2048, BN * 128, 1024), idPV, (!first || kk > 0) ? 1u : 0u);
+            tc_commit(&sh->pv_done[b]);
+            tc_commit(&sh->empty_v[sv]);
+          }
+          __syncwarp();
+          first = false;
+          ++u;
+        }
+        if (!ok) break;
+        if (lane == 0) tc_commit(&sh->o_full[ob]);
+        __syncwarp();
+      }
+      if (!ok && lane == 0) {
+        tc_commit(&sh->drain[1]);
+        drain_wait(&sh->drain[1], 0);
+      }
+      __syncwarp();
+    }
+  } else if (warp < 12) {
+    // ------------------------------------------------------------- softmax
+    setmaxnreg_inc<kRegsSoftmax>();
+    const int grp = (warp - 4) >> 2;     // 0: rows 32q+0..15, 1: rows 32q+16..31
+    const int quarter = warp & 3;
+    const int j4 = lane & 3;             // column slot within each chunk
+    const int rA = quarter * 32 + grp * 16 + (lane >> 2);  // the thread's two rows: rA, rA + 8
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32 + grp * 16) << 16;
+    const float sl2 = prm.scale_log2;
+    const uint64_t scale2 = f2_pack(sl2, sl2);
+    int u = 0;
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      const int w = next_item(i, sh, prm);
+      if (w < 0) break;
+      const Item it = item_of(w, prm);
+      const int ob = i & 1;
+      const uint32_t tO = tmem + lane_off + C::COL_O + ob * D;
+      float mA = -INFINITY, mB = -INFINITY;  // reference max of rows rA, rA+8 (log2 units)
+      float lA = 0.f, lB = 0.f;              // this thread's share of the row sums
+      int nt = 0;
+      for (int n = 0; n < it.cnt; ++n) {
+        const int kb = entry_kb(it, n, NB);
+        if (kb < 0) continue;
+        const int b = u & 1;
+        const uint32_t tS = tmem + lane_off + C::COL_S + b * BN;
+        if (!(ok = warp_wait(&sh->s_full[b], (u >> 1) & 1, sh, prm))) break;
+        tc_fence_after();
+        // s[chunk][0..1]: row rA, keys 8*chunk + 2*j4 + {0,1}; s[chunk][2..3]: row rA+8
+        uint32_t sr[2][32];
+        tmem_ld_16x256b_x8(tS, sr[0]);
+        tmem_ld_16x256b_x8(tS + 64, sr[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) reg_fence(sr[q][e]);
+        const int valid = kb == NB - 1 ? L - kb * BN : BN;
+        if (valid < BN) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int key = (q * 8 + (e >> 2)) * 8 + 2 * j4 + (e & 1);
+              if (key >= valid) sr[q][e] = __float_as_uint(-INFINITY);
+            }
+        }
+        float xa = -INFINITY, xb = -INFINITY, ya = -INFINITY, yb = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            xa = max3(xa, __uint_as_float(sr[q][e]), __uint_as_float(sr[q][e + 1]));
+            ya = max3(ya, __uint_as_float(sr[q][e + 2]), __uint_as_float(sr[q][e + 3]));
+            xb = max3(xb, __uint_as_float(sr[q][e + 4]), __uint_as_float(sr[q][e + 5]));
+            yb = max3(yb, __uint_as_float(sr[q][e + 6]), __uint_as_float(sr[q][e + 7]));
+          }
+        float mxA = fmaxf(xa, xb), mxB = fmaxf(ya, yb);
+        mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, 1));
+        mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, 1));
+        mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, 2));
+        mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, 2));
+        const float nA = fmaxf(mA, mxA * sl2), nB = fmaxf(mB, mxB * sl2);
+        const bool rsA = nA > mA + kRescaleThreshold, rsB = nB > mB + kRescaleThreshold;
+        float fA = 1.f, fB = 1.f;
+        if (rsA) {
+          fA = ex2_approx(mA - nA);  // 0 when mA is -inf
+          lA *= fA;
+          mA = nA;
+        }
+        if (rsB) {
+          fB = ex2_approx(mB - nB);
+          lB *= fB;
+          mB = nB;
+        }
+        if (nt > 0 && __any_sync(0xffffffffu, rsA || rsB)) {
+          // O must hold the previous block's PV before it is rescaled
+          if (!(ok = warp_wait(&sh->pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1, sh, prm))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int cc = 0; cc < D / 64; ++cc) {
+            uint32_t o[32];
+            tmem_ld_16x256b_x8(tO + cc * 64, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              reg_fence(o[e]);
+              o[e] = __float_as_uint(__uint_as_float(o[e]) * ((e & 2) ? fB : fA));
+            }
+            tmem_st_16x256b_x8(tO + cc * 64, o);
+          }
+          tmem_wait_st();
+        }
+        const uint64_t negA = f2_pack(mA == -INFINITY ? 0.f : -mA, mA == -INFINITY ? 0.f : -mA);
+        const uint64_t negB = f2_pack(mB == -INFINITY ? 0.f : -mB, mB == -INFINITY ? 0.f : -mB);
+        uint64_t accA0 = 0ull, accA1 = 0ull, accB0 = 0ull, accB1 = 0ull;
+        uint32_t pk[32];  // P columns 4*chunk + j4: {row rA, row rA+8} per chunk
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint32_t* c4 = &sr[k >> 3][(k & 7) * 4];
+          const uint64_t xA = f2_fma(f2_pack(__uint_as_float(c4[0]), __uint_as_float(c4[1])), scale2, negA);
+          const uint64_t xB = f2_fma(f2_pack(__uint_as_float(c4[2]), __uint_as_float(c4[3])), scale2, negB);
+          float a0, a1, b0, b1;
+          f2_unpack(xA, a0, a1);
+          f2_unpack(xB, b0, b1);
+          const float pa0 = ex2_approx(a0), pa1 = ex2_approx(a1);
+          const float pb0 = ex2_approx(b0), pb1 = ex2_approx(b1);
+          if (k & 1) {
+            accA1 = f2_add(accA1, f2_pack(pa0, pa1));
+            accB1 = f2_add(accB1, f2_pack(pb0, pb1));
+          } else {
+            accA0 = f2_add(accA0, f2_pack(pa0, pa1));
+            accB0 = f2_add(accB0, f2_pack(pb0, pb1));
+          }
+          pk[2 * k] = pack_bf16x2(pa0, pa1);
+          pk[2 * k + 1] = pack_bf16x2(pb0, pb1);
+        }
+        tmem_st_16x128b_x16(tS, pk);
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(f2_add(accA0, accA1), a0, a1);
+          f2_unpack(f2_add(accB0, accB1), b0, b1);
+          lA += a0 + a1;
+          lB += b0 + b1;
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sh->p_full[b]);
+        ++u;
+        ++nt;
+      }
+      if (!ok) break;
+      // full row sums, then hand the statistics of this item to the epilogue
+      lA += __shfl_xor_sync(0xffffffffu, lA, 1);
+      lB += __shfl_xor_sync(0xffffffffu, lB, 1);
+      lA += __shfl_xor_sync(0xffffffffu, lA, 2);
+      lB += __shfl_xor_sync(0xffffffffu, lB, 2);
+      if (i >= 2 && !(ok = warp_wait(&sh->stats_free[ob], ((i - 2) >> 1) & 1, sh, prm))) break;
+      float* st = stats + ob * 2 * BM;
+      if (j4 == 0) {
+        st[rA] = lA;
+        st[rA + 8] = lB;
+        st[BM + rA] = mA;
+        st[BM + rA + 8] = mB;
+      }
+      mbar_arrive(&sh->stats_full[ob]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    setmaxnreg_dec<kRegsEpilogue>();
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      const int w = next_item(i, sh, prm);
+      if (w < 0) break;
+      const Item it = item_of(w, prm);
+      const int ob = i & 1;
+      if (!(ok = warp_wait(&sh->o_full[ob], (i >> 1) & 1, sh, prm))) break;
+      if (!(ok = warp_wait(&sh->stats_full[ob], (i >> 1) & 1, sh, prm))) break;
+      tc_fence_after();
+      const float* st = stats + ob * 2 * BM;
+      const float l = st[r];
+      const float m_ref = st[BM + r];
+      const int grow = it.qb * BM + r;
+      const bool store = grow < L;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const size_t row_elem = (static_cast<size_t>(it.bh) * L + (store ? grow : 0)) * D;
+      const float a = prm.R ? __ldg(prm.alpha + it.bh % prm.H) : 0.f;
+      const uint32_t tO = tmem + lane_off + C::COL_O + ob * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t regs[32];
+        tmem_ld32(tO + cc * 32, regs);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) reg_fence(regs[e]);
+        if (store) {
+          float v[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = l > 0.f ? __uint_as_float(regs[e]) * inv_l : 0.f;
+          if (prm.R) {
+            const uint4* rp = reinterpret_cast<const uint4*>(prm.R + row_elem + cc * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 rv = __ldg(rp + q);
+              const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                v[q * 8 + 2 * e] += a * __uint_as_float(rw[e] << 16);
+                v[q * 8 + 2 * e + 1] += a * __uint_as_float(rw[e] & 0xFFFF0000u);
+              }
+            }
+          }
+          uint4* op = reinterpret_cast<uint4*>(prm.o + row_elem + cc * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 ov;
+            ov.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+            ov.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+            ov.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+            ov.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+            op[q] = ov;
+          }
+        }
+      }
+      if (store)
+        prm.lse[static_cast<size_t>(it.bh) * L + grow] =
+            l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      tc_fence_before();
+      mbar_arrive(&sh->o_empty[ob]);
+      mbar_arrive(&sh->stats_free[ob]);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0) {
+    // the last CTA of the launch leaves the work counter at zero for reuse;
+    // every CTA has made its final fetch before it counts itself done
+    SchedSlot* sched = &g_sched[prm.sched_slot];
+    __threadfence();
+    if (atomicAdd(&sched->done, 1u) == gridDim.x - 1) {
+      atomicExch(&sched->next, 0u);
+      atomicExch(&sched->done, 0u);
+      __threadfence();
+    }
+  }
+}
+
+// ------------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, int D, int L, int BH, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int D>
+int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
+  using C = Cfg<D>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(sparse_attn_tile_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return BSA_ECUDA;
+    configured = true;
+  }
+  const int BH = s.B * s.H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, D, s.L, BH, BM) || !make_map(&mk, a.k, D, s.L, BH, BN) ||
+      !make_map(&mv, a.v, D, s.L, BH, BN))
+    return BSA_ECUDA;
+  Params prm;
+  prm.kept_idx = a.kept_idx;
+  prm.kept_cnt = a.kept_cnt;
+  prm.R = a.R;
+  prm.alpha = a.alpha;
+  prm.o = a.o;
+  prm.lse = a.lse;
+  prm.status = a.status;
+  prm.H = s.H;
+  prm.L = s.L;
+  prm.NB = n_blocks(s.L, s.blk);
+  prm.NT = prm.NB;  // one work item per 128-token query block
+  prm.n_work = BH * prm.NT;
+  prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  prm.dense = a.kept_idx == nullptr;
+  static std::atomic<unsigned int> launches{0};
+  prm.sched_slot = static_cast<int>(launches.fetch_add(1u) % kSchedSlots);
+  const int grid = prm.n_work < num_sms() ? prm.n_work : num_sms();
+  sparse_attn_tile_kernel<D><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ECUDA;
+}
+
+}  // namespace tile_attn
+
+int launch_sparse_attn_tile(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
+  if (s.blk != 128) return BSA_ESHAPE;
+  if (s.D == 128) return tile_attn::run<128>(s, a, st);
+  if (s.D == 64) return tile_attn::run<64>(s, a, st);
+  return BSA_ESHAPE;
+}
+
+}  // namespace bsa

@@ -48,6 +48,10 @@ struct AttnArgs {
   int32_t* status;
 };
 // Returns BSA_OK / BSA_ECUDA (tensor-map encoding or launch failure).
+// blk = 128: persistent one-tile-per-step kernel (attention_tile.cu);
+// blk = 64: paired-tile kernel over the union of kept lists (attention.cu).
 int launch_sparse_attn(const bsa_shape& s, const AttnArgs& a, cudaStream_t st);
+int launch_sparse_attn_pair(const bsa_shape& s, const AttnArgs& a, cudaStream_t st);
+int launch_sparse_attn_tile(const bsa_shape& s, const AttnArgs& a, cudaStream_t st);
 
 }  // namespace bsa

@@ -149,6 +149,46 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 #undef BSA_R8
 #undef BSA_W8
 
+// 16-lane TMEM accesses (warp-collective; the warp addresses 16 lanes of its
+// quarter starting at the address's lane field).
+//   16x256b: thread t reads lanes (t/4) and (t/4)+8, two adjacent 32-bit
+//            columns 2*(t%4), 2*(t%4)+1 of every 8-column chunk; per chunk the
+//            registers are {lane t/4: col 2j, 2j+1}, {lane t/4+8: col 2j, 2j+1}.
+//   16x128b: thread t holds column (t%4) of every 4-column chunk for lanes
+//            (t/4) and (t/4)+8; per chunk the registers are {lane t/4}, {lane t/4+8}.
+#define BSA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
+                  "=r"(r[i + 6]), "=r"(r[i + 7])
+#define BSA_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), \
+                  "r"(r[i + 6]), "r"(r[i + 7])
+// 8 chunks of 8 columns = 64 columns, 32 registers
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : BSA_R8(0), BSA_R8(8), BSA_R8(16), BSA_R8(24)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      BSA_W8(0), BSA_W8(8), BSA_W8(16), BSA_W8(24)
+      : "memory");
+}
+// 16 chunks of 4 columns = 64 columns, 32 registers
+__device__ __forceinline__ void tmem_st_16x128b_x16(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      BSA_W8(0), BSA_W8(8), BSA_W8(16), BSA_W8(24)
+      : "memory");
+}
+#undef BSA_R8
+#undef BSA_W8
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
