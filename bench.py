@@ -76,19 +76,27 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash():
-    p = os.path.join(ROOT, "block_sparse_attention_logits_b200", "csrc", "attention.cu")
+def attention_kernel(blk):
+    """Source file and kernel name of the attention kernel a block size runs."""
+    if blk == 128:
+        return "attention_tile.cu", "sparse_attn_tile_kernel<128>"
+    return "attention.cu", "sparse_attn_kernel<128,64>"
+
+
+def source_hash(fname):
+    p = os.path.join(ROOT, "block_sparse_attention_logits_b200", "csrc", fname)
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
 
 
-def profiled_traffic(workload):
+def profiled_traffic(workload, blk):
     """DRAM bytes per attention launch from the committed ncu summary, only if
-    it was taken on the current attention source."""
+    it was taken on the current source of the kernel that runs."""
     p = os.path.join(ROOT, "profiles", "attention_traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(workload)
-    if not d or d.get("attention_cu_sha256_16") != source_hash():
+    fname, _ = attention_kernel(blk)
+    if not d or d.get("kernel_source") != fname or d.get("kernel_source_sha256_16") != source_hash(fname):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -342,11 +350,11 @@ def run_ours(args, w, world, rank, local):
     peaks, peak_src = load_peaks()
     attn_avg_ms = float(np.mean(attn_ms))
     achieved = flops / (attn_avg_ms * 1e-3) / 1e12
-    traffic = profiled_traffic(w.name)
+    traffic = profiled_traffic(w.name, w.blk)
     roofline = {"bound": "tensor", "achieved": round(achieved, 2),
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                 "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
-                "traffic": traffic, "kernel": "sparse_attn_kernel<128,128>",
+                "traffic": traffic, "kernel": attention_kernel(w.blk)[1],
                 "peak_kind": f"{peak_src} sustained (kernel timed inside a long step)",
                 "peak_burst": peaks["bf16_tflops"], "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4)}
 
