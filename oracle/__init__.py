@@ -21,6 +21,8 @@ Sources (cited by page title and section in every function):
   scoring.
 * CalibAtt (calibrated sparse attention), abstract and Fig. 5 -- threshold the
   top key blocks per query block, skip the unselected blocks.
+* the GSRS abstract -- exact attention weights evaluated inside the
+  FlashAttention computation (the kept share of the attention mass).
 
 Modules:
   hilbert     -- 3-D Hilbert order of the latent grid, perm / inv
@@ -28,9 +30,11 @@ Modules:
   topp        -- cumulative top-p block selection, mask and kept lists
   attention   -- masked softmax attention over the kept blocks (O, LSE)
   correction  -- dense-minus-sparse refinement and the alpha-scaled correction
+  refresh     -- the outputs of a single-pass dense refresh (dense and sparse
+                 attention, refinement, exact kept attention mass)
 
 Every function carries a "Pinned by" note naming the tests in
 ``tests/test_oracle.py`` that tie it to something other than itself.
 """
 
-from . import hilbert, scoring, topp, attention, correction  # noqa: F401
+from . import hilbert, scoring, topp, attention, correction, refresh  # noqa: F401

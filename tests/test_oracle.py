@@ -19,6 +19,7 @@ import torch
 from oracle import attention as oatt
 from oracle import correction as ocor
 from oracle import hilbert as ohil
+from oracle import refresh as oref
 from oracle import scoring as osco
 from oracle import topp as otop
 
@@ -377,6 +378,82 @@ def test_correction_identities():
     half = ocor.apply_correction(osp, R, np.array([0.0, 0.5, 1.0]))
     assert np.allclose(half[:, 1], osp[:, 1] + 0.5 * R[:, 1])
     assert np.allclose(half[:, 2], full[:, 2]) and np.allclose(half[:, 0], osp[:, 0])
+
+
+# ------------------------------------------------------------ fused refresh
+
+def _refresh_case(seed, B=1, H=2, L=150, D=8, blk=32):
+    rng = np.random.default_rng(seed)
+    q, k, v = (rng.standard_normal((B, H, L, D)) for _ in range(3))
+    NB = (L + blk - 1) // blk
+    idx = np.zeros((B, H, NB, NB), np.int32)
+    cnt = np.zeros((B, H, NB), np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(NB):
+                kept = np.sort(rng.choice(NB, rng.integers(1, NB + 1), replace=False))
+                idx[b, h, i, :len(kept)] = kept
+                cnt[b, h, i] = len(kept)
+    return q, k, v, idx, cnt, NB
+
+
+def test_refresh_keep_all_gives_unit_mass_and_zero_refinement():
+    q, k, v, _, _, NB = _refresh_case(21)
+    fi, fc = oref.full_lists(1, 2, NB)
+    Od, Ld, Os, Ls, R, mass = oref.fused_refresh(q, k, v, fi, fc, 32)
+    assert np.array_equal(Od, Os) and np.array_equal(Ld, Ls)
+    assert np.all(R == 0) and np.all(mass == 1.0)
+
+
+def test_refresh_mass_closed_form_for_constant_keys():
+    rng = np.random.default_rng(22)
+    B, H, L, D, blk = 1, 1, 150, 8, 32   # 5 blocks, the last one holds 22 tokens
+    q = rng.standard_normal((B, H, L, D))
+    k = np.tile(rng.standard_normal(D), (B, H, L, 1))
+    v = rng.standard_normal((B, H, L, D))
+    NB = 5
+    idx = np.zeros((B, H, NB, NB), np.int32)
+    cnt = np.zeros((B, H, NB), np.int32)
+    idx[0, 0, :, :2] = [0, 4]
+    cnt[:] = 2
+    *_, mass = oref.fused_refresh(q, k, v, idx, cnt, blk)
+    assert np.allclose(mass, (32 + 22) / 150, atol=1e-12)
+
+
+def test_refresh_dense_is_mass_weighted_mixture_of_kept_and_complement():
+    q, k, v, idx, cnt, NB = _refresh_case(23)
+    Od, Ld, Os, Ls, R, mass = oref.fused_refresh(q, k, v, idx, cnt, 32)
+    ci, cc = oref.complement_lists(idx, cnt, NB)
+    Oc, Lc = oatt.masked_attention(q, k, v, ci, cc, 32)
+    full = cc == 0  # rows that keep every block have an empty complement
+    fullr = np.repeat(full, 32, axis=2)[:, :, :150]
+    Oc = np.where(fullr[..., None], 0.0, Oc)
+    mix = mass[..., None] * Os + (1 - mass[..., None]) * Oc
+    assert np.allclose(Od, mix, atol=1e-12)
+    assert np.allclose(Ld, np.logaddexp(Ls, np.where(fullr, -np.inf, Lc)), atol=1e-12)
+    assert np.all((mass > 0) & (mass <= 1 + 1e-15))
+
+
+def test_refresh_refinement_matches_torch_rounding():
+    q, k, v, idx, cnt, _ = _refresh_case(24)
+    Od, _, Os, _, R, _ = oref.fused_refresh(q, k, v, idx, cnt, 32)
+    t = lambda a: torch.from_numpy(np.asarray(a, np.float64)).to(torch.bfloat16).float()
+    ref = (t(Od) - t(Os)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(R.view(np.uint32), ref.view(np.uint32))
+
+
+def test_refresh_empty_kept_row():
+    q, k, v, idx, cnt, _ = _refresh_case(25)
+    cnt[0, 1, 2] = 0
+    _, _, Os, Ls, _, mass = oref.fused_refresh(q, k, v, idx, cnt, 32)
+    rows = slice(64, 96)
+    assert np.all(Os[0, 1, rows] == 0) and np.all(np.isneginf(Ls[0, 1, rows])) and np.all(mass[0, 1, rows] == 0)
+
+
+def test_planted_mistake_inverted_mass_is_caught(monkeypatch):
+    monkeypatch.setattr(oref, "kept_mass", lambda ls, ld: np.exp(np.asarray(ld) - np.asarray(ls)))
+    with pytest.raises(AssertionError):
+        test_refresh_mass_closed_form_for_constant_keys()
 
 
 # ------------------------------------------------- planted mistakes are caught
