@@ -162,6 +162,49 @@ def sparse_attn_fwd(q, k, v, blk, kept_idx=None, kept_cnt=None, R=None, alpha=No
     return o, lse
 
 
+def sparse_attn_refresh(q, k, v, blk, kept_idx, kept_cnt, want_r=True, want_mass=True, out=None, status=None):
+    """Dense refresh in one pass over every key block.
+
+    Returns (o_dense, lse_dense, o_sparse, lse_sparse, R, kept_mass): the dense
+    and the kept-block attention (bf16 O, float32 LSE), R = bf16(bf16(o_dense)
+    - bf16(o_sparse)) (None unless want_r) and the kept share of the attention
+    weight per row (None unless want_mass).  blk must be 128.  `out` may hold
+    preallocated tensors under the same names.
+    """
+    B, H, L, D = q.shape
+    nb = n_blocks(L, blk)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, torch.bfloat16, (B, H, L, D), name)
+    _need(kept_idx, torch.int32, (B, H, nb, nb), "kept_idx")
+    _need(kept_cnt, torch.int32, (B, H, nb), "kept_cnt")
+    out = dict(out or {})
+    dev = q.device
+    o_d = out.get("o_dense", None)
+    o_d = o_d if o_d is not None else torch.empty_like(q)
+    o_s = out.get("o_sparse", None)
+    o_s = o_s if o_s is not None else torch.empty_like(q)
+    l_d = out.get("lse_dense", None)
+    l_d = l_d if l_d is not None else torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    l_s = out.get("lse_sparse", None)
+    l_s = l_s if l_s is not None else torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    R = out.get("R", None) if want_r else None
+    R = R if (R is not None or not want_r) else torch.empty_like(q)
+    mass = out.get("kept_mass", None) if want_mass else None
+    mass = mass if (mass is not None or not want_mass) else torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    for name, t in (("o_dense", o_d), ("o_sparse", o_s)):
+        _need(t, torch.bfloat16, (B, H, L, D), name)
+    for name, t in (("lse_dense", l_d), ("lse_sparse", l_s)):
+        _need(t, torch.float32, (B, H, L), name)
+    if R is not None:
+        _need(R, torch.bfloat16, (B, H, L, D), "R")
+    if mass is not None:
+        _need(mass, torch.float32, (B, H, L), "kept_mass")
+    check("bsa_sparse_attn_refresh", _lib.load().bsa_sparse_attn_refresh(
+        Shape(B, H, L, D, blk), _ptr(q), _ptr(k), _ptr(v), _ptr(kept_idx), _ptr(kept_cnt),
+        _ptr(o_d), _ptr(l_d), _ptr(o_s), _ptr(l_s), _ptr(R), _ptr(mass), _ptr(status), _stream()))
+    return o_d, l_d, o_s, l_s, R, mass
+
+
 def refresh_refinement(o_dense, o_sparse, out=None):
     """R = bf16(o_dense - o_sparse)."""
     B, H, L, D = o_dense.shape

@@ -143,6 +143,37 @@ int bsa_sparse_attn_fwd(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const
   return bsa::launch_sparse_attn(s, a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int bsa_sparse_attn_refresh(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
+                            const int32_t* kept_idx, const int32_t* kept_cnt, bsa_bf16* o_dense, float* lse_dense,
+                            bsa_bf16* o_sparse, float* lse_sparse, bsa_bf16* R, float* kept_mass, int32_t* status,
+                            bsa_stream stream) {
+  if (!q || !k || !v || !kept_idx || !kept_cnt || !o_dense || !lse_dense || !o_sparse || !lse_sparse)
+    return BSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kept_idx) || !aligned16(kept_cnt) ||
+      !aligned16(o_dense) || !aligned16(lse_dense) || !aligned16(o_sparse) || !aligned16(lse_sparse))
+    return BSA_EINVAL;
+  if ((R && !aligned16(R)) || (kept_mass && !aligned16(kept_mass))) return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (s.blk != 128) return BSA_ESHAPE;
+  if (int r = check_device()) return r;
+  bsa::AttnArgs a;
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  a.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  a.kept_idx = kept_idx;
+  a.kept_cnt = kept_cnt;
+  a.R = nullptr;
+  a.alpha = nullptr;
+  a.o = reinterpret_cast<__nv_bfloat16*>(o_dense);
+  a.lse = lse_dense;
+  a.status = status;
+  a.o2 = reinterpret_cast<__nv_bfloat16*>(o_sparse);
+  a.lse2 = lse_sparse;
+  a.r_out = reinterpret_cast<__nv_bfloat16*>(R);
+  a.mass = kept_mass;
+  return bsa::launch_sparse_attn(s, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int bsa_refresh_refinement(bsa_shape s, const bsa_bf16* o_dense, const bsa_bf16* o_sparse, bsa_bf16* R,
                            bsa_stream stream) {
   if (!o_dense || !o_sparse || !R) return BSA_EINVAL;

@@ -46,6 +46,19 @@
 // rescaled in TMEM (after the previous PV completed), and the final 1/l uses
 // the same reference.
 //
+// Fused refresh (kFused).  Every key block is visited once; the PV of a kept
+// block accumulates into OK, that of any other block into OR (TMEM: S0 | S1 |
+// OK | OR, so O is single-buffered across items and the PV of an item waits
+// until the epilogue has read the previous item's O).  One shared reference
+// max serves both; the softmax keeps the total row sum and the kept row sum.
+// The epilogue writes the dense output (OK + OR) / l, the sparse output
+// OK / l_kept, both LSEs, R = bf16(bf16(O_dense) - bf16(O_sparse)) and the kept
+// share of the attention weight l_kept / l (RECAP section 1 and section 3.4
+// with Fig. 3: a dense refresh renews the refinement; GSRS abstract: exact
+// attention weights within the attention computation).  Membership of a block
+// in the kept set comes from the ascending kept list; entries that are out of
+// range or out of order are skipped and flagged.
+//
 // Every wait is bounded (2 s of globaltimer); a timeout sets BSA_DEV_TIMEOUT
 // in the caller's status word and makes every role give up; the MMA issuers
 // and TMA producers wait (bounded) for their operations in flight before TMEM
@@ -94,6 +107,10 @@ struct Params {
   const float* alpha;
   __nv_bfloat16* o;
   float* lse;
+  __nv_bfloat16* o2;     // fused refresh: sparse output
+  float* lse2;           //                sparse LSE
+  __nv_bfloat16* r_out;  //                refinement (nullable)
+  float* mass;           //                kept attention share (nullable)
   int32_t* status;
   int H, L, NB, NT, n_work;
   float scale_log2;
@@ -105,7 +122,7 @@ template <int D>
 struct Cfg {
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int STATS_BYTES = 2 * 2 * BM * 4;  // [item parity][l, m][row]
+  static constexpr int STATS_BYTES = 2 * 3 * BM * 4;  // [item parity][l, m, l_kept][row]
   static constexpr int MISC_BYTES = 512;
   static constexpr int SLOTS = (227 * 1024 - 1024 - 2 * Q_BYTES - STATS_BYTES - MISC_BYTES) / KV_BYTES;
   static constexpr int NSK = ((SLOTS + 1) / 2) > 4 ? 4 : (SLOTS + 1) / 2;
@@ -180,16 +197,29 @@ __device__ __forceinline__ int next_item(int i, Shared* sh, const Params& prm) {
 // One work item: a 128-row query block of one (batch, head) and its key list.
 struct Item {
   int bh, qb, cnt;
-  const int32_t* list;  // null in dense mode
-  bool bad_cnt;         // the count was outside [0, NB] and was clamped
+  const int32_t* list;   // null in dense mode
+  bool bad_cnt;          // the count was outside [0, NB] and was clamped
+  const int32_t* klist;  // fused refresh: the kept list (ascending) ...
+  int kcnt;              // ... and its length
 };
 
+template <bool kFused>
 __device__ __forceinline__ Item item_of(int w, const Params& prm) {
   Item it;
   it.bh = w / prm.NT;
   it.qb = w - it.bh * prm.NT;
   it.bad_cnt = false;
-  if (prm.dense) {
+  it.klist = nullptr;
+  it.kcnt = 0;
+  if (kFused) {
+    const size_t r = static_cast<size_t>(it.bh) * prm.NB + it.qb;
+    const int c = __ldg(prm.kept_cnt + r);
+    it.bad_cnt = c < 0 || c > prm.NB;
+    it.kcnt = c < 0 ? 0 : (c > prm.NB ? prm.NB : c);
+    it.klist = prm.kept_idx + r * prm.NB;
+    it.cnt = prm.NB;
+    it.list = nullptr;
+  } else if (prm.dense) {
     it.cnt = prm.NB;
     it.list = nullptr;
   } else {
@@ -208,11 +238,29 @@ __device__ __forceinline__ int entry_kb(const Item& it, int n, int NB) {
   return static_cast<unsigned>(kb) < static_cast<unsigned>(NB) ? kb : -1;
 }
 
-template <int D>
+// Fused refresh: is key block j (visited in ascending order) in the kept list?
+// kp walks the list; entries below j were out of order or repeated.
+__device__ __forceinline__ bool kept_at(const Item& it, int j, int& kp, bool& bad) {
+  int e = kp < it.kcnt ? __ldg(it.klist + kp) : INT_MAX;
+  while (e < j) {
+    bad = true;
+    ++kp;
+    e = kp < it.kcnt ? __ldg(it.klist + kp) : INT_MAX;
+  }
+  if (e == j) {
+    ++kp;
+    return true;
+  }
+  return false;
+}
+
+template <int D, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const Params prm) {
   using C = Cfg<D>;
+  constexpr int OB = kFused ? 1 : 2;          // O buffers across items
+  constexpr int OB_RESCALE = kFused ? 2 : 1;  // accumulators per item
   constexpr int NSK = C::NSK;
   constexpr int NSV = C::NSV;
   extern __shared__ uint8_t smem_raw[];
@@ -285,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         w = __shfl_sync(0xffffffffu, w, 0);
         if (w < 0) break;
-        const Item it = item_of(w, prm);
+        const Item it = item_of<kFused>(w, prm);
         if (it.bad_cnt && lane == 0) flag_status(prm, BSA_DEV_BAD_INDEX);
         const int qb = i & 1;
         if (i >= 2 && !(ok = warp_wait(&sh->q_empty[qb], ((i - 2) >> 1) & 1, sh, prm))) break;
@@ -326,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; ok; ++i) {
         const int w = next_item(i, sh, prm);
         if (w < 0) break;
-        const Item it = item_of(w, prm);
+        const Item it = item_of<kFused>(w, prm);
         for (int n = 0; n < it.cnt; ++n) {
           const int kb = entry_kb(it, n, NB);
           if (kb < 0) continue;
@@ -355,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; ok; ++i) {
         const int w = next_item(i, sh, prm);
         if (w < 0) break;
-        const Item it = item_of(w, prm);
+        const Item it = item_of<kFused>(w, prm);
         const int qb = i & 1;
         if (!(ok = warp_wait(&sh->q_full[qb], (i >> 1) & 1, sh, prm))) break;
         const uint32_t qa = q_base + qb * C::Q_BYTES;
@@ -399,31 +447,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; ok; ++i) {
         const int w = next_item(i, sh, prm);
         if (w < 0) break;
-        const Item it = item_of(w, prm);
-        const int ob = i & 1;
-        if (i >= 2 && !(ok = warp_wait(&sh->o_empty[ob], ((i - 2) >> 1) & 1, sh, prm))) break;
-        bool first = true;
+        const Item it = item_of<kFused>(w, prm);
+        const int ob = kFused ? 0 : (i & 1);
+        if (i >= OB && !(ok = warp_wait(&sh->o_empty[ob], ((i - OB) / OB) & 1, sh, prm))) break;
+        bool first = true, first_rest = true;
+        int kp = 0;
+        bool bad = false;
         for (int n = 0; n < it.cnt; ++n) {
-          if (entry_kb(it, n, NB) < 0) continue;
+          const int kb = entry_kb(it, n, NB);
+          if (kb < 0) continue;
+          const bool kept = !kFused || kept_at(it, kb, kp, bad);
           const int sv = u % NSV;
           const int b = u & 1;
           if (!(ok = warp_wait(&sh->p_full[b], (u >> 1) & 1, sh, prm))) break;
           if (!(ok = warp_wait(&sh->full_v[sv], (u / NSV) & 1, sh, prm))) break;
           tc_fence_after();
+          const bool fresh = kept ? first : first_rest;
           if (lane == 0) {
             const uint32_t va = v_base + sv * C::KV_BYTES;
+            const uint32_t dst = tmem + C::COL_O + (kFused ? (kept ? 0 : D) : ob * D);
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)
-              mma_ts(tmem + C::COL_O + ob * D, tmem + C::COL_S + b * BN + kk * 8,
-                     sdesc_sw128(va + kk * 2048, BN * 128, 1024), idPV, (!first || kk > 0) ? 1u : 0u);
+              mma_ts(dst, tmem + C::COL_S + b * BN + kk * 8, sdesc_sw128(va + kk * 2048, BN * 128, 1024), idPV,
+                     (!fresh || kk > 0) ? 1u : 0u);
             tc_commit(&sh->pv_done[b]);
             tc_commit(&sh->empty_v[sv]);
           }
           __syncwarp();
-          first = false;
+          if (kept)
+            first = false;
+          else
+            first_rest = false;
           ++u;
         }
         if (!ok) break;
+        if (kFused && (bad || kp < it.kcnt) && lane == 0) flag_status(prm, BSA_DEV_BAD_INDEX);
         if (lane == 0) tc_commit(&sh->o_full[ob]);
         __syncwarp();
       }
@@ -448,15 +506,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; ok; ++i) {
       const int w = next_item(i, sh, prm);
       if (w < 0) break;
-      const Item it = item_of(w, prm);
-      const int ob = i & 1;
+      const Item it = item_of<kFused>(w, prm);
+      const int ob = kFused ? 0 : (i & 1);
+      const int sb = i & 1;  // statistics buffer
       const uint32_t tO = tmem + lane_off + C::COL_O + ob * D;
       float mA = -INFINITY, mB = -INFINITY;  // reference max of rows rA, rA+8 (log2 units)
       float lA = 0.f, lB = 0.f;              // this thread's share of the row sums
+      float kA = 0.f, kB = 0.f;              // fused refresh: the same over the kept blocks
       int nt = 0;
+      int kp = 0;
+      bool bad = false;
       for (int n = 0; n < it.cnt; ++n) {
         const int kb = entry_kb(it, n, NB);
         if (kb < 0) continue;
+        const bool kept = !kFused || kept_at(it, kb, kp, bad);
         const int b = u & 1;
         const uint32_t tS = tmem + lane_off + C::COL_S + b * BN;
         if (!(ok = warp_wait(&sh->s_full[b], (u >> 1) & 1, sh, prm))) break;
@@ -501,11 +564,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (rsA) {
           fA = ex2_approx(mA - nA);  // 0 when mA is -inf
           lA *= fA;
+          kA *= fA;
           mA = nA;
         }
         if (rsB) {
           fB = ex2_approx(mB - nB);
           lB *= fB;
+          kB *= fB;
           mB = nB;
         }
         if (nt > 0 && __any_sync(0xffffffffu, rsA || rsB)) {
@@ -513,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = warp_wait(&sh->pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1, sh, prm))) break;
           tc_fence_after();
 #pragma unroll
-          for (int cc = 0; cc < D / 64; ++cc) {
+          for (int cc = 0; cc < OB_RESCALE * D / 64; ++cc) {  // fused: OK and OR
             uint32_t o[32];
             tmem_ld_16x256b_x8(tO + cc * 64, o);
             tmem_wait_ld();
@@ -557,6 +622,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           f2_unpack(f2_add(accB0, accB1), b0, b1);
           lA += a0 + a1;
           lB += b0 + b1;
+          if (kFused && kept) {
+            kA += a0 + a1;
+            kB += b0 + b1;
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -570,15 +639,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       lB += __shfl_xor_sync(0xffffffffu, lB, 1);
       lA += __shfl_xor_sync(0xffffffffu, lA, 2);
       lB += __shfl_xor_sync(0xffffffffu, lB, 2);
-      if (i >= 2 && !(ok = warp_wait(&sh->stats_free[ob], ((i - 2) >> 1) & 1, sh, prm))) break;
-      float* st = stats + ob * 2 * BM;
+      if (kFused) {
+        kA += __shfl_xor_sync(0xffffffffu, kA, 1);
+        kB += __shfl_xor_sync(0xffffffffu, kB, 1);
+        kA += __shfl_xor_sync(0xffffffffu, kA, 2);
+        kB += __shfl_xor_sync(0xffffffffu, kB, 2);
+      }
+      if (i >= 2 && !(ok = warp_wait(&sh->stats_free[sb], ((i - 2) >> 1) & 1, sh, prm))) break;
+      float* st = stats + sb * 3 * BM;
       if (j4 == 0) {
         st[rA] = lA;
         st[rA + 8] = lB;
         st[BM + rA] = mA;
         st[BM + rA + 8] = mB;
+        if (kFused) {
+          st[2 * BM + rA] = kA;
+          st[2 * BM + rA + 8] = kB;
+        }
       }
-      mbar_arrive(&sh->stats_full[ob]);
+      mbar_arrive(&sh->stats_full[sb]);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -590,62 +669,128 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; ok; ++i) {
       const int w = next_item(i, sh, prm);
       if (w < 0) break;
-      const Item it = item_of(w, prm);
-      const int ob = i & 1;
-      if (!(ok = warp_wait(&sh->o_full[ob], (i >> 1) & 1, sh, prm))) break;
-      if (!(ok = warp_wait(&sh->stats_full[ob], (i >> 1) & 1, sh, prm))) break;
+      const Item it = item_of<kFused>(w, prm);
+      const int ob = kFused ? 0 : (i & 1);
+      const int sb = i & 1;
+      if (!(ok = warp_wait(&sh->o_full[ob], (i / OB) & 1, sh, prm))) break;
+      if (!(ok = warp_wait(&sh->stats_full[sb], (i >> 1) & 1, sh, prm))) break;
       tc_fence_after();
-      const float* st = stats + ob * 2 * BM;
+      const float* st = stats + sb * 3 * BM;
       const float l = st[r];
       const float m_ref = st[BM + r];
       const int grow = it.qb * BM + r;
       const bool store = grow < L;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const size_t row_elem = (static_cast<size_t>(it.bh) * L + (store ? grow : 0)) * D;
-      const float a = prm.R ? __ldg(prm.alpha + it.bh % prm.H) : 0.f;
       const uint32_t tO = tmem + lane_off + C::COL_O + ob * D;
+      if constexpr (kFused) {
+        // dense = (OK + OR) / l, sparse = OK / l_kept.  OK holds data only if
+        // some block was kept (l_kept > 0), OR only if some block was not,
+        // which is exactly when l differs from l_kept (the two sums add the
+        // same terms in the same order otherwise); an accumulator that no PV
+        // of this item wrote still holds an earlier item's values.
+        const float lk = st[2 * BM + r];
+        mbar_arrive(&sh->stats_free[sb]);
+        const bool rest = l != lk;
+        const bool kept_any = lk > 0.f;
+        const float inv_k = lk > 0.f ? 1.f / lk : 0.f;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t regs[32];
-        tmem_ld32(tO + cc * 32, regs);
-        tmem_wait_ld();
+        for (int cc = 0; cc < D / 16; ++cc) {
+          uint32_t ok_[16], or_[16];
+          tmem_ld16(tO + cc * 16, ok_);
+          tmem_ld16(tO + D + cc * 16, or_);
+          tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) reg_fence(regs[e]);
-        if (store) {
-          float v[32];
+          for (int e = 0; e < 16; ++e) {
+            reg_fence(ok_[e]);
+            reg_fence(or_[e]);
+          }
+          if (cc == D / 16 - 1) {
+            // OK and OR have been read out: the next item's PV may overwrite them
+            tc_fence_before();
+            mbar_arrive(&sh->o_empty[ob]);
+          }
+          if (store) {
+            uint32_t pd[8], ps[8], pr[8];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = l > 0.f ? __uint_as_float(regs[e]) * inv_l : 0.f;
-          if (prm.R) {
-            const uint4* rp = reinterpret_cast<const uint4*>(prm.R + row_elem + cc * 32);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 rv = __ldg(rp + q);
-              const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                v[q * 8 + 2 * e] += a * __uint_as_float(rw[e] << 16);
-                v[q * 8 + 2 * e + 1] += a * __uint_as_float(rw[e] & 0xFFFF0000u);
+            for (int e = 0; e < 8; ++e) {
+              float d0 = kept_any ? __uint_as_float(ok_[2 * e]) : 0.f;
+              float d1 = kept_any ? __uint_as_float(ok_[2 * e + 1]) : 0.f;
+              const float s0 = d0 * inv_k, s1 = d1 * inv_k;
+              if (rest) {
+                d0 += __uint_as_float(or_[2 * e]);
+                d1 += __uint_as_float(or_[2 * e + 1]);
               }
+              pd[e] = pack_bf16x2(d0 * inv_l, d1 * inv_l);
+              ps[e] = pack_bf16x2(s0, s1);
+              // R = bf16(bf16(O_dense) - bf16(O_sparse))
+              pr[e] = pack_bf16x2(__uint_as_float(pd[e] << 16) - __uint_as_float(ps[e] << 16),
+                                  __uint_as_float(pd[e] & 0xFFFF0000u) - __uint_as_float(ps[e] & 0xFFFF0000u));
+            }
+            uint4* od = reinterpret_cast<uint4*>(prm.o + row_elem + cc * 16);
+            uint4* os = reinterpret_cast<uint4*>(prm.o2 + row_elem + cc * 16);
+            od[0] = make_uint4(pd[0], pd[1], pd[2], pd[3]);
+            od[1] = make_uint4(pd[4], pd[5], pd[6], pd[7]);
+            os[0] = make_uint4(ps[0], ps[1], ps[2], ps[3]);
+            os[1] = make_uint4(ps[4], ps[5], ps[6], ps[7]);
+            if (prm.r_out) {
+              uint4* orr = reinterpret_cast<uint4*>(prm.r_out + row_elem + cc * 16);
+              orr[0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+              orr[1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
             }
           }
-          uint4* op = reinterpret_cast<uint4*>(prm.o + row_elem + cc * 32);
+        }
+        if (store) {
+          const size_t rr = static_cast<size_t>(it.bh) * L + grow;
+          prm.lse[rr] = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+          prm.lse2[rr] = lk > 0.f ? (m_ref + log2f(lk)) * 0.69314718055994531f : -INFINITY;
+          if (prm.mass) prm.mass[rr] = l > 0.f ? lk / l : 0.f;  // exactly 1 when every block is kept
+        }
+      } else {
+        const float a = prm.R ? __ldg(prm.alpha + it.bh % prm.H) : 0.f;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 ov;
-            ov.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-            ov.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-            ov.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-            ov.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-            op[q] = ov;
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t regs[32];
+          tmem_ld32(tO + cc * 32, regs);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) reg_fence(regs[e]);
+          if (store) {
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = l > 0.f ? __uint_as_float(regs[e]) * inv_l : 0.f;
+            if (prm.R) {
+              const uint4* rp = reinterpret_cast<const uint4*>(prm.R + row_elem + cc * 32);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint4 rv = __ldg(rp + q);
+                const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  v[q * 8 + 2 * e] += a * __uint_as_float(rw[e] << 16);
+                  v[q * 8 + 2 * e + 1] += a * __uint_as_float(rw[e] & 0xFFFF0000u);
+                }
+              }
+            }
+            uint4* op = reinterpret_cast<uint4*>(prm.o + row_elem + cc * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 ov;
+              ov.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+              ov.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+              ov.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+              ov.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+              op[q] = ov;
+            }
           }
         }
+        if (store)
+          prm.lse[static_cast<size_t>(it.bh) * L + grow] =
+              l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        tc_fence_before();
+        mbar_arrive(&sh->o_empty[ob]);
+        mbar_arrive(&sh->stats_free[sb]);
       }
-      if (store)
-        prm.lse[static_cast<size_t>(it.bh) * L + grow] =
-            l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
-      tc_fence_before();
-      mbar_arrive(&sh->o_empty[ob]);
-      mbar_arrive(&sh->stats_free[ob]);
     }
   }
 
@@ -708,12 +853,12 @@ int num_sms() {
   return n;
 }
 
-template <int D>
+template <int D, bool kFused>
 int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   using C = Cfg<D>;
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(sparse_attn_tile_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(sparse_attn_tile_kernel<D, kFused>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return BSA_ECUDA;
     configured = true;
@@ -730,6 +875,10 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   prm.alpha = a.alpha;
   prm.o = a.o;
   prm.lse = a.lse;
+  prm.o2 = a.o2;
+  prm.lse2 = a.lse2;
+  prm.r_out = a.r_out;
+  prm.mass = a.mass;
   prm.status = a.status;
   prm.H = s.H;
   prm.L = s.L;
@@ -741,7 +890,7 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   static std::atomic<unsigned int> launches{0};
   prm.sched_slot = static_cast<int>(launches.fetch_add(1u) % kSchedSlots);
   const int grid = prm.n_work < num_sms() ? prm.n_work : num_sms();
-  sparse_attn_tile_kernel<D><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, prm);
+  sparse_attn_tile_kernel<D, kFused><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ECUDA;
 }
 
@@ -749,8 +898,13 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
 
 int launch_sparse_attn_tile(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   if (s.blk != 128) return BSA_ESHAPE;
-  if (s.D == 128) return tile_attn::run<128>(s, a, st);
-  if (s.D == 64) return tile_attn::run<64>(s, a, st);
+  if (a.o2) {
+    if (s.D == 128) return tile_attn::run<128, true>(s, a, st);
+    if (s.D == 64) return tile_attn::run<64, true>(s, a, st);
+    return BSA_ESHAPE;
+  }
+  if (s.D == 128) return tile_attn::run<128, false>(s, a, st);
+  if (s.D == 64) return tile_attn::run<64, false>(s, a, st);
   return BSA_ESHAPE;
 }
 

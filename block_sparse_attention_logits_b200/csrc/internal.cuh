@@ -46,6 +46,12 @@ struct AttnArgs {
   __nv_bfloat16* o;
   float* lse;
   int32_t* status;
+  // fused refresh (blk = 128 only): non-null o2 selects it; o/lse receive the
+  // dense output, o2/lse2 the sparse output over the kept blocks
+  __nv_bfloat16* o2 = nullptr;
+  float* lse2 = nullptr;
+  __nv_bfloat16* r_out = nullptr;  // nullable
+  float* mass = nullptr;           // nullable
 };
 // Returns BSA_OK / BSA_ECUDA (tensor-map encoding or launch failure).
 // blk = 128: persistent one-tile-per-step kernel (attention_tile.cu);

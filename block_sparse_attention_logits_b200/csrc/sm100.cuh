@@ -146,6 +146,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       BSA_W8(0), BSA_W8(8), BSA_W8(16), BSA_W8(24)
       : "memory");
 }
+// 16 consecutive 32-bit columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : BSA_R8(0), BSA_R8(8)
+      : "r"(taddr));
+}
 #undef BSA_R8
 #undef BSA_W8
 

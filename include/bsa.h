@@ -201,6 +201,34 @@ BSA_API int bsa_refresh_refinement(bsa_shape s, const bsa_bf16* o_dense, const b
                            bsa_stream stream);
 
 /*
+ * bsa_sparse_attn_refresh -- a dense refresh in one pass over every key block.
+ * Defines: the dense refresh that renews the cached refinement (RECAP,
+ * section 1 and section 3.4 with Fig. 3) and the exact share of the attention
+ * weight carried by the kept blocks, evaluated inside the attention
+ * computation (GSRS abstract).  With K(i) the kept blocks of query block i and
+ * s_c = q_r . k_c / sqrt(D) over keys c < L:
+ *   lse_dense[r]  = log sum_{all c} exp(s_c),  o_dense[r]  = sum_c exp(s_c - lse_dense[r]) v_c
+ *   lse_sparse[r] = log sum_{c in K(i)} exp(s_c),  o_sparse[r] likewise over K(i)
+ *   R[r]          = bf16( bf16(o_dense[r]) - bf16(o_sparse[r]) )   (as bsa_refresh_refinement)
+ *   kept_mass[r]  = exp(lse_sparse[r] - lse_dense[r])             (0 for an empty K(i))
+ * One pass: every key block is read once; a kept block's P.V goes to one
+ * accumulator and any other block's to a second, under one running max.
+ * Arguments: q, k, v bf16 [B,H,L,D]; kept_idx/kept_cnt (required) as produced
+ * by bsa_select_topp_mask -- each row's list must be ascending; entries out of
+ * range or out of order are skipped and flagged in status.  Outputs o_dense,
+ * o_sparse bf16 [B,H,L,D]; lse_dense, lse_sparse float32 [B,H,L] (natural
+ * log); R bf16 [B,H,L,D] or NULL; kept_mass float32 [B,H,L] or NULL.
+ * s.blk must be 128 and s.D 64 or 128.
+ * status: optional device int32 as for bsa_sparse_attn_fwd.
+ * Errors: BSA_EINVAL on null required or misaligned pointers; BSA_ESHAPE;
+ * BSA_ENODEV; BSA_ECUDA.
+ */
+BSA_API int bsa_sparse_attn_refresh(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
+                            const int32_t* kept_idx, const int32_t* kept_cnt, bsa_bf16* o_dense,
+                            float* lse_dense, bsa_bf16* o_sparse, float* lse_sparse, bsa_bf16* R,
+                            float* kept_mass, int32_t* status, bsa_stream stream);
+
+/*
  * bsa_apply_correction -- standalone form of the fused correction.
  * Defines: fresh sparse statistics regulating how strongly the aging cached
  * refinement is applied (RECAP, section 1 and abstract), here as a

@@ -30,7 +30,8 @@ def declared_symbols():
 def test_header_declares_the_boundary():
     syms = declared_symbols()
     for name in ("bsa_score_blocks", "bsa_select_topp_mask", "bsa_reorder_tokens", "bsa_permute_tokens",
-                 "bsa_sparse_attn_fwd", "bsa_refresh_refinement", "bsa_apply_correction", "bsa_strerror"):
+                 "bsa_sparse_attn_fwd", "bsa_sparse_attn_refresh", "bsa_refresh_refinement", "bsa_apply_correction",
+                 "bsa_strerror"):
         assert name in syms
     assert set(syms) == set(_lib.EXPORTS)
 
@@ -104,6 +105,28 @@ def test_attention_validation(lib):
                                    NULL, NULL) == _lib.BSA_ESHAPE
     assert lib.bsa_sparse_attn_fwd(Shape(70000, 1, 10, 64, 64), *args, NULL, NULL, NULL, NULL, FAKE, FAKE,
                                    NULL, NULL) == _lib.BSA_ESHAPE
+
+
+def test_refresh_validation(lib):
+    s = Shape(1, 2, 1000, 128, 128)
+    qkv = (FAKE, FAKE, FAKE)
+    ok_out = (FAKE, FAKE, FAKE, FAKE)  # o_dense, lse_dense, o_sparse, lse_sparse
+    # the kept lists are required
+    assert lib.bsa_sparse_attn_refresh(s, *qkv, NULL, FAKE, *ok_out, NULL, NULL, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_refresh(s, *qkv, FAKE, NULL, *ok_out, NULL, NULL, NULL, NULL) == _lib.BSA_EINVAL
+    # every output but R and kept_mass is required
+    for miss in range(4):
+        outs = list(ok_out)
+        outs[miss] = NULL
+        assert lib.bsa_sparse_attn_refresh(s, *qkv, FAKE, FAKE, *outs, NULL, NULL, NULL, NULL) == _lib.BSA_EINVAL
+    # misaligned optional output
+    assert lib.bsa_sparse_attn_refresh(s, *qkv, FAKE, FAKE, *ok_out, ctypes.c_void_p(FAKE.value + 2), NULL, NULL,
+                                       NULL) == _lib.BSA_EINVAL
+    # only 128-token blocks
+    assert lib.bsa_sparse_attn_refresh(Shape(1, 2, 1000, 128, 64), *qkv, FAKE, FAKE, *ok_out, NULL, NULL, NULL,
+                                       NULL) == _lib.BSA_ESHAPE
+    assert lib.bsa_sparse_attn_refresh(Shape(1, 2, 1000, 96, 128), *qkv, FAKE, FAKE, *ok_out, NULL, NULL, NULL,
+                                       NULL) == _lib.BSA_ESHAPE
 
 
 def test_elementwise_validation(lib):
