@@ -55,6 +55,7 @@ def parse_args():
     ap.add_argument("--heads", type=int, default=0,
                     help="run only the first N heads of the workload (small profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-refresh", action="store_true", help="skip the dense-refresh timing")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()
 
@@ -344,6 +345,43 @@ def run_ours(args, w, world, rank, local):
                "ms_per_step": round(e_ms / Ke, 3), "steps": Ke,
                "h2d_bytes_per_step": 3 * B * H * L * D * 2, "d2h_bytes_per_step": B * H * L * D * 2 + B * H * L * 4}
 
+    # dense refresh on the same inputs and kept lists: the single-pass call
+    # against the two-pass path (dense call, sparse call, refinement)
+    refresh = None
+    if not args.no_refresh and blk == 128:
+        qs, ks, vs = (bufs["qh"], bufs["kh"], bufs["vh"]) if w.hilbert else (q, k, v)
+        rb = dict(o_dense=torch.empty_like(q), o_sparse=torch.empty_like(q), R=torch.empty_like(q),
+                  lse_dense=torch.empty((B, H, L), dtype=torch.float32, device=dev),
+                  lse_sparse=torch.empty((B, H, L), dtype=torch.float32, device=dev),
+                  kept_mass=torch.empty((B, H, L), dtype=torch.float32, device=dev))
+
+        def fused():
+            api.sparse_attn_refresh(qs, ks, vs, blk, bufs["idx"], bufs["cnt"], out=rb, status=status)
+
+        def two_pass():
+            api.sparse_attn_fwd(qs, ks, vs, blk, o=rb["o_dense"], lse=rb["lse_dense"], status=status)
+            api.sparse_attn_fwd(qs, ks, vs, blk, bufs["idx"], bufs["cnt"], o=rb["o_sparse"], lse=rb["lse_sparse"],
+                                status=status)
+            api.refresh_refinement(rb["o_dense"], rb["o_sparse"], out=rb["R"])
+
+        times = {}
+        for name, fn in (("fused", fused), ("two_pass", two_pass)):
+            fn()
+            barrier()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record()
+            for _ in range(3):
+                fn()
+            a1.record()
+            barrier()
+            times[name] = a0.elapsed_time(a1) / 3
+        dense_tflop = 4.0 * B * H * L * L * D / 1e12
+        refresh = {"fused_ms": round(times["fused"], 3), "two_pass_ms": round(times["two_pass"], 3),
+                   "dense_tflop": round(dense_tflop, 2),
+                   "fused_dense_equiv_tflops": round(dense_tflop / (times["fused"] * 1e-3), 1),
+                   "calls": "fused: bsa_sparse_attn_refresh; two-pass: dense + sparse bsa_sparse_attn_fwd + "
+                            "bsa_refresh_refinement"}
+
     if status.item() != 0:
         raise RuntimeError(f"attention kernel reported status {status.item()}")
 
@@ -378,7 +416,7 @@ def run_ours(args, w, world, rank, local):
                  "dense_equiv_tflops": round(4.0 * B * H * L * L * D / (attn_avg_ms * 1e-3) / 1e12, 2)},
         "stages_ms": {"score_and_select": round(float(np.mean(sel_ms)), 4), "attention": round(attn_avg_ms, 4),
                       "gather_scatter_and_rest": round(ms_step - attn_avg_ms - float(np.mean(sel_ms)), 4)},
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "refresh": refresh,
         "gpu_launches": LAUNCHES_PER_STEP * K if w.hilbert else (LAUNCHES_PER_STEP - 4) * K,
         "clocks": clk,
     }

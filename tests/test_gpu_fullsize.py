@@ -20,6 +20,7 @@ from block_sparse_attention_logits_b200.synthetic import drift_, make_qkv, rando
 from oracle import attention as oatt
 from oracle import correction as ocor
 from oracle import hilbert as ohil
+from oracle import refresh as oref
 from oracle import scoring as osco
 from oracle import topp as otop
 
@@ -198,3 +199,41 @@ def test_mask_reuse_sweep_720p_shape():
             ref_L = Ls
         torch.cuda.synchronize()
         assert_attention_close(to_np(out), to_np(lse), ref_O, ref_L, f"sweep step {step}")
+
+
+def test_fused_refresh_720p_shape():
+    """The single-pass refresh on the 720P shape (4 heads, Hilbert order, the
+    oracle's kept lists): dense and sparse outputs, R and the kept share on
+    sampled query blocks against the oracle, and every element against the
+    library's two-pass path (dense call, sparse call, refresh_refinement)."""
+    import dataclasses
+    w = dataclasses.replace(configs.WAN14B_720P, H=4)
+    t = make_qkv(w.B, w.H, w.grid, w.D, w.fp)
+    perm, _ = api.reorder_tokens(*w.grid, device=DEV)
+    perm_o, _ = ohil.hilbert_perm(*w.grid)
+    qd, kd, vd = (api.permute_tokens(t[n].to(DEV), perm) for n in "qkv")
+    qn, kn, vn = (ohil.permute_rows(t[n].float().numpy(), perm_o) for n in "qkv")
+    Po = _oracle_probs(qn, kn, w.blk)
+    _, idx_o, cnt_o = otop.select_topp_mask_fast(Po, np.full(w.H, w.p[0], np.float32))
+    idx_d, cnt_d = torch.from_numpy(idx_o).to(DEV), torch.from_numpy(cnt_o).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    od, ld, os_, ls, R, mass = api.sparse_attn_refresh(qd, kd, vd, w.blk, idx_d, cnt_d, status=status)
+    o1, l1 = api.sparse_attn_fwd(qd, kd, vd, w.blk)
+    o2, l2 = api.sparse_attn_fwd(qd, kd, vd, w.blk, idx_d, cnt_d)
+    R2 = api.refresh_refinement(o1, o2)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    units = _sample_units(w.H, w.NB, np.random.default_rng(13), heads=2, per_head=3)
+    Od, Ld, Os, Ls, Rr, Mr = oref.fused_refresh(qn, kn, vn, idx_o, cnt_o, w.blk, units=units)
+    assert_attention_close(to_np(od), to_np(ld), Od, Ld, "fused dense")
+    assert_attention_close(to_np(os_), to_np(ls), Os, Ls, "fused sparse")
+    sel = ~np.isnan(Od)
+    assert np.max(np.abs(to_np(R)[sel] - Rr[sel])) <= 2 * 2e-2
+    msel = ~np.isnan(Ld)
+    assert np.max(np.abs(to_np(mass)[msel] - Mr[msel])) <= 2e-3
+    # against the two-pass path, every element
+    # one bf16 ulp of the output plus the accumulation-order difference
+    assert bool(((od.float() - o1.float()).abs() <= 1e-2 + 2.0 ** -7 * o1.float().abs()).all())
+    assert bool(((os_.float() - o2.float()).abs() <= 1e-2 + 2.0 ** -7 * o2.float().abs()).all())
+    assert (R.float() - R2.float()).abs().max().item() <= 4e-2
+    assert (ld - l1).abs().max().item() <= 1e-3 and (ls - l2).abs().max().item() <= 1e-3

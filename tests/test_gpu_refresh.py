@@ -90,7 +90,10 @@ def test_refresh_agrees_with_the_two_pass_path():
     o1, l1 = api.sparse_attn_fwd(qd, kd, vd, BLK)
     o2, l2 = api.sparse_attn_fwd(qd, kd, vd, BLK, torch.from_numpy(idx).to(DEV), torch.from_numpy(cnt).to(DEV))
     torch.cuda.synchronize()
-    assert np.max(np.abs(od - to_np(o1))) <= 1e-2 and np.max(np.abs(os_ - to_np(o2))) <= 1e-2
+    # one bf16 ulp of the output plus the accumulation-order difference
+    a1, a2 = to_np(o1), to_np(o2)
+    assert np.all(np.abs(od - a1) <= 1e-2 + 2.0 ** -7 * np.abs(a1))
+    assert np.all(np.abs(os_ - a2) <= 1e-2 + 2.0 ** -7 * np.abs(a2))
     assert np.max(np.abs(ld - to_np(l1))) <= 1e-3 and np.max(np.abs(ls - to_np(l2))) <= 1e-3
 
 
