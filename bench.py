@@ -42,6 +42,7 @@ from block_sparse_attention_logits_b200.synthetic import make_qkv, random_bf16  
 METRIC = "block-sparse attn ms/call & TFLOP/s on kept blocks vs bf16 TC peak at 90% sparsity"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 LAUNCHES_PER_STEP = 8  # 3 gathers, pooling, block softmax, selection, attention, scatter
+E2E_MAX_CHUNKS = 8     # head chunks of the pipelined end-to-end step
 
 
 def parse_args():
@@ -311,20 +312,71 @@ def run_ours(args, w, world, rank, local):
     ms_step = elapsed_ms / K
     value = flops * world / (ms_step * 1e-3) / 1e12
 
-    # e2e: host buffers in, result out, through the same API calls
+    # e2e: host buffers in, result out, through the same API calls.  Heads are
+    # independent, so the step runs over head chunks on three streams: the
+    # copy-in of chunk c+1 and the copy-out of chunk c-1 overlap the compute of
+    # chunk c (PCIe carries 3.1 GB per step; the compute takes ~14 ms).
     e2e = None
     if not args.no_e2e:
         o_host = torch.empty((B, H, L, D), dtype=torch.bfloat16, pin_memory=pin)
         lse_host = torch.empty((B, H, L), dtype=torch.float32, pin_memory=pin)
         qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        n_chunks = max(d for d in range(1, E2E_MAX_CHUNKS + 1) if H % d == 0) if B == 1 else 1
+        if (L * (H // n_chunks)) % 4:  # keep every float32 [L] slice 16-byte aligned
+            n_chunks = 1
+        hc = H // n_chunks
+        s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(n_chunks)]
+        ev_cmp = [torch.cuda.Event() for _ in range(n_chunks)]
+        chunk_bufs = []
+        for c in range(n_chunks):
+            hs = slice(c * hc, (c + 1) * hc)
+            # token-row buffers are head slices (16-byte aligned offsets); the
+            # per-block score and list buffers get their own allocations (an
+            # [NB, NB] slice of an odd NB is not 16-byte aligned)
+            chunk_bufs.append({n: (t[:, hs] if n in ("qh", "kh", "vh", "oh", "o", "lse") else
+                                   torch.empty_like(t[:, hs])) for n, t in bufs.items()})
+
+        def chunk_step(c, qi, ki, vi):
+            b = chunk_bufs[c]
+            hs = slice(c * hc, (c + 1) * hc)
+            if w.hilbert:
+                api.permute_tokens(qi, perm, out=b["qh"])
+                api.permute_tokens(ki, perm, out=b["kh"])
+                api.permute_tokens(vi, perm, out=b["vh"])
+                qs, ks, vs = b["qh"], b["kh"], b["vh"]
+            else:
+                qs, ks, vs = qi, ki, vi
+            api.score_blocks(qs, ks, blk, b["qp"], b["kp"], b["probs"])
+            api.select_topp_mask(b["probs"], p, L, blk, D, b["mask"], b["idx"], b["cnt"])
+            api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h[:, hs], alpha[hs], b["oh"], b["lse"],
+                                status=status)
+            if w.hilbert:
+                api.permute_tokens(b["oh"], perm, inverse=True, out=b["o"])
+                return b["o"], b["lse"]
+            return b["oh"], b["lse"]
 
         def e2e_step():
-            qd.copy_(host["q"], non_blocking=True)
-            kd.copy_(host["k"], non_blocking=True)
-            vd.copy_(host["v"], non_blocking=True)
-            o, lse = step(qd, kd, vd)
-            o_host.copy_(o, non_blocking=True)
-            lse_host.copy_(lse, non_blocking=True)
+            cur = torch.cuda.current_stream(dev)
+            for s_ in (s_in, s_cmp, s_out):
+                s_.wait_stream(cur)
+            for c in range(n_chunks):
+                hs = slice(c * hc, (c + 1) * hc)
+                with torch.cuda.stream(s_in):
+                    qd[:, hs].copy_(host["q"][:, hs], non_blocking=True)
+                    kd[:, hs].copy_(host["k"][:, hs], non_blocking=True)
+                    vd[:, hs].copy_(host["v"][:, hs], non_blocking=True)
+                    ev_in[c].record(s_in)
+                with torch.cuda.stream(s_cmp):
+                    s_cmp.wait_event(ev_in[c])
+                    o, lse = chunk_step(c, qd[:, hs], kd[:, hs], vd[:, hs])
+                    ev_cmp[c].record(s_cmp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_cmp[c])
+                    o_host[:, hs].copy_(o, non_blocking=True)
+                    lse_host[:, hs].copy_(lse, non_blocking=True)
+            for s_ in (s_in, s_cmp, s_out):
+                cur.wait_stream(s_)
 
         for _ in range(2):
             e2e_step()
@@ -341,8 +393,14 @@ def run_ours(args, w, world, rank, local):
             t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
             torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
             e_ms = float(t.item())
+        # the pipelined step must give the one-stream step's result
+        o_ref, _ = step(q, k, v)
+        torch.cuda.synchronize()
+        if not torch.equal(o_ref.cpu(), o_host):
+            raise RuntimeError("pipelined end-to-end step disagrees with the one-stream step")
         e2e = {"value": round(flops * world / (e_ms / Ke * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                "ms_per_step": round(e_ms / Ke, 3), "steps": Ke,
+               "pipeline": f"{n_chunks} head chunks on 3 streams (copy-in, compute, copy-out)",
                "h2d_bytes_per_step": 3 * B * H * L * D * 2, "d2h_bytes_per_step": B * H * L * D * 2 + B * H * L * 4}
 
     # dense refresh on the same inputs and kept lists: the single-pass call
