@@ -6,9 +6,10 @@
 //   pool:    one CTA per (block, head, Q|K); 16-byte vector loads, fp32
 //            accumulation, a shared-memory tree over the row groups; the
 //            partial last block divides by its own token count.  HBM-bound.
-//   softmax: one CTA per (16 query blocks, head); pooled rows staged in
-//            shared memory, two query rows per thread, raw logits
-//            written to `probs`, then each warp normalises its rows in place.
+//   softmax: one CTA per (64 query blocks, head); pooled means staged
+//            transposed in shared memory, a 4x4 register tile of logits per
+//            thread, raw logits written to `probs`, then each warp
+//            normalises its rows in place.
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
@@ -55,59 +56,70 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   }
 }
 
-constexpr int kRows = 16;  // query blocks per CTA
-constexpr int kCols = 32;  // key blocks per shared-memory chunk
+constexpr int kTile = 64;   // query blocks per CTA, key blocks per tile
+constexpr int kPad = 68;    // row pitch (floats) of the transposed tiles: 16-byte aligned
 
+// Logits of a 64-query-block strip against all key blocks, 64 key blocks at a
+// time: Q and K means staged transposed ([d][block]) in shared memory, each
+// thread a 4x4 register tile (two 16-byte shared loads per 16 FMAs); raw
+// scaled logits go to `probs`, then each warp normalises 8 of the strip's rows
+// in place (max, exp and sum, divide).
 template <int D>
 __global__ void __launch_bounds__(256) block_softmax_kernel(const float* __restrict__ qp,
                                                             const float* __restrict__ kp, float* __restrict__ probs,
                                                             int NB, float scale) {
-  __shared__ __align__(16) float qs[kRows][D + 4];
-  __shared__ __align__(16) float ks[kCols][D + 4];
+  extern __shared__ __align__(16) float sm[];
+  float* qT = sm;              // [D][kPad]
+  float* kT = sm + D * kPad;   // [D][kPad]
   const size_t bh = blockIdx.y;
-  const int i0 = blockIdx.x * kRows;
+  const int i0 = blockIdx.x * kTile;
   const int tid = threadIdx.x;
-  for (int e = tid; e < kRows * D; e += 256) {
+  // fill: consecutive threads take consecutive d of one block row (coalesced)
+  for (int e = tid; e < kTile * D; e += 256) {
     const int rr = e / D, d = e % D;
-    qs[rr][d] = (i0 + rr < NB) ? qp[(bh * NB + i0 + rr) * D + d] : 0.f;
+    qT[d * kPad + rr] = (i0 + rr < NB) ? __ldg(qp + (bh * NB + i0 + rr) * D + d) : 0.f;
   }
-  // thread -> query rows {ra, ra+8} and one key column of each 32-column
-  // chunk: threads 0..127 take columns 0..15, threads 128..255 columns 16..31
-  const int tr = tid >> 4;
-  const int ra = tr & 7, rb = ra + 8;
-  const int col = (tid & 15) + (tr >= 8 ? 16 : 0);
-  for (int j0 = 0; j0 < NB; j0 += kCols) {
+  const int r0 = (tid >> 4) * 4;  // the thread's 4 query rows ...
+  const int c0 = (tid & 15) * 4;  // ... and 4 key columns within the tile
+  for (int j0 = 0; j0 < NB; j0 += kTile) {
     __syncthreads();
-    for (int e = tid; e < kCols * D; e += 256) {
+    for (int e = tid; e < kTile * D; e += 256) {
       const int cc = e / D, d = e % D;
-      ks[cc][d] = (j0 + cc < NB) ? kp[(bh * NB + j0 + cc) * D + d] : 0.f;
+      kT[d * kPad + cc] = (j0 + cc < NB) ? __ldg(kp + (bh * NB + j0 + cc) * D + d) : 0.f;
     }
     __syncthreads();
-    float s0 = 0.f, s1 = 0.f;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
 #pragma unroll 8
-    for (int d = 0; d < D; d += 4) {
-      const float4 kv = *reinterpret_cast<const float4*>(&ks[col][d]);
-      const float4 a = *reinterpret_cast<const float4*>(&qs[ra][d]);
-      const float4 b = *reinterpret_cast<const float4*>(&qs[rb][d]);
-      s0 = fmaf(a.x, kv.x, s0);
-      s0 = fmaf(a.y, kv.y, s0);
-      s0 = fmaf(a.z, kv.z, s0);
-      s0 = fmaf(a.w, kv.w, s0);
-      s1 = fmaf(b.x, kv.x, s1);
-      s1 = fmaf(b.y, kv.y, s1);
-      s1 = fmaf(b.z, kv.z, s1);
-      s1 = fmaf(b.w, kv.w, s1);
+    for (int d = 0; d < D; ++d) {
+      const float4 qa = *reinterpret_cast<const float4*>(qT + d * kPad + r0);
+      const float4 kb = *reinterpret_cast<const float4*>(kT + d * kPad + c0);
+      const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
+      const float kv[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(qv[a], kv[b], acc[a][b]);
     }
-    const int j = j0 + col;
-    if (j < NB) {
-      if (i0 + ra < NB) probs[(bh * NB + i0 + ra) * NB + j] = s0 * scale;
-      if (i0 + rb < NB) probs[(bh * NB + i0 + rb) * NB + j] = s1 * scale;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int i = i0 + r0 + a;
+      if (i >= NB) break;
+      float* row = probs + (bh * NB + i) * NB;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int j = j0 + c0 + b;
+        if (j < NB) row[j] = acc[a][b] * scale;
+      }
     }
   }
   __syncthreads();
-  // row softmax: warp w handles rows w and w+8
+  // row softmax: warp w normalises rows w, w+8, ...
   const int w = tid >> 5, lane = tid & 31;
-  for (int rr = w; rr < kRows; rr += 8) {
+  for (int rr = w; rr < kTile; rr += 8) {
     const int i = i0 + rr;
     if (i >= NB) break;
     float* row = probs + (bh * NB + i) * NB;
@@ -143,12 +155,23 @@ cudaError_t launch_pool(const bsa_shape& s, const __nv_bfloat16* q, const __nv_b
 cudaError_t launch_block_softmax(const bsa_shape& s, const float* qp, const float* kp, float* probs,
                                  cudaStream_t st) {
   const int NB = n_blocks(s.L, s.blk);
-  dim3 grid((NB + kRows - 1) / kRows, s.B * s.H);
+  dim3 grid((NB + kTile - 1) / kTile, s.B * s.H);
   const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(s.D)));
+  static bool configured = false;
+  if (!configured) {
+    // 69.6 KB of transposed tiles at D = 128: above the default 48 KB
+    cudaError_t e = cudaFuncSetAttribute(block_softmax_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         2 * 128 * kPad * 4);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(block_softmax_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               2 * 64 * kPad * 4);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
   if (s.D == 128)
-    block_softmax_kernel<128><<<grid, 256, 0, st>>>(qp, kp, probs, NB, scale);
+    block_softmax_kernel<128><<<grid, 256, 2 * 128 * kPad * 4, st>>>(qp, kp, probs, NB, scale);
   else
-    block_softmax_kernel<64><<<grid, 256, 0, st>>>(qp, kp, probs, NB, scale);
+    block_softmax_kernel<64><<<grid, 256, 2 * 64 * kPad * 4, st>>>(qp, kp, probs, NB, scale);
   return cudaGetLastError();
 }
 
