@@ -32,9 +32,11 @@ Modules:
   correction  -- dense-minus-sparse refinement and the alpha-scaled correction
   refresh     -- the outputs of a single-pass dense refresh (dense and sparse
                  attention, refinement, exact kept attention mass)
+  reuse       -- query-key drift of the block means, and scoring / selection
+                 restricted to an earlier candidate set
 
 Every function carries a "Pinned by" note naming the tests in
 ``tests/test_oracle.py`` that tie it to something other than itself.
 """
 
-from . import hilbert, scoring, topp, attention, correction, refresh  # noqa: F401
+from . import hilbert, scoring, topp, attention, correction, refresh, reuse  # noqa: F401

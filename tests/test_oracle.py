@@ -20,6 +20,7 @@ from oracle import attention as oatt
 from oracle import correction as ocor
 from oracle import hilbert as ohil
 from oracle import refresh as oref
+from oracle import reuse as oreu
 from oracle import scoring as osco
 from oracle import topp as otop
 
@@ -454,6 +455,113 @@ def test_planted_mistake_inverted_mass_is_caught(monkeypatch):
     monkeypatch.setattr(oref, "kept_mass", lambda ls, ld: np.exp(np.asarray(ld) - np.asarray(ls)))
     with pytest.raises(AssertionError):
         test_refresh_mass_closed_form_for_constant_keys()
+
+
+# ------------------------------------------------------------- mask reuse
+
+def test_drift_closed_forms():
+    rng = np.random.default_rng(31)
+    qb, kb = rng.standard_normal((2, 3, 7, 8)), rng.standard_normal((2, 3, 7, 8))
+    assert np.all(oreu.block_drift(qb, kb, qb, kb) == 0)
+    # uniform scaling of the query means by c: drift |c - 1|
+    for c in (0.5, 1.1, 3.0):
+        assert np.allclose(oreu.block_drift(qb, kb, c * qb, kb), abs(c - 1), atol=1e-12)
+    # one perturbed entry: its size over the reference norm; the larger side wins
+    kq = kb.copy()
+    kq[1, 2, 3, 4] += 0.25
+    d = oreu.block_drift(qb, kb, qb, kq)
+    assert np.isclose(d[1, 2], 0.25 / np.sqrt((kb[1, 2] ** 2).sum()), atol=1e-12)
+    assert np.all(np.delete(d.ravel(), 1 * 3 + 2) == 0)
+    both = oreu.block_drift(qb, kb, 1.2 * qb, kq)
+    assert np.isclose(both[1, 2], max(0.2, d[1, 2]))
+    z = np.zeros_like(qb)
+    assert np.all(oreu.block_drift(z, z, z, z) == 0) and np.all(np.isinf(oreu.block_drift(z, kb, qb, kb)))
+
+
+def test_restricted_scoring_all_candidates_and_scipy():
+    import scipy.special
+    rng = np.random.default_rng(32)
+    B, H, L, D, blk = 1, 2, 300, 16, 32
+    q, k = rng.standard_normal((B, H, L, D)), rng.standard_normal((B, H, L, D))
+    qb, kb, P = osco.score_blocks(q, k, blk)
+    NB = qb.shape[2]
+    allc = np.ones((B, H, NB, NB), np.uint8)
+    assert np.allclose(oreu.restricted_probs(qb, kb, allc), P, rtol=1e-6, atol=0)
+    cand = rng.random((B, H, NB, NB)) < 0.4
+    cand[0, 1, 3] = False  # a row without candidates
+    Pr = oreu.restricted_probs(qb, kb, cand)
+    assert np.all(Pr[~cand] == 0) and np.all(Pr[0, 1, 3] == 0)
+    s = osco.block_logits(qb, kb)
+    for (b, h, i) in [(0, 0, 0), (0, 1, 5), (0, 0, NB - 1)]:
+        sel = cand[b, h, i]
+        if sel.any():
+            ref = scipy.special.softmax(s[b, h, i, sel])
+            assert np.allclose(Pr[b, h, i, sel], ref, rtol=1e-6)
+            assert abs(Pr[b, h, i].astype(np.float64).sum() - 1) < 1e-6
+
+
+def test_restricted_selection_all_candidates_equals_unrestricted():
+    rng = np.random.default_rng(33)
+    P = rng.dirichlet(np.ones(12), size=(1, 2, 12)).astype(np.float32)
+    pv = np.array([0.7, 0.95], np.float32)
+    allc = np.ones(P.shape, np.uint8)
+    a = otop.select_topp_mask_fast(P, pv)
+    b = oreu.select_topp_mask_restricted(P, pv, allc)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_restricted_selection_golden_row_and_edges():
+    P = np.array([0.4, 0.3, 0.2, 0.1], np.float32)
+    cand = np.array([0, 1, 0, 1], np.uint8)
+    # target 0.7 of the candidates' mass 0.4: block 1 alone (0.3) reaches it
+    kept, k = oreu.select_row_restricted(P, 0.7, cand)
+    assert k == 1 and list(kept) == [1]
+    kept, k = oreu.select_row_restricted(P, 0.9, cand)
+    assert k == 2 and list(kept) == [1, 3]
+    kept, k = oreu.select_row_restricted(P, 1.0, cand)
+    assert list(kept) == [1, 3]
+    kept, k = oreu.select_row_restricted(P, 0.5, np.zeros(4, np.uint8))
+    assert k == 0 and kept.size == 0
+
+
+@pytest.mark.parametrize("seed", [34, 35, 36])
+def test_restricted_selection_matches_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    nb = 9
+    P = rng.dirichlet(np.ones(nb)).astype(np.float32)
+    cand = np.flatnonzero(rng.random(nb) < 0.6)
+    if cand.size == 0:
+        cand = np.array([0])
+    cm = np.zeros(nb, np.uint8)
+    cm[cand] = 1
+    p = np.float32(rng.uniform(0.3, 0.95))
+    kept, k = oreu.select_row_restricted(P, p, cm)
+    u = otop.fixed_point_mass(otop.clamp_probs(P))
+    T = int(np.ceil(np.float64(p) * np.float64(int(u[cand].sum()))))
+    assert set(kept) <= set(cand)
+    assert int(u[kept].sum()) >= T
+    for r in range(1, k):   # no smaller candidate subset reaches T
+        for sub in itertools.combinations(cand, r):
+            assert int(u[list(sub)].sum()) < T
+    # the kept set is the ordered top-k of the candidates
+    order = sorted(cand, key=lambda j: (-float(P[j]), j))
+    assert sorted(order[:k]) == list(kept)
+
+
+def test_planted_mistake_restricted_target_is_caught(monkeypatch):
+    def full_row_target(P_row, p, cand_row):
+        cand = np.flatnonzero(np.asarray(cand_row).astype(bool))
+        Pc = otop.clamp_probs(P_row)
+        u = otop.fixed_point_mass(Pc)
+        T = int(np.ceil(np.float64(np.float32(p)) * np.float64(int(u.sum()))))   # wrong total
+        order = sorted(cand, key=lambda j: (-float(Pc[j]), j))
+        csum = np.cumsum(u[order])
+        k = int(np.argmax(csum >= T)) + 1 if csum[-1] >= T else len(order)
+        return np.sort(np.array(order[:k], np.int32)), k
+    monkeypatch.setattr(oreu, "select_row_restricted", full_row_target)
+    with pytest.raises(AssertionError):
+        test_restricted_selection_golden_row_and_edges()
 
 
 # ------------------------------------------------- planted mistakes are caught
