@@ -11,7 +11,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbsa.so")
 
 EXPORTS = (
-    "bsa_strerror", "bsa_version", "bsa_score_blocks", "bsa_select_topp_mask",
+    "bsa_strerror", "bsa_version", "bsa_score_blocks", "bsa_score_blocks_restricted", "bsa_block_drift",
+    "bsa_select_topp_mask", "bsa_select_topp_mask_restricted",
     "bsa_reorder_workspace_bytes", "bsa_reorder_tokens", "bsa_reorder_tokens_noalloc", "bsa_permute_tokens",
     "bsa_sparse_attn_fwd", "bsa_sparse_attn_refresh", "bsa_refresh_refinement", "bsa_apply_correction",
 )
@@ -52,7 +53,10 @@ def load():
         "bsa_strerror": (ctypes.c_char_p, [_I]),
         "bsa_version": (_I, []),
         "bsa_score_blocks": (_I, [Shape, _P, _P, _P, _P, _P, _P]),
+        "bsa_score_blocks_restricted": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P]),
+        "bsa_block_drift": (_I, [Shape, _P, _P, _P, _P, _P, _P]),
         "bsa_select_topp_mask": (_I, [Shape, _P, ctypes.POINTER(ctypes.c_float), _P, _P, _P, _P]),
+        "bsa_select_topp_mask_restricted": (_I, [Shape, _P, ctypes.POINTER(ctypes.c_float), _P, _P, _P, _P, _P]),
         "bsa_reorder_workspace_bytes": (_SZ, [_I, _I, _I]),
         "bsa_reorder_tokens": (_I, [_I, _I, _I, _P, _P, _P, _SZ, _P]),
         "bsa_reorder_tokens_noalloc": (_I, [_I, _I, _I, _P, _P, _P]),

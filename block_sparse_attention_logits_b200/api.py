@@ -55,11 +55,12 @@ def _shape(q, blk):
     return Shape(B, H, L, D, blk)
 
 
-def score_blocks(q, k, blk, q_pool=None, k_pool=None, probs=None):
+def score_blocks(q, k, blk, q_pool=None, k_pool=None, probs=None, candidates=None):
     """Block means of Q and K and the per-query-block softmax of their logits.
 
     q, k: bf16 [B,H,L,D].  Returns (q_pool, k_pool, probs): float32
-    [B,H,NB,D], [B,H,NB,D], [B,H,NB,NB].
+    [B,H,NB,D], [B,H,NB,D], [B,H,NB,NB].  With `candidates` (uint8
+    [B,H,NB,NB]) each row's softmax runs over its candidate blocks only.
     """
     B, H, L, D = q.shape
     nb = n_blocks(L, blk)
@@ -72,17 +73,39 @@ def score_blocks(q, k, blk, q_pool=None, k_pool=None, probs=None):
     _need(q_pool, torch.float32, (B, H, nb, D), "q_pool")
     _need(k_pool, torch.float32, (B, H, nb, D), "k_pool")
     _need(probs, torch.float32, (B, H, nb, nb), "probs")
-    check("bsa_score_blocks", _lib.load().bsa_score_blocks(
-        _shape(q, blk), _ptr(q), _ptr(k), _ptr(q_pool), _ptr(k_pool), _ptr(probs), _stream()))
+    if candidates is None:
+        check("bsa_score_blocks", _lib.load().bsa_score_blocks(
+            _shape(q, blk), _ptr(q), _ptr(k), _ptr(q_pool), _ptr(k_pool), _ptr(probs), _stream()))
+    else:
+        _need(candidates, torch.uint8, (B, H, nb, nb), "candidates")
+        check("bsa_score_blocks_restricted", _lib.load().bsa_score_blocks_restricted(
+            _shape(q, blk), _ptr(q), _ptr(k), _ptr(candidates), _ptr(q_pool), _ptr(k_pool), _ptr(probs),
+            _stream()))
     return q_pool, k_pool, probs
 
 
-def select_topp_mask(probs, p, L, blk, D=128, mask=None, kept_idx=None, kept_cnt=None):
+def block_drift(q_pool_ref, k_pool_ref, q_pool, k_pool, L, blk, drift=None):
+    """Per-head query-key drift of the block means since a reference step:
+    max of the relative Frobenius changes of the Q and K means.  Inputs
+    float32 [B,H,NB,D]; returns float32 [B*H] on the device."""
+    B, H, nb, D = q_pool.shape
+    for name, t in (("q_pool_ref", q_pool_ref), ("k_pool_ref", k_pool_ref), ("q_pool", q_pool), ("k_pool", k_pool)):
+        _need(t, torch.float32, (B, H, nb, D), name)
+    drift = drift if drift is not None else torch.empty((B * H,), dtype=torch.float32, device=q_pool.device)
+    _need(drift, torch.float32, (B * H,), "drift")
+    check("bsa_block_drift", _lib.load().bsa_block_drift(
+        Shape(B, H, L, D, blk), _ptr(q_pool_ref), _ptr(k_pool_ref), _ptr(q_pool), _ptr(k_pool), _ptr(drift),
+        _stream()))
+    return drift
+
+
+def select_topp_mask(probs, p, L, blk, D=128, mask=None, kept_idx=None, kept_cnt=None, candidates=None):
     """Cumulative top-p selection per query block.
 
     probs: float32 [B,H,NB,NB]; p: per-head thresholds (sequence of H floats
     in (0,1]) or one float for every head.  Returns (mask uint8, kept_idx
-    int32, kept_cnt int32).
+    int32, kept_cnt int32).  With `candidates` (uint8 [B,H,NB,NB]) the search
+    runs over each row's candidate blocks only.
     """
     B, H, nb, _ = probs.shape
     _need(probs, torch.float32, (B, H, nb, nb), "probs")
@@ -99,8 +122,14 @@ def select_topp_mask(probs, p, L, blk, D=128, mask=None, kept_idx=None, kept_cnt
     _need(kept_idx, torch.int32, (B, H, nb, nb), "kept_idx")
     _need(kept_cnt, torch.int32, (B, H, nb), "kept_cnt")
     parr = (ctypes.c_float * H)(*p)
-    check("bsa_select_topp_mask", _lib.load().bsa_select_topp_mask(
-        Shape(B, H, L, D, blk), _ptr(probs), parr, _ptr(mask), _ptr(kept_idx), _ptr(kept_cnt), _stream()))
+    if candidates is None:
+        check("bsa_select_topp_mask", _lib.load().bsa_select_topp_mask(
+            Shape(B, H, L, D, blk), _ptr(probs), parr, _ptr(mask), _ptr(kept_idx), _ptr(kept_cnt), _stream()))
+    else:
+        _need(candidates, torch.uint8, (B, H, nb, nb), "candidates")
+        check("bsa_select_topp_mask_restricted", _lib.load().bsa_select_topp_mask_restricted(
+            Shape(B, H, L, D, blk), _ptr(probs), parr, _ptr(candidates), _ptr(mask), _ptr(kept_idx),
+            _ptr(kept_cnt), _stream()))
     return mask, kept_idx, kept_cnt
 
 

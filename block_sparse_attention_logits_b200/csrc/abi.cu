@@ -73,13 +73,42 @@ int bsa_score_blocks(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, float* q
   const auto* qb = reinterpret_cast<const __nv_bfloat16*>(q);
   const auto* kb = reinterpret_cast<const __nv_bfloat16*>(k);
   if (cudaError_t e = bsa::launch_pool(s, qb, kb, q_pool, k_pool, st)) return from_cuda(e);
-  return from_cuda(bsa::launch_block_softmax(s, q_pool, k_pool, probs, st));
+  return from_cuda(bsa::launch_block_softmax(s, q_pool, k_pool, probs, nullptr, st));
 }
 
-int bsa_select_topp_mask(bsa_shape s, const float* probs, const float* p_host, uint8_t* mask, int32_t* kept_idx,
-                         int32_t* kept_cnt, bsa_stream stream) {
+int bsa_score_blocks_restricted(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const uint8_t* candidates,
+                                float* q_pool, float* k_pool, float* probs, bsa_stream stream) {
+  if (!q || !k || !candidates || !q_pool || !k_pool || !probs) return BSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(candidates) || !aligned16(q_pool) || !aligned16(k_pool) ||
+      !aligned16(probs))
+    return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (int r = check_device()) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const auto* qb = reinterpret_cast<const __nv_bfloat16*>(q);
+  const auto* kb = reinterpret_cast<const __nv_bfloat16*>(k);
+  if (cudaError_t e = bsa::launch_pool(s, qb, kb, q_pool, k_pool, st)) return from_cuda(e);
+  return from_cuda(bsa::launch_block_softmax(s, q_pool, k_pool, probs, candidates, st));
+}
+
+int bsa_block_drift(bsa_shape s, const float* q_pool_ref, const float* k_pool_ref, const float* q_pool,
+                    const float* k_pool, float* drift, bsa_stream stream) {
+  if (!q_pool_ref || !k_pool_ref || !q_pool || !k_pool || !drift) return BSA_EINVAL;
+  if (!aligned16(q_pool_ref) || !aligned16(k_pool_ref) || !aligned16(q_pool) || !aligned16(k_pool) ||
+      !aligned16(drift))
+    return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (int r = check_device()) return r;
+  return from_cuda(bsa::launch_drift(s, q_pool_ref, k_pool_ref, q_pool, k_pool, drift,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+int select_common(bsa_shape s, const float* probs, const float* p_host, const uint8_t* cand, uint8_t* mask,
+                  int32_t* kept_idx, int32_t* kept_cnt, bsa_stream stream) {
   if (!probs || !p_host || !mask || !kept_idx || !kept_cnt) return BSA_EINVAL;
   if (!aligned16(probs) || !aligned16(mask) || !aligned16(kept_idx) || !aligned16(kept_cnt)) return BSA_EINVAL;
+  if (cand && !aligned16(cand)) return BSA_EINVAL;
   if (int r = check_block_shape(s)) return r;
   if (s.H > bsa::kMaxHeadsP) return BSA_ESHAPE;
   bsa::TopP tp;
@@ -90,7 +119,20 @@ int bsa_select_topp_mask(bsa_shape s, const float* probs, const float* p_host, u
     tp.p[h] = p;
   }
   if (int r = check_device()) return r;
-  return from_cuda(bsa::launch_select(s, probs, tp, mask, kept_idx, kept_cnt, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(
+      bsa::launch_select(s, probs, tp, cand, mask, kept_idx, kept_cnt, reinterpret_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+int bsa_select_topp_mask(bsa_shape s, const float* probs, const float* p_host, uint8_t* mask, int32_t* kept_idx,
+                         int32_t* kept_cnt, bsa_stream stream) {
+  return select_common(s, probs, p_host, nullptr, mask, kept_idx, kept_cnt, stream);
+}
+
+int bsa_select_topp_mask_restricted(bsa_shape s, const float* probs, const float* p_host, const uint8_t* candidates,
+                                    uint8_t* mask, int32_t* kept_idx, int32_t* kept_cnt, bsa_stream stream) {
+  if (!candidates) return BSA_EINVAL;
+  return select_common(s, probs, p_host, candidates, mask, kept_idx, kept_cnt, stream);
 }
 
 size_t bsa_reorder_workspace_bytes(int T, int Hh, int W) { return bsa::hilbert_workspace_bytes(T, Hh, W); }

@@ -22,10 +22,15 @@ inline int n_blocks(int L, int blk) { return (L + blk - 1) / blk; }
 // launchers (return cudaSuccess or the launch error)
 cudaError_t launch_pool(const bsa_shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, float* qp, float* kp,
                         cudaStream_t st);
+// cand: optional uint8 [B,H,NB,NB]; non-null restricts each row's softmax and
+// top-p search to its candidate blocks (the others get P = 0 / are never kept)
 cudaError_t launch_block_softmax(const bsa_shape& s, const float* qp, const float* kp, float* probs,
-                                 cudaStream_t st);
-cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p, uint8_t* mask, int32_t* idx,
-                          int32_t* cnt, cudaStream_t st);
+                                 const uint8_t* cand, cudaStream_t st);
+cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p, const uint8_t* cand, uint8_t* mask,
+                          int32_t* idx, int32_t* cnt, cudaStream_t st);
+// drift[b*H + h] of the block means against reference means, [B,H,NB,D] each
+cudaError_t launch_drift(const bsa_shape& s, const float* qp_ref, const float* kp_ref, const float* qp,
+                         const float* kp, float* drift, cudaStream_t st);
 size_t hilbert_workspace_bytes(int T, int Hh, int W);
 cudaError_t launch_hilbert(int T, int Hh, int W, int32_t* perm, int32_t* inv, void* ws, cudaStream_t st);
 cudaError_t launch_permute(const bsa_shape& s, const __nv_bfloat16* x, const int32_t* perm, __nv_bfloat16* y,

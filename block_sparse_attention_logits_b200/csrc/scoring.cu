@@ -67,7 +67,7 @@ constexpr int kPad = 68;    // row pitch (floats) of the transposed tiles: 16-by
 template <int D>
 __global__ void __launch_bounds__(256) block_softmax_kernel(const float* __restrict__ qp,
                                                             const float* __restrict__ kp, float* __restrict__ probs,
-                                                            int NB, float scale) {
+                                                            const uint8_t* __restrict__ cand, int NB, float scale) {
   extern __shared__ __align__(16) float sm[];
   float* qT = sm;              // [D][kPad]
   float* kT = sm + D * kPad;   // [D][kPad]
@@ -123,19 +123,62 @@ __global__ void __launch_bounds__(256) block_softmax_kernel(const float* __restr
     const int i = i0 + rr;
     if (i >= NB) break;
     float* row = probs + (bh * NB + i) * NB;
+    const uint8_t* crow = cand ? cand + (bh * NB + i) * NB : nullptr;
     float m = -INFINITY;
-    for (int j = lane; j < NB; j += 32) m = fmaxf(m, row[j]);
+    for (int j = lane; j < NB; j += 32)
+      if (!crow || crow[j]) m = fmaxf(m, row[j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float sum = 0.f;
     for (int j = lane; j < NB; j += 32) {
-      const float e = expf(row[j] - m);
+      const float e = (!crow || crow[j]) ? expf(row[j] - m) : 0.f;
       row[j] = e;
       sum += e;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    for (int j = lane; j < NB; j += 32) row[j] = row[j] / sum;
+    // a row without candidates (sum 0) stays all zeros
+    for (int j = lane; j < NB; j += 32) row[j] = sum > 0.f ? row[j] / sum : 0.f;
+  }
+}
+
+// Query-key drift of one head (head-wise top-p abstract, Temporal Mask Reuse):
+// max of ||x - x_ref||_F / ||x_ref||_F over x = block means of Q and of K,
+// with 0/0 -> 0 and a change from an all-zero reference -> +inf.  One CTA per
+// (b, h); float64 sums of squares.
+__global__ void __launch_bounds__(256) drift_kernel(const float* __restrict__ qr, const float* __restrict__ kr,
+                                                    const float* __restrict__ q, const float* __restrict__ k,
+                                                    float* __restrict__ drift, long long n) {
+  const size_t base = static_cast<size_t>(blockIdx.x) * n;
+  double s[4] = {0.0, 0.0, 0.0, 0.0};  // |dq|^2, |q_ref|^2, |dk|^2, |k_ref|^2
+  for (long long e = threadIdx.x; e < n; e += 256) {
+    const double a = qr[base + e], b = q[base + e], c = kr[base + e], d = k[base + e];
+    s[0] += (b - a) * (b - a);
+    s[1] += a * a;
+    s[2] += (d - c) * (d - c);
+    s[3] += c * c;
+  }
+  __shared__ double part[4][8];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    double v = s[t];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) part[t][threadIdx.x >> 5] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot[4];
+    for (int t = 0; t < 4; ++t) {
+      tot[t] = 0.0;
+      for (int w = 0; w < 8; ++w) tot[t] += part[t][w];
+    }
+    double r = 0.0;
+    for (int t = 0; t < 4; t += 2) {
+      const double rel = tot[t] == 0.0 ? 0.0 : (tot[t + 1] == 0.0 ? INFINITY : sqrt(tot[t] / tot[t + 1]));
+      r = rel > r ? rel : r;
+    }
+    drift[blockIdx.x] = static_cast<float>(r);
   }
 }
 
@@ -153,7 +196,7 @@ cudaError_t launch_pool(const bsa_shape& s, const __nv_bfloat16* q, const __nv_b
 }
 
 cudaError_t launch_block_softmax(const bsa_shape& s, const float* qp, const float* kp, float* probs,
-                                 cudaStream_t st) {
+                                 const uint8_t* cand, cudaStream_t st) {
   const int NB = n_blocks(s.L, s.blk);
   dim3 grid((NB + kTile - 1) / kTile, s.B * s.H);
   const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(s.D)));
@@ -169,9 +212,16 @@ cudaError_t launch_block_softmax(const bsa_shape& s, const float* qp, const floa
     configured = true;
   }
   if (s.D == 128)
-    block_softmax_kernel<128><<<grid, 256, 2 * 128 * kPad * 4, st>>>(qp, kp, probs, NB, scale);
+    block_softmax_kernel<128><<<grid, 256, 2 * 128 * kPad * 4, st>>>(qp, kp, probs, cand, NB, scale);
   else
-    block_softmax_kernel<64><<<grid, 256, 2 * 64 * kPad * 4, st>>>(qp, kp, probs, NB, scale);
+    block_softmax_kernel<64><<<grid, 256, 2 * 64 * kPad * 4, st>>>(qp, kp, probs, cand, NB, scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_drift(const bsa_shape& s, const float* qp_ref, const float* kp_ref, const float* qp,
+                         const float* kp, float* drift, cudaStream_t st) {
+  const long long n = static_cast<long long>(n_blocks(s.L, s.blk)) * s.D;
+  drift_kernel<<<s.B * s.H, 256, 0, st>>>(qp_ref, kp_ref, qp, kp, drift, n);
   return cudaGetLastError();
 }
 

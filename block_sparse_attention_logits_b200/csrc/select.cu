@@ -13,6 +13,11 @@
 // order while the running mass is still below T (a warp prefix scan).  All
 // sums are exact uint64 integer sums, so the result does not depend on the
 // order of summation and equals the sequential definition bit for bit.
+//
+// Restricted form (GSRS abstract: later searches restricted to an early
+// candidate set): with a candidate mask the search runs over the candidate
+// blocks only -- the others carry key 0 and mass 0 and are never kept, the
+// target is p times the candidates' mass, p = 1 keeps every candidate.
 #include "internal.cuh"
 
 namespace bsa {
@@ -45,6 +50,7 @@ __device__ __forceinline__ uint64_t warp_sum(uint64_t v) {
 }
 
 __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ probs, const __grid_constant__ TopP tp,
+                                                     const uint8_t* __restrict__ cand,
                                                      uint8_t* __restrict__ mask, int32_t* __restrict__ kept_idx,
                                                      int32_t* __restrict__ kept_cnt, int H, int NB, long long rows,
                                                      int nbp) {
@@ -62,7 +68,10 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ p
   uint8_t* mrow = mask + row * NB;
   int32_t* irow = kept_idx + row * NB;
 
-  if (p == 1.0f) {
+  // candidates (optional): the other blocks are never kept; their key and
+  // mass are 0, so the search and the target ignore them
+  const uint8_t* crow = cand ? cand + row * NB : nullptr;
+  if (p == 1.0f && !crow) {
     for (int j = lane; j < NB; j += 32) {
       mrow[j] = 1;
       irow[j] = j;
@@ -73,7 +82,8 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ p
 
   uint64_t total = 0;
   for (int j = lane; j < NB; j += 32) {
-    const uint32_t key = prob_key(__ldg(P + j));
+    const bool in = !crow || crow[j];
+    const uint32_t key = in ? prob_key(__ldg(P + j)) : 0u;
     const uint64_t u = fixed_mass(key);
     keys[j] = key;
     us[j] = u;
@@ -84,12 +94,19 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ p
   const uint64_t T = static_cast<uint64_t>(ceil(static_cast<double>(p) * static_cast<double>(total)));
 
   uint32_t tau;
-  if (T == 0) {
-    // nothing to reach: keep the first block of the order (max key, lowest index)
+  if (p == 1.0f) {
+    // every candidate is kept
+    for (int j = lane; j < NB; j += 32)
+      if (crow[j]) keys[j] = kSelected;
+    tau = kSelected - 1u;
+  } else if (T == 0) {
+    // nothing to reach: keep the first block of the order (max key, lowest
+    // index) among the eligible blocks; none if there is no candidate
     uint32_t best_key = 0;
     int best_j = 0x7FFFFFFF;
     for (int j = lane; j < NB; j += 32) {
       const uint32_t kj = keys[j];
+      if (crow && !crow[j]) continue;
       if (kj > best_key || (kj == best_key && j < best_j)) {
         best_key = kj;
         best_j = j;
@@ -105,7 +122,7 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ p
       }
     }
     __syncwarp();
-    if (lane == 0) keys[best_j] = kSelected;
+    if (lane == 0 && best_j < NB) keys[best_j] = kSelected;
     tau = kSelected - 1u;
   } else {
     // largest tau with sum_{key >= tau} u >= T (bit 31 is never set in a key)
@@ -151,8 +168,8 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ p
 
 }  // namespace
 
-cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p, uint8_t* mask, int32_t* idx,
-                          int32_t* cnt, cudaStream_t st) {
+cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p, const uint8_t* cand, uint8_t* mask,
+                          int32_t* idx, int32_t* cnt, cudaStream_t st) {
   const int NB = n_blocks(s.L, s.blk);
   const int nbp = (NB + 1) & ~1;
   const size_t per_warp = static_cast<size_t>(nbp) * 12;
@@ -169,7 +186,8 @@ cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p,
   }
   const long long rows = static_cast<long long>(s.B) * s.H * NB;
   const long long grid = (rows + warps - 1) / warps;
-  select_kernel<<<static_cast<unsigned>(grid), warps * 32, smem, st>>>(probs, p, mask, idx, cnt, s.H, NB, rows, nbp);
+  select_kernel<<<static_cast<unsigned>(grid), warps * 32, smem, st>>>(probs, p, cand, mask, idx, cnt, s.H, NB, rows,
+                                                                       nbp);
   return cudaGetLastError();
 }
 

@@ -164,6 +164,51 @@ BSA_API int bsa_permute_tokens(bsa_shape s, const bsa_bf16* x, const int32_t* pe
                        bsa_stream stream);
 
 /*
+ * bsa_block_drift -- query-key drift of each head since a reference step.
+ * Defines: Temporal Mask Reuse skips mask prediction based on query-key drift
+ * (head-wise adaptive top-p abstract).  From the block means that
+ * bsa_score_blocks writes (float32 [B,H,NB,D]) at the step that predicted the
+ * mask (q_pool_ref, k_pool_ref) and at the current step (q_pool, k_pool):
+ *   drift[b*H + h] = max( ||q_pool - q_pool_ref||_F / ||q_pool_ref||_F ,
+ *                         ||k_pool - k_pool_ref||_F / ||k_pool_ref||_F )
+ * over the head's [NB, D] means (0/0 -> 0; a change from an all-zero
+ * reference -> +inf).  Output drift: device float32 [B*H].  The caller keeps
+ * a head's mask while its drift stays at or below its threshold.
+ * Errors: BSA_EINVAL on null/misaligned pointers; BSA_ESHAPE; BSA_ENODEV.
+ */
+BSA_API int bsa_block_drift(bsa_shape s, const float* q_pool_ref, const float* k_pool_ref, const float* q_pool,
+                    const float* k_pool, float* drift, bsa_stream stream);
+
+/*
+ * bsa_score_blocks_restricted -- bsa_score_blocks with each query block's
+ * softmax taken over its candidate key blocks only.
+ * Defines: later top-p searches restricted to an early candidate set (GSRS
+ * abstract).  candidates: device uint8 [B,H,NB,NB], nonzero = candidate (for
+ * instance an earlier mask, possibly widened).  probs[b,h,i,j] = softmax over
+ * the candidates j of row i of the block logits, 0 for non-candidates; a row
+ * without candidates is all zeros.  Pooled means as bsa_score_blocks.
+ * Errors: as bsa_score_blocks, BSA_EINVAL for a null candidates pointer.
+ */
+BSA_API int bsa_score_blocks_restricted(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const uint8_t* candidates,
+                                float* q_pool, float* k_pool, float* probs, bsa_stream stream);
+
+/*
+ * bsa_select_topp_mask_restricted -- top-p selection over the candidate key
+ * blocks of each row.
+ * Defines: GSRS abstract (search restricted to an early candidate set) with
+ * the top-p rule of bsa_select_topp_mask: candidates ordered by (P desc,
+ * index asc), target T = ceil(p_h * sum of the candidates' fixed-point
+ * masses), the shortest prefix reaching T is kept (at least one block when a
+ * candidate exists); p_h == 1 keeps every candidate; non-candidates are never
+ * kept; a row without candidates keeps nothing (count 0).
+ * Arguments and errors as bsa_select_topp_mask, plus candidates (device uint8
+ * [B,H,NB,NB], required).
+ */
+BSA_API int bsa_select_topp_mask_restricted(bsa_shape s, const float* probs, const float* p_host,
+                                    const uint8_t* candidates, uint8_t* mask, int32_t* kept_idx,
+                                    int32_t* kept_cnt, bsa_stream stream);
+
+/*
  * bsa_sparse_attn_fwd -- block-sparse attention forward with an optional
  * fused correction epilogue.
  * Defines: computing the selected connections densely and skipping the

@@ -107,6 +107,23 @@ def test_attention_validation(lib):
                                    NULL, NULL) == _lib.BSA_ESHAPE
 
 
+def test_reuse_validation(lib):
+    s = Shape(1, 2, 1000, 128, 128)
+    ph = (ctypes.c_float * 2)(0.9, 0.9)
+    # restricted calls require the candidate mask
+    assert lib.bsa_score_blocks_restricted(s, FAKE, FAKE, NULL, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_select_topp_mask_restricted(s, FAKE, ph, NULL, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_select_topp_mask_restricted(s, FAKE, (ctypes.c_float * 2)(0.9, 1.5), FAKE, FAKE, FAKE, FAKE,
+                                               NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_score_blocks_restricted(Shape(1, 2, 1000, 96, 128), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                           NULL) == _lib.BSA_ESHAPE
+    for miss in range(5):
+        args = [FAKE] * 5
+        args[miss] = NULL
+        assert lib.bsa_block_drift(s, *args, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_block_drift(Shape(1, 2, 1000, 128, 96), FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == _lib.BSA_ESHAPE
+
+
 def test_refresh_validation(lib):
     s = Shape(1, 2, 1000, 128, 128)
     qkv = (FAKE, FAKE, FAKE)
