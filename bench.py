@@ -70,6 +70,28 @@ def dist_info():
     return world, rank, local
 
 
+def init_dist(world, backend="nccl"):
+    """One process group per job (rendezvous from MASTER_ADDR/PORT); a short
+    timeout so that ranks waiting on a dead peer end with an error."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+
+
+def max_over_ranks(ms, world, dev=None):
+    """The job's time is its slowest rank's."""
+    if world <= 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(flops_per_rank, ms_per_step, world):
+    """Whole-job throughput in TFLOP/s: every rank runs the workload (weak scaling)."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -218,9 +240,7 @@ def run_ours(args, w, world, rank, local):
     from block_sparse_attention_logits_b200 import api, _lib
     from block_sparse_attention_logits_b200 import build as bsa_build
 
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    init_dist(world)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     bsa_build.build()
@@ -305,12 +325,9 @@ def run_ours(args, w, world, rank, local):
     elapsed_ms = start.elapsed_time(stop)
     attn_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(K)]
     sel_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     ms_step = elapsed_ms / K
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = job_value(flops, ms_step, world)
 
     # e2e: host buffers in, result out, through the same API calls.  Heads are
     # independent, so the step runs over head chunks on three streams: the
@@ -388,17 +405,13 @@ def run_ours(args, w, world, rank, local):
             e2e_step()
         e2.record()
         barrier()
-        e_ms = s2.elapsed_time(e2)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(s2.elapsed_time(e2), world, dev)
         # the pipelined step must give the one-stream step's result
         o_ref, _ = step(q, k, v)
         torch.cuda.synchronize()
         if not torch.equal(o_ref.cpu(), o_host):
             raise RuntimeError("pipelined end-to-end step disagrees with the one-stream step")
-        e2e = {"value": round(flops * world / (e_ms / Ke * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        e2e = {"value": round(job_value(flops, e_ms / Ke, world), 3), "unit": "TFLOP/s",
                "ms_per_step": round(e_ms / Ke, 3), "steps": Ke,
                "pipeline": f"{n_chunks} head chunks on 3 streams (copy-in, compute, copy-out)",
                "h2d_bytes_per_step": 3 * B * H * L * D * 2, "d2h_bytes_per_step": B * H * L * D * 2 + B * H * L * 4}
