@@ -41,7 +41,7 @@ from block_sparse_attention_logits_b200.synthetic import make_qkv, random_bf16  
 
 METRIC = "block-sparse attn ms/call & TFLOP/s on kept blocks vs bf16 TC peak at 90% sparsity"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 8  # 3 gathers, pooling, block softmax, selection, attention, scatter
+LAUNCHES_PER_STEP = 7  # 3 gathers, pooling, block softmax, selection, attention (writes O in grid order)
 E2E_MAX_CHUNKS = 8     # head chunks of the pipelined end-to-end step
 
 
@@ -287,13 +287,15 @@ def run_ours(args, w, world, rank, local):
         api.select_topp_mask(b["probs"], p, L, blk, D, b["mask"], b["idx"], b["cnt"])
         if events:
             events[1].record()
-        api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h, alpha, b["oh"], b["lse"], status=status)
+        if w.hilbert:
+            # the epilogue writes O and LSE back in grid order
+            api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h, alpha, b["o"], b["lse"], status=status,
+                                out_rows=perm)
+        else:
+            api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h, alpha, b["oh"], b["lse"], status=status)
         if events:
             events[2].record()
-        if w.hilbert:
-            api.permute_tokens(b["oh"], perm, inverse=True, out=b["o"])
-            return b["o"], b["lse"]
-        return b["oh"], b["lse"]
+        return (b["o"] if w.hilbert else b["oh"]), b["lse"]
 
     def barrier():
         if world > 1:
@@ -366,11 +368,12 @@ def run_ours(args, w, world, rank, local):
                 qs, ks, vs = qi, ki, vi
             api.score_blocks(qs, ks, blk, b["qp"], b["kp"], b["probs"])
             api.select_topp_mask(b["probs"], p, L, blk, D, b["mask"], b["idx"], b["cnt"])
+            if w.hilbert:
+                api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h[:, hs], alpha[hs], b["o"], b["lse"],
+                                    status=status, out_rows=perm)
+                return b["o"], b["lse"]
             api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h[:, hs], alpha[hs], b["oh"], b["lse"],
                                 status=status)
-            if w.hilbert:
-                api.permute_tokens(b["oh"], perm, inverse=True, out=b["o"])
-                return b["o"], b["lse"]
             return b["oh"], b["lse"]
 
         def e2e_step():
@@ -488,7 +491,7 @@ def run_ours(args, w, world, rank, local):
         "stages_ms": {"score_and_select": round(float(np.mean(sel_ms)), 4), "attention": round(attn_avg_ms, 4),
                       "gather_scatter_and_rest": round(ms_step - attn_avg_ms - float(np.mean(sel_ms)), 4)},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "refresh": refresh,
-        "gpu_launches": LAUNCHES_PER_STEP * K if w.hilbert else (LAUNCHES_PER_STEP - 4) * K,
+        "gpu_launches": LAUNCHES_PER_STEP * K if w.hilbert else (LAUNCHES_PER_STEP - 3) * K,
         "clocks": clk,
     }
     if world > 1:

@@ -14,7 +14,7 @@ EXPORTS = (
     "bsa_strerror", "bsa_version", "bsa_score_blocks", "bsa_score_blocks_restricted", "bsa_block_drift",
     "bsa_select_topp_mask", "bsa_select_topp_mask_restricted",
     "bsa_reorder_workspace_bytes", "bsa_reorder_tokens", "bsa_reorder_tokens_noalloc", "bsa_permute_tokens",
-    "bsa_sparse_attn_fwd", "bsa_sparse_attn_refresh", "bsa_refresh_refinement", "bsa_apply_correction",
+    "bsa_sparse_attn_fwd", "bsa_sparse_attn_fwd_scatter", "bsa_sparse_attn_refresh", "bsa_refresh_refinement", "bsa_apply_correction",
 )
 
 BSA_OK, BSA_EINVAL, BSA_ESHAPE, BSA_ENODEV, BSA_ECUDA, BSA_EWORKSPACE = range(6)
@@ -62,6 +62,7 @@ def load():
         "bsa_reorder_tokens_noalloc": (_I, [_I, _I, _I, _P, _P, _P]),
         "bsa_permute_tokens": (_I, [Shape, _P, _P, _P, _I, _P]),
         "bsa_sparse_attn_fwd": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "bsa_sparse_attn_fwd_scatter": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_sparse_attn_refresh": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_refresh_refinement": (_I, [Shape, _P, _P, _P, _P]),
         "bsa_apply_correction": (_I, [Shape, _P, _P, _P, _P, _P]),

@@ -164,12 +164,13 @@ def permute_tokens(x, perm, inverse=False, out=None):
 
 
 def sparse_attn_fwd(q, k, v, blk, kept_idx=None, kept_cnt=None, R=None, alpha=None,
-                    o=None, lse=None, status=None):
+                    o=None, lse=None, status=None, out_rows=None):
     """Block-sparse attention over the kept blocks (dense when kept_* are None).
 
     Returns (o bf16 [B,H,L,D], lse float32 [B,H,L]).  With R / alpha the
     epilogue adds alpha_h * R.  `status` (int32 [1] on the device, zeroed by
-    the caller) receives BSA_DEV_* bits.
+    the caller) receives BSA_DEV_* bits.  With `out_rows` (int32 [L], a
+    permutation; blk 128) output row r goes to row out_rows[r] of o and lse.
     """
     B, H, L, D = q.shape
     nb = n_blocks(L, blk)
@@ -185,9 +186,15 @@ def sparse_attn_fwd(q, k, v, blk, kept_idx=None, kept_cnt=None, R=None, alpha=No
     lse = lse if lse is not None else torch.empty((B, H, L), dtype=torch.float32, device=q.device)
     _need(o, torch.bfloat16, (B, H, L, D), "o")
     _need(lse, torch.float32, (B, H, L), "lse")
-    check("bsa_sparse_attn_fwd", _lib.load().bsa_sparse_attn_fwd(
-        Shape(B, H, L, D, blk), _ptr(q), _ptr(k), _ptr(v), _ptr(kept_idx), _ptr(kept_cnt),
-        _ptr(R), _ptr(alpha), _ptr(o), _ptr(lse), _ptr(status), _stream()))
+    if out_rows is None:
+        check("bsa_sparse_attn_fwd", _lib.load().bsa_sparse_attn_fwd(
+            Shape(B, H, L, D, blk), _ptr(q), _ptr(k), _ptr(v), _ptr(kept_idx), _ptr(kept_cnt),
+            _ptr(R), _ptr(alpha), _ptr(o), _ptr(lse), _ptr(status), _stream()))
+    else:
+        _need(out_rows, torch.int32, (L,), "out_rows")
+        check("bsa_sparse_attn_fwd_scatter", _lib.load().bsa_sparse_attn_fwd_scatter(
+            Shape(B, H, L, D, blk), _ptr(q), _ptr(k), _ptr(v), _ptr(kept_idx), _ptr(kept_cnt),
+            _ptr(R), _ptr(alpha), _ptr(out_rows), _ptr(o), _ptr(lse), _ptr(status), _stream()))
     return o, lse
 
 

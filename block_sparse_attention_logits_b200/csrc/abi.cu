@@ -160,16 +160,30 @@ int bsa_permute_tokens(bsa_shape s, const bsa_bf16* x, const int32_t* perm, bsa_
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int bsa_sparse_attn_fwd_scatter(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
+                                const int32_t* kept_idx, const int32_t* kept_cnt, const bsa_bf16* R,
+                                const float* alpha, const int32_t* out_rows, bsa_bf16* o, float* lse,
+                                int32_t* status, bsa_stream stream);
+
 int bsa_sparse_attn_fwd(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v, const int32_t* kept_idx,
                         const int32_t* kept_cnt, const bsa_bf16* R, const float* alpha, bsa_bf16* o, float* lse,
                         int32_t* status, bsa_stream stream) {
+  return bsa_sparse_attn_fwd_scatter(s, q, k, v, kept_idx, kept_cnt, R, alpha, nullptr, o, lse, status, stream);
+}
+
+int bsa_sparse_attn_fwd_scatter(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
+                                const int32_t* kept_idx, const int32_t* kept_cnt, const bsa_bf16* R,
+                                const float* alpha, const int32_t* out_rows, bsa_bf16* o, float* lse,
+                                int32_t* status, bsa_stream stream) {
   if (!q || !k || !v || !o || !lse) return BSA_EINVAL;
   if ((kept_idx == nullptr) != (kept_cnt == nullptr)) return BSA_EINVAL;
   if ((R == nullptr) != (alpha == nullptr)) return BSA_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return BSA_EINVAL;
   if ((kept_idx && !aligned16(kept_idx)) || (kept_cnt && !aligned16(kept_cnt)) || (R && !aligned16(R)))
     return BSA_EINVAL;
+  if (out_rows && !aligned16(out_rows)) return BSA_EINVAL;
   if (int r = check_block_shape(s)) return r;
+  if (out_rows && s.blk != 128) return BSA_ESHAPE;
   if (int r = check_device()) return r;
   bsa::AttnArgs a;
   a.q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -182,6 +196,7 @@ int bsa_sparse_attn_fwd(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const
   a.o = reinterpret_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.status = status;
+  a.out_rows = out_rows;
   return bsa::launch_sparse_attn(s, a, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -111,6 +111,7 @@ struct Params {
   float* lse2;           //                sparse LSE
   __nv_bfloat16* r_out;  //                refinement (nullable)
   float* mass;           //                kept attention share (nullable)
+  const int32_t* out_rows;  // output row map (nullable = identity)
   int32_t* status;
   int H, L, NB, NT, n_work;
   float scale_log2;
@@ -679,9 +680,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float l = st[r];
       const float m_ref = st[BM + r];
       const int grow = it.qb * BM + r;
-      const bool store = grow < L;
+      // output row: the row map (fused correction path only), checked
+      int orow = grow;
+      if (!kFused && prm.out_rows && grow < L) {
+        orow = __ldg(prm.out_rows + grow);
+        if (static_cast<unsigned>(orow) >= static_cast<unsigned>(L)) {
+          flag_status(prm, BSA_DEV_BAD_INDEX);
+          orow = -1;
+        }
+      }
+      const bool store = grow < L && orow >= 0;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const size_t row_elem = (static_cast<size_t>(it.bh) * L + (store ? grow : 0)) * D;
+      const size_t out_elem = (static_cast<size_t>(it.bh) * L + (store ? orow : 0)) * D;
       const uint32_t tO = tmem + lane_off + C::COL_O + ob * D;
       if constexpr (kFused) {
         // dense = (OK + OR) / l, sparse = OK / l_kept.  OK holds data only if
@@ -772,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
-            uint4* op = reinterpret_cast<uint4*>(prm.o + row_elem + cc * 32);
+            uint4* op = reinterpret_cast<uint4*>(prm.o + out_elem + cc * 32);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               uint4 ov;
@@ -785,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (store)
-          prm.lse[static_cast<size_t>(it.bh) * L + grow] =
+          prm.lse[static_cast<size_t>(it.bh) * L + orow] =
               l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
         tc_fence_before();
         mbar_arrive(&sh->o_empty[ob]);
@@ -879,6 +890,7 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   prm.lse2 = a.lse2;
   prm.r_out = a.r_out;
   prm.mass = a.mass;
+  prm.out_rows = a.out_rows;
   prm.status = a.status;
   prm.H = s.H;
   prm.L = s.L;

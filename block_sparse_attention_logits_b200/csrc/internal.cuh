@@ -57,6 +57,9 @@ struct AttnArgs {
   float* lse2 = nullptr;
   __nv_bfloat16* r_out = nullptr;  // nullable
   float* mass = nullptr;           // nullable
+  // blk = 128, not the fused refresh: output row r of (b, h) goes to row
+  // out_rows[r] of o and lse (nullable = identity)
+  const int32_t* out_rows = nullptr;
 };
 // Returns BSA_OK / BSA_ECUDA (tensor-map encoding or launch failure).
 // blk = 128: persistent one-tile-per-step kernel (attention_tile.cu);

@@ -236,6 +236,23 @@ BSA_API int bsa_sparse_attn_fwd(bsa_shape s, const bsa_bf16* q, const bsa_bf16* 
                         const float* alpha, bsa_bf16* o, float* lse, int32_t* status, bsa_stream stream);
 
 /*
+ * bsa_sparse_attn_fwd_scatter -- bsa_sparse_attn_fwd that writes each output
+ * row through a row map, so that attention on Hilbert-ordered tokens returns
+ * O and LSE in grid order without a separate scatter (DFSAttn abstract: the
+ * tokens are reordered along a Hilbert curve for the attention only).
+ * Same computation and arguments as bsa_sparse_attn_fwd, plus out_rows: device
+ * int32 [L]; output row r of every (b, h) goes to row out_rows[r] of o and lse
+ * (the `perm` of bsa_reorder_tokens undoes the curve order).  R is read in the
+ * order of q/k/v.  out_rows must be a permutation of [0, L); a row whose
+ * target is out of range is skipped and flagged (BSA_DEV_BAD_INDEX).
+ * s.blk must be 128 (BSA_ESHAPE otherwise).
+ */
+BSA_API int bsa_sparse_attn_fwd_scatter(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
+                                const int32_t* kept_idx, const int32_t* kept_cnt, const bsa_bf16* R,
+                                const float* alpha, const int32_t* out_rows, bsa_bf16* o, float* lse,
+                                int32_t* status, bsa_stream stream);
+
+/*
  * bsa_refresh_refinement -- renew the cached refinement at a dense refresh.
  * Defines: the refinement cached at a dense refresh and renewed only there
  * (RECAP, sections 1, 3.4 and 4.3).

@@ -146,6 +146,16 @@ def test_refresh_validation(lib):
                                        NULL) == _lib.BSA_ESHAPE
 
 
+def test_scatter_validation(lib):
+    args = [FAKE] * 3
+    ok = (NULL, NULL, NULL, NULL)  # kept_idx, kept_cnt, R, alpha
+    # the row map needs 128-token blocks and 16-byte alignment
+    assert lib.bsa_sparse_attn_fwd_scatter(Shape(1, 2, 1000, 128, 64), *args, *ok, FAKE, FAKE, FAKE, NULL,
+                                           NULL) == _lib.BSA_ESHAPE
+    assert lib.bsa_sparse_attn_fwd_scatter(Shape(1, 2, 1000, 128, 128), *args, *ok,
+                                           ctypes.c_void_p(FAKE.value + 4), FAKE, FAKE, NULL, NULL) == _lib.BSA_EINVAL
+
+
 def test_elementwise_validation(lib):
     assert lib.bsa_refresh_refinement(Shape(1, 1, 10, 12, 0), FAKE, FAKE, FAKE, NULL) == _lib.BSA_ESHAPE
     assert lib.bsa_refresh_refinement(Shape(1, 1, 10, 16, 0), FAKE, NULL, FAKE, NULL) == _lib.BSA_EINVAL

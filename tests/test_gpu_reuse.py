@@ -2,7 +2,7 @@
 query-key drift of the block means, scoring restricted to candidate blocks
 and the restricted top-p selection (bit-exact given the same float32 scores),
 with rows that have no candidates, candidates of zero mass, p = 1 heads and
-ties."""
+ties.  Also the attention call that writes its output through a row map."""
 
 import numpy as np
 import pytest
@@ -92,3 +92,42 @@ def test_restricted_selection_bit_exact(seed):
                 assert np.array_equal(ig[b, h, r, :cg[b, h, r]], io[b, h, r, :co[b, h, r]])
     assert cg[0, 0, 2] == 0
     assert np.all((to_np(m) == 1) <= (cand == 1))
+
+
+def test_scatter_output_equals_attention_then_inverse_permute():
+    """bsa_sparse_attn_fwd_scatter writes the same numbers as attention in curve
+    order followed by the inverse permutation (both are this library's kernels;
+    the curve-order attention itself is checked against the oracle elsewhere)."""
+    from block_sparse_attention_logits_b200._lib import BSA_DEV_BAD_INDEX
+    grid = (3, 9, 16)
+    B, H, D, blk = 1, 2, 128, 128
+    L = grid[0] * grid[1] * grid[2]
+    NB = (L + blk - 1) // blk
+    q, k, v = (random_bf16((B, H, L, D), 70 + j).to(DEV) for j in range(3))
+    R = random_bf16((B, H, L, D), 73, scale=0.05).to(DEV)
+    alpha = torch.tensor([0.3, 0.8], dtype=torch.float32, device=DEV)
+    perm, _ = api.reorder_tokens(*grid, device=DEV)
+    qh, kh, vh = (api.permute_tokens(x, perm) for x in (q, k, v))
+    Rh = api.permute_tokens(R, perm)
+    _, _, P = api.score_blocks(qh, kh, blk)
+    _, idx, cnt = api.select_topp_mask(P, 0.9, L, blk, D)
+    oh, lh = api.sparse_attn_fwd(qh, kh, vh, blk, idx, cnt, Rh, alpha)
+    o_ref = api.permute_tokens(oh, perm, inverse=True)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, lse = api.sparse_attn_fwd(qh, kh, vh, blk, idx, cnt, Rh, alpha, status=status, out_rows=perm)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(o, o_ref)
+    lse_ref = torch.empty_like(lh)
+    lse_ref[:, :, perm.long()] = lh
+    assert torch.equal(lse, lse_ref)
+    # an out-of-range row target is skipped and flagged
+    bad = perm.clone()
+    bad[5] = L + 3
+    o2 = torch.zeros_like(o)
+    api.sparse_attn_fwd(qh, kh, vh, blk, idx, cnt, Rh, alpha, o=o2, status=status, out_rows=bad)
+    torch.cuda.synchronize()
+    assert status.item() & BSA_DEV_BAD_INDEX
+    keep = torch.ones(L, dtype=torch.bool, device=DEV)
+    keep[perm[5].long()] = False
+    assert torch.equal(o2[:, :, keep], o[:, :, keep])
