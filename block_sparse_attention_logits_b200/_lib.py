@@ -11,7 +11,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbsa.so")
 
 EXPORTS = (
-    "bsa_strerror", "bsa_version", "bsa_score_blocks", "bsa_score_blocks_restricted", "bsa_block_drift",
+    "bsa_strerror", "bsa_version", "bsa_score_blocks", "bsa_score_blocks_gather", "bsa_score_blocks_restricted",
+    "bsa_block_drift",
     "bsa_select_topp_mask", "bsa_select_topp_mask_restricted",
     "bsa_reorder_workspace_bytes", "bsa_reorder_tokens", "bsa_reorder_tokens_noalloc", "bsa_permute_tokens",
     "bsa_sparse_attn_fwd", "bsa_sparse_attn_fwd_scatter", "bsa_sparse_attn_refresh", "bsa_refresh_refinement", "bsa_apply_correction",
@@ -53,6 +54,7 @@ def load():
         "bsa_strerror": (ctypes.c_char_p, [_I]),
         "bsa_version": (_I, []),
         "bsa_score_blocks": (_I, [Shape, _P, _P, _P, _P, _P, _P]),
+        "bsa_score_blocks_gather": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_score_blocks_restricted": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_block_drift": (_I, [Shape, _P, _P, _P, _P, _P, _P]),
         "bsa_select_topp_mask": (_I, [Shape, _P, ctypes.POINTER(ctypes.c_float), _P, _P, _P, _P]),

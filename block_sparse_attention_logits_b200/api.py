@@ -84,6 +84,31 @@ def score_blocks(q, k, blk, q_pool=None, k_pool=None, probs=None, candidates=Non
     return q_pool, k_pool, probs
 
 
+def score_blocks_gather(q, k, perm, blk, q_out=None, k_out=None, q_pool=None, k_pool=None, probs=None):
+    """permute_tokens(q), permute_tokens(k) and score_blocks of the results in
+    one pass.  Returns (q_out, k_out, q_pool, k_pool, probs)."""
+    B, H, L, D = q.shape
+    nb = n_blocks(L, blk)
+    _need(q, torch.bfloat16, (B, H, L, D), "q")
+    _need(k, torch.bfloat16, (B, H, L, D), "k")
+    _need(perm, torch.int32, (L,), "perm")
+    dev = q.device
+    q_out = q_out if q_out is not None else torch.empty_like(q)
+    k_out = k_out if k_out is not None else torch.empty_like(k)
+    q_pool = q_pool if q_pool is not None else torch.empty((B, H, nb, D), dtype=torch.float32, device=dev)
+    k_pool = k_pool if k_pool is not None else torch.empty((B, H, nb, D), dtype=torch.float32, device=dev)
+    probs = probs if probs is not None else torch.empty((B, H, nb, nb), dtype=torch.float32, device=dev)
+    for name, t in (("q_out", q_out), ("k_out", k_out)):
+        _need(t, torch.bfloat16, (B, H, L, D), name)
+    _need(q_pool, torch.float32, (B, H, nb, D), "q_pool")
+    _need(k_pool, torch.float32, (B, H, nb, D), "k_pool")
+    _need(probs, torch.float32, (B, H, nb, nb), "probs")
+    check("bsa_score_blocks_gather", _lib.load().bsa_score_blocks_gather(
+        _shape(q, blk), _ptr(q), _ptr(k), _ptr(perm), _ptr(q_out), _ptr(k_out), _ptr(q_pool), _ptr(k_pool),
+        _ptr(probs), _stream()))
+    return q_out, k_out, q_pool, k_pool, probs
+
+
 def block_drift(q_pool_ref, k_pool_ref, q_pool, k_pool, L, blk, drift=None):
     """Per-head query-key drift of the block means since a reference step:
     max of the relative Frobenius changes of the Q and K means.  Inputs

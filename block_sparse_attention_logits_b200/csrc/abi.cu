@@ -91,6 +91,23 @@ int bsa_score_blocks_restricted(bsa_shape s, const bsa_bf16* q, const bsa_bf16* 
   return from_cuda(bsa::launch_block_softmax(s, q_pool, k_pool, probs, candidates, st));
 }
 
+int bsa_score_blocks_gather(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const int32_t* perm, bsa_bf16* q_out,
+                            bsa_bf16* k_out, float* q_pool, float* k_pool, float* probs, bsa_stream stream) {
+  if (!q || !k || !perm || !q_out || !k_out || !q_pool || !k_pool || !probs) return BSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(perm) || !aligned16(q_out) || !aligned16(k_out) ||
+      !aligned16(q_pool) || !aligned16(k_pool) || !aligned16(probs))
+    return BSA_EINVAL;
+  if (q_out == q || q_out == k || k_out == q || k_out == k || q_out == k_out) return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (int r = check_device()) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaError_t e = bsa::launch_pool(s, reinterpret_cast<const __nv_bfloat16*>(q),
+                                       reinterpret_cast<const __nv_bfloat16*>(k), q_pool, k_pool, st, perm,
+                                       reinterpret_cast<__nv_bfloat16*>(q_out), reinterpret_cast<__nv_bfloat16*>(k_out)))
+    return from_cuda(e);
+  return from_cuda(bsa::launch_block_softmax(s, q_pool, k_pool, probs, nullptr, st));
+}
+
 int bsa_block_drift(bsa_shape s, const float* q_pool_ref, const float* k_pool_ref, const float* q_pool,
                     const float* k_pool, float* drift, bsa_stream stream) {
   if (!q_pool_ref || !k_pool_ref || !q_pool || !k_pool || !drift) return BSA_EINVAL;

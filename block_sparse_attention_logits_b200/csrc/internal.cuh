@@ -20,8 +20,11 @@ struct TopP {
 inline int n_blocks(int L, int blk) { return (L + blk - 1) / blk; }
 
 // launchers (return cudaSuccess or the launch error)
+// perm (nullable): gather form -- token t is input row perm[t]; the gathered
+// rows are also written to q_out / k_out
 cudaError_t launch_pool(const bsa_shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, float* qp, float* kp,
-                        cudaStream_t st);
+                        cudaStream_t st, const int32_t* perm = nullptr, __nv_bfloat16* q_out = nullptr,
+                        __nv_bfloat16* k_out = nullptr);
 // cand: optional uint8 [B,H,NB,NB]; non-null restricts each row's softmax and
 // top-p search to its candidate blocks (the others get P = 0 / are never kept)
 cudaError_t launch_block_softmax(const bsa_shape& s, const float* qp, const float* kp, float* probs,

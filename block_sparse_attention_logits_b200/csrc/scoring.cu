@@ -26,10 +26,14 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& v) {
   }
 }
 
+// With `perm` (gathering form) token t of the block is row perm[t] of the
+// input, and the gathered rows are also written to q_out / k_out in order.
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k, float* __restrict__ qp,
-                                                   float* __restrict__ kp, int L, int blk, int NB) {
+                                                   float* __restrict__ kp, int L, int blk, int NB,
+                                                   const int32_t* __restrict__ perm, __nv_bfloat16* __restrict__ q_out,
+                                                   __nv_bfloat16* __restrict__ k_out) {
   constexpr int TPR = D / 8;        // threads per token row (8 bf16 each)
   constexpr int RPI = 256 / TPR;    // rows in flight per iteration
   __shared__ float part[RPI][D + 1];
@@ -41,10 +45,21 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   const int n = min(blk, L - t0);
   const int c = threadIdx.x % TPR;
   const int r = threadIdx.x / TPR;
-  const uint4* base = reinterpret_cast<const uint4*>(x + (bh * L + t0) * D) + c;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (perm) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + bh * L * D) + c;
+    uint4* dst = reinterpret_cast<uint4*>((blockIdx.z ? k_out : q_out) + (bh * L + t0) * D) + c;
 #pragma unroll 4
-  for (int row = r; row < n; row += RPI) add_bf16x8(acc, __ldg(base + static_cast<size_t>(row) * TPR));
+    for (int row = r; row < n; row += RPI) {
+      const uint4 v = __ldg(src + static_cast<size_t>(__ldg(perm + t0 + row)) * TPR);
+      dst[static_cast<size_t>(row) * TPR] = v;
+      add_bf16x8(acc, v);
+    }
+  } else {
+    const uint4* base = reinterpret_cast<const uint4*>(x + (bh * L + t0) * D) + c;
+#pragma unroll 4
+    for (int row = r; row < n; row += RPI) add_bf16x8(acc, __ldg(base + static_cast<size_t>(row) * TPR));
+  }
 #pragma unroll
   for (int e = 0; e < 8; ++e) part[r][c * 8 + e] = acc[e];
   __syncthreads();
@@ -185,13 +200,13 @@ __global__ void __launch_bounds__(256) drift_kernel(const float* __restrict__ qr
 }  // namespace
 
 cudaError_t launch_pool(const bsa_shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, float* qp, float* kp,
-                        cudaStream_t st) {
+                        cudaStream_t st, const int32_t* perm, __nv_bfloat16* q_out, __nv_bfloat16* k_out) {
   const int NB = n_blocks(s.L, s.blk);
   dim3 grid(NB, s.B * s.H, 2);
   if (s.D == 128)
-    pool_kernel<128><<<grid, 256, 0, st>>>(q, k, qp, kp, s.L, s.blk, NB);
+    pool_kernel<128><<<grid, 256, 0, st>>>(q, k, qp, kp, s.L, s.blk, NB, perm, q_out, k_out);
   else
-    pool_kernel<64><<<grid, 256, 0, st>>>(q, k, qp, kp, s.L, s.blk, NB);
+    pool_kernel<64><<<grid, 256, 0, st>>>(q, k, qp, kp, s.L, s.blk, NB, perm, q_out, k_out);
   return cudaGetLastError();
 }
 

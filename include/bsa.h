@@ -164,6 +164,20 @@ BSA_API int bsa_permute_tokens(bsa_shape s, const bsa_bf16* x, const int32_t* pe
                        bsa_stream stream);
 
 /*
+ * bsa_score_blocks_gather -- the token reorder of q and k fused with scoring.
+ * Same as bsa_permute_tokens(q -> q_out), bsa_permute_tokens(k -> k_out)
+ * (inverse = 0, q_out[b,h,t,:] = q[b,h,perm[t],:]) followed by
+ * bsa_score_blocks(q_out, k_out), in one pass that reads q and k once.
+ * perm: device int32 [L], a permutation of [0, L) (e.g. from
+ * bsa_reorder_tokens; not checked on the device).  q_out, k_out: bf16
+ * [B,H,L,D], not overlapping q, k or each other.  Outputs and errors as
+ * bsa_score_blocks and bsa_permute_tokens.
+ */
+BSA_API int bsa_score_blocks_gather(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const int32_t* perm,
+                            bsa_bf16* q_out, bsa_bf16* k_out, float* q_pool, float* k_pool, float* probs,
+                            bsa_stream stream);
+
+/*
  * bsa_block_drift -- query-key drift of each head since a reference step.
  * Defines: Temporal Mask Reuse skips mask prediction based on query-key drift
  * (head-wise adaptive top-p abstract).  From the block means that

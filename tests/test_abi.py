@@ -156,6 +156,17 @@ def test_scatter_validation(lib):
                                            ctypes.c_void_p(FAKE.value + 4), FAKE, FAKE, NULL, NULL) == _lib.BSA_EINVAL
 
 
+def test_gather_scoring_validation(lib):
+    s = Shape(1, 2, 1000, 128, 128)
+    other = ctypes.c_void_p(2 << 20)
+    third = ctypes.c_void_p(3 << 20)
+    # perm required; outputs may not alias the inputs or each other
+    assert lib.bsa_score_blocks_gather(s, FAKE, other, NULL, third, ctypes.c_void_p(4 << 20), FAKE, FAKE, FAKE,
+                                       NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_score_blocks_gather(s, FAKE, other, FAKE, FAKE, third, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_score_blocks_gather(s, FAKE, other, FAKE, third, third, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+
+
 def test_elementwise_validation(lib):
     assert lib.bsa_refresh_refinement(Shape(1, 1, 10, 12, 0), FAKE, FAKE, FAKE, NULL) == _lib.BSA_ESHAPE
     assert lib.bsa_refresh_refinement(Shape(1, 1, 10, 16, 0), FAKE, NULL, FAKE, NULL) == _lib.BSA_EINVAL

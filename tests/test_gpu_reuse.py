@@ -131,3 +131,20 @@ def test_scatter_output_equals_attention_then_inverse_permute():
     keep = torch.ones(L, dtype=torch.bool, device=DEV)
     keep[perm[5].long()] = False
     assert torch.equal(o2[:, :, keep], o[:, :, keep])
+
+
+def test_score_blocks_gather_equals_permute_then_score():
+    """The gathering scorer gives the same bits as the two permutes followed by
+    bsa_score_blocks (both this library's kernels; scoring itself is checked
+    against the oracle elsewhere)."""
+    grid = (3, 9, 16)
+    B, H, D, blk = 1, 3, 128, 128
+    L = grid[0] * grid[1] * grid[2]
+    q, k = (random_bf16((B, H, L, D), 80 + j).to(DEV) for j in range(2))
+    perm, _ = api.reorder_tokens(*grid, device=DEV)
+    qh, kh = api.permute_tokens(q, perm), api.permute_tokens(k, perm)
+    qp, kp, P = api.score_blocks(qh, kh, blk)
+    q2, k2, qp2, kp2, P2 = api.score_blocks_gather(q, k, perm, blk)
+    torch.cuda.synchronize()
+    for a, b in ((qh, q2), (kh, k2), (qp, qp2), (kp, kp2), (P, P2)):
+        assert torch.equal(a, b)
