@@ -56,7 +56,7 @@ def parse_args():
     ap.add_argument("--heads", type=int, default=0,
                     help="run only the first N heads of the workload (small profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-refresh", action="store_true", help="skip the dense-refresh timing")
+    ap.add_argument("--no-refresh", action="store_true", help="skip the dense-refresh and mask-reuse timings")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()
 
@@ -455,6 +455,40 @@ def run_ours(args, w, world, rank, local):
                    "calls": "fused: bsa_sparse_attn_refresh; two-pass: dense + sparse bsa_sparse_attn_fwd + "
                             "bsa_refresh_refinement"}
 
+    # mask reuse on the same inputs: drift of the block means against a
+    # reference step, and scoring / selection restricted to the current mask
+    reuse = None
+    if not args.no_refresh:
+        qp_ref = bufs["qp"] * 1.01
+        kp_ref = bufs["kp"].clone()
+        cand = bufs["mask"].clone()
+        rprobs, rmask = torch.empty_like(bufs["probs"]), torch.empty_like(bufs["mask"])
+        ridx, rcnt = torch.empty_like(bufs["idx"]), torch.empty_like(bufs["cnt"])
+        qs_, ks_ = (bufs["qh"], bufs["kh"]) if w.hilbert else (q, k)
+
+        def drift():
+            api.block_drift(qp_ref, kp_ref, bufs["qp"], bufs["kp"], L, blk)
+
+        def restricted():
+            api.score_blocks(qs_, ks_, blk, bufs["qp"], bufs["kp"], rprobs, candidates=cand)
+            api.select_topp_mask(rprobs, p, L, blk, D, rmask, ridx, rcnt, candidates=cand)
+
+        rt = {}
+        for name, fn in (("drift", drift), ("restricted_score_select", restricted)):
+            fn()
+            barrier()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record()
+            for _ in range(5):
+                fn()
+            a1.record()
+            barrier()
+            rt[name] = round(a0.elapsed_time(a1) / 5, 4)
+        reuse = {"drift_ms": rt["drift"], "restricted_score_select_ms": rt["restricted_score_select"],
+                 "candidates": "the step's own mask",
+                 "kept_fraction_of_candidates": round(rcnt.double().sum().item() / max(cand.double().sum().item(), 1),
+                                                      4)}
+
     if status.item() != 0:
         raise RuntimeError(f"attention kernel reported status {status.item()}")
 
@@ -489,7 +523,7 @@ def run_ours(args, w, world, rank, local):
                  "dense_equiv_tflops": round(4.0 * B * H * L * L * D / (attn_avg_ms * 1e-3) / 1e12, 2)},
         "stages_ms": {"gather_score_and_select": round(float(np.mean(sel_ms)), 4), "attention": round(attn_avg_ms, 4),
                       "rest": round(ms_step - attn_avg_ms - float(np.mean(sel_ms)), 4)},
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "refresh": refresh,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "refresh": refresh, "reuse": reuse,
         "gpu_launches": LAUNCHES_PER_STEP * K if w.hilbert else (LAUNCHES_PER_STEP - 1) * K,
         "clocks": clk,
     }
