@@ -56,7 +56,8 @@ def parse_args():
     ap.add_argument("--heads", type=int, default=0,
                     help="run only the first N heads of the workload (small profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-refresh", action="store_true", help="skip the dense-refresh and mask-reuse timings")
+    ap.add_argument("--no-refresh", action="store_true",
+                    help="skip the dense-refresh, mask-reuse, elementwise and sweep timings")
     ap.add_argument("--no-cpu", action="store_true")
     return ap.parse_args()
 
@@ -489,6 +490,74 @@ def run_ours(args, w, world, rank, local):
                  "kept_fraction_of_candidates": round(rcnt.double().sum().item() / max(cand.double().sum().item(), 1),
                                                       4)}
 
+    # the elementwise calls (refinement at a refresh, standalone correction):
+    # HBM-bound, three [B,H,L,D] bf16 streams each
+    elementwise = None
+    sweep = None
+    if not args.no_refresh and blk == 128:
+        peaks_e, _ = load_peaks()
+        oa, ob_, oc = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        ew = {}
+        for name, fn in (("refresh_refinement", lambda: api.refresh_refinement(bufs["oh"], q, out=oa)),
+                         ("apply_correction", lambda: api.apply_correction(bufs["oh"], R_h, alpha, out=ob_))):
+            fn()
+            barrier()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record()
+            for _ in range(10):
+                fn()
+            a1.record()
+            barrier()
+            ms = a0.elapsed_time(a1) / 10
+            gbs = 3 * B * H * L * D * 2 / (ms * 1e-3) / 1e9
+            ew[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peaks_e["hbm_gbs"], 3)}
+        elementwise = ew
+        del oa, ob_, oc
+
+        # the mask-reuse sweep on this shape: Q and K drift by N(0, w.drift or
+        # 0.05) per step (drawn on the device, outside the timed region); the
+        # mask is recomputed every 3rd step, a dense refresh renews R every 5th
+        # step, the other steps run sparse attention with the fused alpha*R
+        if w.hilbert:
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(2024)
+            qd_, kd_ = q.clone(), k.clone()
+            sigma = w.drift if w.drift > 0 else 0.05
+            Rs = torch.zeros_like(q)
+            sb = dict(o_dense=torch.empty_like(q), o_sparse=torch.empty_like(q), R=Rs,
+                      lse_dense=torch.empty((B, H, L), dtype=torch.float32, device=dev),
+                      lse_sparse=torch.empty((B, H, L), dtype=torch.float32, device=dev))
+            steps_ms, kinds = [], []
+            for st_ in range(10):
+                if st_ > 0:
+                    for x in (qd_, kd_):
+                        x.copy_((x.float() + sigma * torch.randn(x.shape, generator=gen, device=dev)).to(x.dtype))
+                barrier()
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record()
+                b_ = bufs
+                if st_ % 3 == 0:
+                    api.score_blocks_gather(qd_, kd_, perm, blk, b_["qh"], b_["kh"], b_["qp"], b_["kp"], b_["probs"])
+                    api.select_topp_mask(b_["probs"], p, L, blk, D, b_["mask"], b_["idx"], b_["cnt"])
+                else:
+                    api.permute_tokens(qd_, perm, out=b_["qh"])
+                    api.permute_tokens(kd_, perm, out=b_["kh"])
+                api.permute_tokens(v, perm, out=b_["vh"])
+                if st_ % 5 == 0:
+                    api.sparse_attn_refresh(b_["qh"], b_["kh"], b_["vh"], blk, b_["idx"], b_["cnt"], want_mass=False,
+                                            out=sb, status=status)
+                    api.permute_tokens(sb["o_dense"], perm, inverse=True, out=b_["o"])
+                    kinds.append("refresh")
+                else:
+                    api.sparse_attn_fwd(b_["qh"], b_["kh"], b_["vh"], blk, b_["idx"], b_["cnt"], Rs, alpha, b_["o"],
+                                        b_["lse"], status=status, out_rows=perm)
+                    kinds.append("sparse+mask" if st_ % 3 == 0 else "sparse, mask reused")
+                a1.record()
+                barrier()
+                steps_ms.append(round(a0.elapsed_time(a1), 3))
+            sweep = {"steps_ms": steps_ms, "kinds": kinds, "total_ms": round(float(np.sum(steps_ms)), 3),
+                     "schedule": f"mask every 3rd step, dense refresh every 5th, Q/K drift N(0, {sigma}) per step"}
+
     if status.item() != 0:
         raise RuntimeError(f"attention kernel reported status {status.item()}")
 
@@ -524,6 +593,7 @@ def run_ours(args, w, world, rank, local):
         "stages_ms": {"gather_score_and_select": round(float(np.mean(sel_ms)), 4), "attention": round(attn_avg_ms, 4),
                       "rest": round(ms_step - attn_avg_ms - float(np.mean(sel_ms)), 4)},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "refresh": refresh, "reuse": reuse,
+        "elementwise": elementwise, "sweep": sweep,
         "gpu_launches": LAUNCHES_PER_STEP * K if w.hilbert else (LAUNCHES_PER_STEP - 1) * K,
         "clocks": clk,
     }
