@@ -273,8 +273,10 @@ def run_ours(args, w, world, rank, local):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     ev = None
 
-    def step(qi, ki, vi, events=None):
-        b = bufs
+    def path(b, qi, ki, vi, Ri, ai, events=None):
+        """One pass of the hot path on buffers `b` (the full set or one head
+        chunk): Hilbert gathers, scoring, selection, sparse attention with the
+        fused correction, output in grid order."""
         if events:
             events[0].record()
         if w.hilbert:
@@ -288,15 +290,16 @@ def run_ours(args, w, world, rank, local):
         api.select_topp_mask(b["probs"], p, L, blk, D, b["mask"], b["idx"], b["cnt"])
         if events:
             events[1].record()
-        if w.hilbert:
-            # the epilogue writes O and LSE back in grid order
-            api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h, alpha, b["o"], b["lse"], status=status,
-                                out_rows=perm)
-        else:
-            api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h, alpha, b["oh"], b["lse"], status=status)
+        # with the Hilbert order the epilogue writes O and LSE back in grid order
+        o = b["o"] if w.hilbert else b["oh"]
+        api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], Ri, ai, o, b["lse"], status=status,
+                            out_rows=perm if w.hilbert else None)
         if events:
             events[2].record()
-        return (b["o"] if w.hilbert else b["oh"]), b["lse"]
+        return o, b["lse"]
+
+    def step(qi, ki, vi, events=None):
+        return path(bufs, qi, ki, vi, R_h, alpha, events)
 
     def barrier():
         if world > 1:
@@ -358,23 +361,8 @@ def run_ours(args, w, world, rank, local):
                                    torch.empty_like(t[:, hs])) for n, t in bufs.items()})
 
         def chunk_step(c, qi, ki, vi):
-            b = chunk_bufs[c]
             hs = slice(c * hc, (c + 1) * hc)
-            if w.hilbert:
-                api.score_blocks_gather(qi, ki, perm, blk, b["qh"], b["kh"], b["qp"], b["kp"], b["probs"])
-                api.permute_tokens(vi, perm, out=b["vh"])
-                qs, ks, vs = b["qh"], b["kh"], b["vh"]
-            else:
-                qs, ks, vs = qi, ki, vi
-                api.score_blocks(qs, ks, blk, b["qp"], b["kp"], b["probs"])
-            api.select_topp_mask(b["probs"], p, L, blk, D, b["mask"], b["idx"], b["cnt"])
-            if w.hilbert:
-                api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h[:, hs], alpha[hs], b["o"], b["lse"],
-                                    status=status, out_rows=perm)
-                return b["o"], b["lse"]
-            api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R_h[:, hs], alpha[hs], b["oh"], b["lse"],
-                                status=status)
-            return b["oh"], b["lse"]
+            return path(chunk_bufs[c], qi, ki, vi, R_h[:, hs], alpha[hs])
 
         def e2e_step():
             cur = torch.cuda.current_stream(dev)
