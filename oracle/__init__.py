@@ -21,6 +21,8 @@ Sources (cited by page title and section in every function):
   scoring.
 * CalibAtt (calibrated sparse attention), abstract and Fig. 5 -- threshold the
   top key blocks per query block, skip the unselected blocks.
+* CalibAtt appendix, Fig. S9, Fig. S10 and Table S3 -- skip lists of
+  interval pairs per query block, per-layer trimming, merging outlier rows.
 * the GSRS abstract -- exact attention weights evaluated inside the
   FlashAttention computation (the kept share of the attention mass).
 
@@ -34,9 +36,11 @@ Modules:
                  attention, refinement, exact kept attention mass)
   reuse       -- query-key drift of the block means, and scoring / selection
                  restricted to an earlier candidate set
+  intervals   -- interval (skip-list) encoding of the kept blocks, merging of
+                 outlier rows to a width, the width for a merge percentage
 
 Every function carries a "Pinned by" note naming the tests in
 ``tests/test_oracle.py`` that tie it to something other than itself.
 """
 
-from . import hilbert, scoring, topp, attention, correction, refresh, reuse  # noqa: F401
+from . import hilbert, scoring, topp, attention, correction, refresh, reuse, intervals  # noqa: F401

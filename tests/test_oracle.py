@@ -19,6 +19,7 @@ import torch
 from oracle import attention as oatt
 from oracle import correction as ocor
 from oracle import hilbert as ohil
+from oracle import intervals as oint
 from oracle import refresh as oref
 from oracle import reuse as oreu
 from oracle import scoring as osco
@@ -562,6 +563,121 @@ def test_planted_mistake_restricted_target_is_caught(monkeypatch):
     monkeypatch.setattr(oreu, "select_row_restricted", full_row_target)
     with pytest.raises(AssertionError):
         test_restricted_selection_golden_row_and_edges()
+
+
+# ----------------------------------------------------- interval skip lists
+
+def _as_lists(pairs):
+    return [[int(a), int(b)] for a, b in pairs]
+
+
+def test_intervals_golden_rows_and_widths():
+    cases = json.load(open(os.path.join(GOLDEN, "interval_cases.json")))
+    for row in cases["rows"]:
+        runs = oint.runs_of(row["kept"])
+        assert _as_lists(runs) == row["runs"], row["name"]
+        for W, want in row["merged"].items():
+            assert _as_lists(oint.merge_runs(runs, int(W))) == want, (row["name"], W)
+    for w in cases["widths"]:
+        hist = oint.run_histogram(w["n_runs"], 16)
+        assert oint.width_for_merge(hist, w["q"]) == w["W"], w["why"]
+
+
+def test_intervals_theoretical_maximum():
+    # every other block kept reaches ceil(NB / 2) runs; the 590 full blocks
+    # of N = 75,600 at 128 tokens give the pages' 295 (Fig. S9)
+    for NB in range(1, 40):
+        assert len(oint.runs_of(range(0, NB, 2))) == oint.max_intervals(NB) == math.ceil(NB / 2)
+    assert 75600 // 128 == 590 and oint.max_intervals(590) == 295
+    NB = 9
+    most = max(len(oint.runs_of([j for j in range(NB) if m >> j & 1])) for m in range(1 << NB))
+    assert most == oint.max_intervals(NB)
+
+
+def test_intervals_brute_force_round_trip():
+    NB = 10
+    rows = [[j for j in range(NB) if m >> j & 1] for m in range(1 << NB)]
+    for kept in rows:
+        runs = oint.runs_of(kept)
+        for s, e in runs:
+            assert 0 <= s < e <= NB
+        for (s0, e0), (s1, e1) in zip(runs, runs[1:]):
+            assert s1 - e0 >= 1          # maximal: a skipped block between runs
+        assert oint.decode_row(runs) == kept
+    # the array forms, every subset at once, W = the theoretical maximum
+    W = oint.max_intervals(NB)
+    idx = np.full((len(rows), NB), -1, np.int32)
+    cnt = np.zeros(len(rows), np.int32)
+    for r, kept in enumerate(rows):
+        idx[r, :len(kept)] = kept
+        cnt[r] = len(kept)
+    iv, n_int, n_runs = oint.kept_to_intervals(idx, cnt, W)
+    assert np.array_equal(n_int, n_runs)
+    assert np.all(iv[np.arange(W)[None, :] >= n_int[:, None]] == -1)
+    mask, idx2, cnt2 = oint.intervals_to_kept(iv, n_int, NB)
+    assert np.array_equal(cnt2, cnt) and np.array_equal(idx2, idx)
+    for r, kept in enumerate(rows):
+        assert np.flatnonzero(mask[r]).tolist() == kept
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_merge_is_fewest_added_blocks_then_leftmost(seed):
+    """Brute force over every choice of gaps to fill: the merged row adds the
+    fewest blocks, and among such choices fills the lexicographically
+    smallest set of gaps (the leftmost)."""
+    rng = np.random.default_rng(seed)
+    NB = 24
+    for _ in range(60):
+        kept = np.flatnonzero(rng.random(NB) < rng.uniform(0.2, 0.7)).tolist()
+        runs = oint.runs_of(kept)
+        n = len(runs)
+        gaps = [runs[r + 1][0] - runs[r][1] for r in range(n - 1)]
+        for W in range(1, n):
+            best = min(itertools.combinations(range(n - 1), n - W),
+                       key=lambda c: (sum(gaps[g] for g in c), c))
+            iv = [list(runs[0])]
+            for r in range(n - 1):
+                if r in best:
+                    iv[-1][1] = runs[r + 1][1]
+                else:
+                    iv.append(list(runs[r + 1]))
+            got = oint.merge_runs(runs, W)
+            assert _as_lists(got) == iv
+            dec = oint.decode_row(got)
+            assert set(kept) <= set(dec) and len(dec) - len(kept) == sum(gaps[g] for g in best)
+
+
+def test_width_for_merge_closed_forms():
+    # a rows with x runs and b rows with y > x runs: the width is max(x, 1)
+    # while ceil(q * (a + b)) <= a, else y
+    for a, b, x, y in [(95, 5, 3, 40), (99, 1, 0, 7), (10, 30, 2, 5), (1, 1, 1, 2)]:
+        n_runs = [x] * a + [y] * b
+        hist = oint.run_histogram(n_runs, 2 * y)
+        for q in (0.5, 0.9, 0.95, 0.99, 1.0):
+            want = max(x, 1) if math.ceil(q * (a + b)) <= a else y
+            assert oint.width_for_merge(hist, q) == want, (a, b, x, y, q)
+    assert oint.list_bytes(10, 591) == 10 * 591 * 4 + 40
+    assert oint.interval_bytes(10, 50) == 10 * 50 * 8 + 40
+
+
+def test_planted_mistake_rightmost_gap_first_is_caught(monkeypatch):
+    def rightmost(runs, W):
+        iv = list(runs)
+        while len(iv) > W:
+            gaps = [iv[r + 1][0] - iv[r][1] for r in range(len(iv) - 1)]
+            r = len(gaps) - 1 - gaps[::-1].index(min(gaps))
+            iv[r:r + 2] = [(iv[r][0], iv[r + 1][1])]
+        return iv
+    monkeypatch.setattr(oint, "merge_runs", rightmost)
+    with pytest.raises(AssertionError):
+        test_intervals_golden_rows_and_widths()
+
+
+def test_planted_mistake_inclusive_end_is_caught(monkeypatch):
+    orig = oint.runs_of
+    monkeypatch.setattr(oint, "runs_of", lambda kept: [(s, e - 1) for s, e in orig(kept)])
+    with pytest.raises(AssertionError):
+        test_intervals_golden_rows_and_widths()
 
 
 # ------------------------------------------------- planted mistakes are caught
