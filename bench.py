@@ -237,6 +237,49 @@ def oracle_sample(w, p, seconds, max_blocks=None):
 
 # ------------------------------------------------------------------- ours
 
+def interval_timings(idx, cnt, L, blk, D, barrier, q=0.95):
+    """The interval (skip-list) form of a step's kept lists: per-row runs and
+    their histogram, the width for merge percentage q, encode and decode
+    (decode writes kept lists only); times in ms per call, sizes in bytes."""
+    from block_sparse_attention_logits_b200 import api
+    B, H, nb = cnt.shape
+    dev = cnt.device
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    n_runs = torch.empty_like(cnt)
+    hist = torch.zeros(api.max_intervals(nb) + 1, dtype=torch.int32, device=dev)
+    api.interval_runs(idx, cnt, L, blk, D, n_runs=n_runs, hist=hist, status=st)
+    Wq = api.interval_width_for_merge(hist, q)
+    Wmax = api.interval_width_for_merge(hist, 1.0)
+    iv = torch.empty((B, H, nb, Wq, 2), dtype=torch.int32, device=dev)
+    n_int, nr2 = torch.empty_like(cnt), torch.empty_like(cnt)
+    kidx, kcnt = torch.empty_like(idx), torch.empty_like(cnt)
+    scratch = torch.zeros_like(hist)
+    calls = (("runs", lambda: api.interval_runs(idx, cnt, L, blk, D, n_runs=nr2, hist=scratch, status=st)),
+             ("encode", lambda: api.kept_to_intervals(idx, cnt, Wq, L, blk, D, iv, n_int, nr2, st)),
+             ("decode", lambda: api.intervals_to_kept(iv, n_int, L, blk, D, kept_idx=kidx, kept_cnt=kcnt,
+                                                      want_mask=False, status=st)))
+    ms = {}
+    for name, fn in calls:
+        fn()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(10):
+            fn()
+        a1.record()
+        barrier()
+        ms[name] = round(a0.elapsed_time(a1) / 10, 4)
+    rows = B * H * nb
+    before = cnt.double().sum().item()
+    return {"runs_ms": ms["runs"], "encode_ms": ms["encode"], "decode_ms": ms["decode"],
+            "merge_q": q, "width_at_q": Wq, "width_max": Wmax, "max_possible": api.max_intervals(nb),
+            "runs_per_row_mean": round(n_runs.double().mean().item(), 2),
+            "rows_merged_frac": round((n_runs > Wq).double().mean().item(), 4),
+            "blocks_added_by_merge_frac": round((kcnt.double().sum().item() - before) / max(before, 1.0), 5),
+            "list_bytes": rows * nb * 4 + rows * 4, "interval_bytes_at_q": rows * Wq * 8 + rows * 4,
+            "interval_bytes_max": rows * Wmax * 8 + rows * 4, "status": int(st.item())}
+
+
 def run_ours(args, w, world, rank, local):
     from block_sparse_attention_logits_b200 import api, _lib
     from block_sparse_attention_logits_b200 import build as bsa_build
@@ -478,6 +521,15 @@ def run_ours(args, w, world, rank, local):
                  "kept_fraction_of_candidates": round(rcnt.double().sum().item() / max(cand.double().sum().item(), 1),
                                                       4)}
 
+    # the interval (skip-list) form of the step's kept lists; a failure here
+    # is reported in its own object and does not lose the step's line
+    intervals = None
+    if not args.no_refresh:
+        try:
+            intervals = interval_timings(bufs["idx"], bufs["cnt"], L, blk, D, barrier)
+        except Exception as e:  # noqa: BLE001
+            intervals = {"error": f"{type(e).__name__}: {e}"}
+
     # the elementwise calls (refinement at a refresh, standalone correction):
     # HBM-bound, three [B,H,L,D] bf16 streams each
     elementwise = None
@@ -581,7 +633,7 @@ def run_ours(args, w, world, rank, local):
         "stages_ms": {"gather_score_and_select": round(float(np.mean(sel_ms)), 4), "attention": round(attn_avg_ms, 4),
                       "rest": round(ms_step - attn_avg_ms - float(np.mean(sel_ms)), 4)},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "refresh": refresh, "reuse": reuse,
-        "elementwise": elementwise, "sweep": sweep,
+        "elementwise": elementwise, "sweep": sweep, "intervals": intervals,
         "gpu_launches": LAUNCHES_PER_STEP * K if w.hilbert else (LAUNCHES_PER_STEP - 1) * K,
         "clocks": clk,
     }

@@ -16,7 +16,8 @@ from ._lib import Shape, check
 __all__ = [
     "score_blocks", "select_topp_mask", "reorder_workspace_bytes", "reorder_tokens",
     "permute_tokens", "sparse_attn_fwd", "refresh_refinement", "apply_correction",
-    "n_blocks", "version",
+    "n_blocks", "version", "interval_runs", "interval_width_for_merge", "kept_to_intervals",
+    "intervals_to_kept", "max_intervals",
 ]
 
 
@@ -155,6 +156,94 @@ def select_topp_mask(probs, p, L, blk, D=128, mask=None, kept_idx=None, kept_cnt
         check("bsa_select_topp_mask_restricted", _lib.load().bsa_select_topp_mask_restricted(
             Shape(B, H, L, D, blk), _ptr(probs), parr, _ptr(candidates), _ptr(mask), _ptr(kept_idx),
             _ptr(kept_cnt), _stream()))
+    return mask, kept_idx, kept_cnt
+
+
+def max_intervals(NB):
+    """Most runs (intervals) a row of NB key blocks can have."""
+    return (NB + 1) // 2
+
+
+def interval_runs(kept_idx, kept_cnt, L, blk, D=128, n_runs=None, hist=None, status=None):
+    """Runs of consecutive kept blocks per row, and their histogram.
+
+    kept_idx int32 [B,H,NB,NB], kept_cnt int32 [B,H,NB].  Returns (n_runs
+    int32 [B,H,NB], hist int32 [max_intervals(NB) + 1]).  A passed-in hist is
+    accumulated into (not cleared); a new one starts at zero.
+    """
+    B, H, nb = kept_cnt.shape
+    _need(kept_idx, torch.int32, (B, H, nb, nb), "kept_idx")
+    _need(kept_cnt, torch.int32, (B, H, nb), "kept_cnt")
+    dev = kept_cnt.device
+    n_runs = n_runs if n_runs is not None else torch.empty((B, H, nb), dtype=torch.int32, device=dev)
+    hist = hist if hist is not None else torch.zeros(max_intervals(nb) + 1, dtype=torch.int32, device=dev)
+    _need(n_runs, torch.int32, (B, H, nb), "n_runs")
+    _need(hist, torch.int32, (max_intervals(nb) + 1,), "hist")
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
+    check("bsa_interval_runs", _lib.load().bsa_interval_runs(
+        Shape(B, H, L, D, blk), _ptr(kept_idx), _ptr(kept_cnt), _ptr(n_runs), _ptr(hist), _ptr(status), _stream()))
+    return n_runs, hist
+
+
+def interval_width_for_merge(hist, q):
+    """Interval width for a merge percentage q in (0, 1] (host computation in
+    libbsa): the smallest W >= 1 that at least ceil(q * rows) rows fit.
+    hist: the interval_runs histogram (any device; copied to the host)."""
+    h = hist.detach().to("cpu", torch.int32).contiguous() if isinstance(hist, torch.Tensor) else \
+        torch.tensor(list(hist), dtype=torch.int32)
+    arr = (ctypes.c_int32 * h.numel())(*h.tolist())
+    w = ctypes.c_int(0)
+    check("bsa_interval_width_for_merge", _lib.load().bsa_interval_width_for_merge(
+        arr, h.numel(), float(q), ctypes.byref(w)))
+    return w.value
+
+
+def kept_to_intervals(kept_idx, kept_cnt, W, L, blk, D=128, intervals=None, n_int=None, n_runs=None, status=None):
+    """Encode kept lists as interval pairs of width W (rows with more runs are
+    merged by filling their smallest gaps).  Returns (intervals int32
+    [B,H,NB,W,2], n_int int32 [B,H,NB], n_runs int32 [B,H,NB])."""
+    B, H, nb = kept_cnt.shape
+    _need(kept_idx, torch.int32, (B, H, nb, nb), "kept_idx")
+    _need(kept_cnt, torch.int32, (B, H, nb), "kept_cnt")
+    dev = kept_cnt.device
+    intervals = intervals if intervals is not None else torch.empty((B, H, nb, W, 2), dtype=torch.int32, device=dev)
+    n_int = n_int if n_int is not None else torch.empty((B, H, nb), dtype=torch.int32, device=dev)
+    n_runs = n_runs if n_runs is not None else torch.empty((B, H, nb), dtype=torch.int32, device=dev)
+    _need(intervals, torch.int32, (B, H, nb, W, 2), "intervals")
+    _need(n_int, torch.int32, (B, H, nb), "n_int")
+    _need(n_runs, torch.int32, (B, H, nb), "n_runs")
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
+    check("bsa_kept_to_intervals", _lib.load().bsa_kept_to_intervals(
+        Shape(B, H, L, D, blk), _ptr(kept_idx), _ptr(kept_cnt), int(W), _ptr(intervals), _ptr(n_int),
+        _ptr(n_runs), _ptr(status), _stream()))
+    return intervals, n_int, n_runs
+
+
+def intervals_to_kept(intervals, n_int, L, blk, D=128, mask=None, kept_idx=None, kept_cnt=None, want_mask=True,
+                      status=None):
+    """Decode interval pairs (int32 [B,H,NB,W,2], n_int int32 [B,H,NB]) into
+    (mask uint8 or None, kept_idx int32 [B,H,NB,NB], kept_cnt int32 [B,H,NB]),
+    the lists sparse_attn_fwd takes."""
+    B, H, nb, W, _ = intervals.shape
+    _need(intervals, torch.int32, (B, H, nb, W, 2), "intervals")
+    _need(n_int, torch.int32, (B, H, nb), "n_int")
+    dev = n_int.device
+    if want_mask:
+        mask = mask if mask is not None else torch.empty((B, H, nb, nb), dtype=torch.uint8, device=dev)
+        _need(mask, torch.uint8, (B, H, nb, nb), "mask")
+    else:
+        mask = None
+    kept_idx = kept_idx if kept_idx is not None else torch.empty((B, H, nb, nb), dtype=torch.int32, device=dev)
+    kept_cnt = kept_cnt if kept_cnt is not None else torch.empty((B, H, nb), dtype=torch.int32, device=dev)
+    _need(kept_idx, torch.int32, (B, H, nb, nb), "kept_idx")
+    _need(kept_cnt, torch.int32, (B, H, nb), "kept_cnt")
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
+    check("bsa_intervals_to_kept", _lib.load().bsa_intervals_to_kept(
+        Shape(B, H, L, D, blk), _ptr(intervals), _ptr(n_int), int(W), _ptr(mask), _ptr(kept_idx), _ptr(kept_cnt),
+        _ptr(status), _stream()))
     return mask, kept_idx, kept_cnt
 
 

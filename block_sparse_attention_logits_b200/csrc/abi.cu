@@ -152,6 +152,65 @@ int bsa_select_topp_mask_restricted(bsa_shape s, const float* probs, const float
   return select_common(s, probs, p_host, candidates, mask, kept_idx, kept_cnt, stream);
 }
 
+int bsa_interval_runs(bsa_shape s, const int32_t* kept_idx, const int32_t* kept_cnt, int32_t* n_runs, int32_t* hist,
+                      int32_t* status, bsa_stream stream) {
+  if (!kept_idx || !kept_cnt || !n_runs) return BSA_EINVAL;
+  if (!aligned16(kept_idx) || !aligned16(kept_cnt) || !aligned16(n_runs) || (hist && !aligned16(hist)))
+    return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (int r = check_device()) return r;
+  return from_cuda(bsa::launch_interval_encode(s, kept_idx, kept_cnt, 0, nullptr, nullptr, n_runs, hist, status,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int bsa_interval_width_for_merge(const int32_t* hist_host, int nbins, double q, int* W_out) {
+  if (!hist_host || !W_out || nbins < 2) return BSA_EINVAL;
+  if (!(q > 0.0) || !(q <= 1.0)) return BSA_EINVAL;  // rejects NaN too
+  long long rows = 0;
+  for (int r = 0; r < nbins; ++r) {
+    if (hist_host[r] < 0) return BSA_EINVAL;
+    rows += hist_host[r];
+  }
+  const double need = std::ceil(q * static_cast<double>(rows));
+  long long covered = hist_host[0];
+  int W = nbins - 1;
+  for (int w = 1; w < nbins; ++w) {
+    covered += hist_host[w];
+    if (static_cast<double>(covered) >= need) {
+      W = w;
+      break;
+    }
+  }
+  *W_out = W;
+  return BSA_OK;
+}
+
+int bsa_kept_to_intervals(bsa_shape s, const int32_t* kept_idx, const int32_t* kept_cnt, int W, int32_t* intervals,
+                          int32_t* n_int, int32_t* n_runs, int32_t* status, bsa_stream stream) {
+  if (!kept_idx || !kept_cnt || !intervals || !n_int) return BSA_EINVAL;
+  if (!aligned16(kept_idx) || !aligned16(kept_cnt) || !aligned16(intervals) || !aligned16(n_int) ||
+      (n_runs && !aligned16(n_runs)))
+    return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (W < 1 || W > n_blocks(s.L, s.blk)) return BSA_EINVAL;
+  if (int r = check_device()) return r;
+  return from_cuda(bsa::launch_interval_encode(s, kept_idx, kept_cnt, W, intervals, n_int, n_runs, nullptr, status,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int bsa_intervals_to_kept(bsa_shape s, const int32_t* intervals, const int32_t* n_int, int W, uint8_t* mask,
+                          int32_t* kept_idx, int32_t* kept_cnt, int32_t* status, bsa_stream stream) {
+  if (!intervals || !n_int || !kept_idx || !kept_cnt) return BSA_EINVAL;
+  if (!aligned16(intervals) || !aligned16(n_int) || !aligned16(kept_idx) || !aligned16(kept_cnt) ||
+      (mask && !aligned16(mask)))
+    return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (W < 1 || W > n_blocks(s.L, s.blk)) return BSA_EINVAL;
+  if (int r = check_device()) return r;
+  return from_cuda(bsa::launch_interval_decode(s, intervals, n_int, W, mask, kept_idx, kept_cnt, status,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t bsa_reorder_workspace_bytes(int T, int Hh, int W) { return bsa::hilbert_workspace_bytes(T, Hh, W); }
 
 int bsa_reorder_tokens(int T, int Hh, int W, int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes,

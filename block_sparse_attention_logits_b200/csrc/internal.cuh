@@ -34,6 +34,15 @@ cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p,
 // drift[b*H + h] of the block means against reference means, [B,H,NB,D] each
 cudaError_t launch_drift(const bsa_shape& s, const float* qp_ref, const float* kp_ref, const float* qp,
                          const float* kp, float* drift, cudaStream_t st);
+// interval form of the kept lists: W == 0 counts runs per row (n_runs
+// required, hist nullable, accumulated); W >= 1 encodes intervals of width W
+int max_intervals(int NB);
+cudaError_t launch_interval_encode(const bsa_shape& s, const int32_t* kept_idx, const int32_t* kept_cnt, int W,
+                                   int32_t* intervals, int32_t* n_int, int32_t* n_runs, int32_t* hist,
+                                   int32_t* status, cudaStream_t st);
+cudaError_t launch_interval_decode(const bsa_shape& s, const int32_t* intervals, const int32_t* n_int, int W,
+                                   uint8_t* mask, int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
+                                   cudaStream_t st);
 size_t hilbert_workspace_bytes(int T, int Hh, int W);
 cudaError_t launch_hilbert(int T, int Hh, int W, int32_t* perm, int32_t* inv, void* ws, cudaStream_t st);
 cudaError_t launch_permute(const bsa_shape& s, const __nv_bfloat16* x, const int32_t* perm, __nv_bfloat16* y,

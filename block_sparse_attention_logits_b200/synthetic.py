@@ -99,3 +99,36 @@ def random_bf16(shape, seed, scale=1.0):
     g = torch.Generator(device="cpu")
     g.manual_seed(int(seed))
     return (torch.randn(shape, generator=g, dtype=torch.float32) * scale).to(torch.bfloat16)
+
+
+def random_kept_lists(B, H, NB, seed, density=0.1, mean_run=2.0, special_rows=True):
+    """Ascending kept key-block lists for the list-encoding stages: int32
+    [B,H,NB,NB] padded with -1 and int32 counts [B,H,NB].
+
+    Each row is an on/off Markov chain along the key blocks: a kept run ends
+    with probability 1/mean_run per block and a skipped run ends with
+    probability density/(mean_run (1 - density)), so runs of kept blocks have
+    mean length mean_run and a `density` share of the blocks is kept in the
+    long run (the clustered rows top-p selection gives on video tokens).
+    With special_rows, rows (0, 0, 0..3) are: empty, every block, every other
+    block (the most runs a row can have) and only the last block.
+    """
+    assert 0.0 < density < 1.0 and mean_run >= 1.0
+    rng = np.random.default_rng(seed)
+    p_off = 1.0 / mean_run
+    p_on = min(1.0, density * p_off / (1.0 - density))
+    u = rng.random((B, H, NB, NB))
+    state = rng.random((B, H, NB)) < density
+    on = np.zeros((B, H, NB, NB), dtype=bool)
+    for j in range(NB):
+        state = np.where(state, u[..., j] >= p_off, u[..., j] < p_on)
+        on[..., j] = state
+    if special_rows and NB >= 4:
+        on[0, 0, 0] = False
+        on[0, 0, 1] = True
+        on[0, 0, 2] = np.arange(NB) % 2 == 0
+        on[0, 0, 3] = np.arange(NB) == NB - 1
+    cnt = on.sum(axis=-1).astype(np.int32)
+    order = np.argsort(~on, axis=-1, kind="stable")
+    idx = np.where(np.arange(NB) < cnt[..., None], order, -1).astype(np.int32)
+    return idx, cnt

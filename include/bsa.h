@@ -223,6 +223,80 @@ BSA_API int bsa_select_topp_mask_restricted(bsa_shape s, const float* probs, con
                                     int32_t* kept_cnt, bsa_stream stream);
 
 /*
+ * Interval (skip-list) form of the kept key blocks.
+ * Defines: skip lists that store, per query-block row, interval pairs of key
+ * blocks; the number of intervals per row (CalibAtt appendix, Fig. S9); per-
+ * layer trimming of the rows to the widest one and merging of outlier rows so
+ * that the width falls further (Fig. S10 (b), (c)); the width chosen by a
+ * merge percentage (Table S3, "Merge %": 100 = no merge, 99, 95).
+ * A row's runs are the maximal runs of consecutive indices of its ascending
+ * kept list, each stored as an int32 pair (start, end), end exclusive.  A row
+ * of NB blocks has at most ceil(NB/2) runs.  Merging a row to width W fills
+ * the gaps between its neighbouring runs smallest first (the leftmost of
+ * equal gaps first) until W intervals remain: the merged row keeps a superset
+ * of its blocks, with the fewest blocks added.
+ * Rows are (b,h,i) of [B,H,NB]; kept_idx/kept_cnt as bsa_select_topp_mask
+ * writes them.  A row whose count lies outside [0, NB] or whose first
+ * kept_cnt entries are not strictly ascending within [0, NB) is malformed:
+ * it is flagged (BSA_DEV_BAD_INDEX in the optional device status word, OR-ed;
+ * the caller zeroes it) and treated as empty, as the calls below state.
+ */
+
+/*
+ * bsa_interval_runs -- runs per row and their histogram.
+ * Outputs n_runs: device int32 [B,H,NB] (0 for a malformed row); hist:
+ * device int32 [ceil(NB/2) + 1] or NULL, hist[r] += the number of well-formed
+ * rows with r runs.  hist is accumulated, not cleared: zero it once, then
+ * accumulate over the heads, layers and steps that will share one width.
+ * Errors: BSA_EINVAL on null required or misaligned pointers; BSA_ESHAPE;
+ * BSA_ENODEV; BSA_ECUDA.
+ */
+BSA_API int bsa_interval_runs(bsa_shape s, const int32_t* kept_idx, const int32_t* kept_cnt, int32_t* n_runs,
+                              int32_t* hist, int32_t* status, bsa_stream stream);
+
+/*
+ * bsa_interval_width_for_merge -- HOST function, no device work: the interval
+ * width for a merge percentage q in (0, 1].  W is the smallest width >= 1
+ * such that at least ceil(q * rows) rows (IEEE double product) have at most W
+ * runs, rows being the sum of the histogram.  q = 1 gives the widest row (no
+ * merge); q = 0.95 merges the 5% widest rows.
+ * Arguments: hist_host: HOST int32 [nbins] (the bsa_interval_runs histogram
+ * copied back, nbins = ceil(NB/2) + 1 >= 2); W_out: HOST int.
+ * Errors: BSA_EINVAL on a null pointer, nbins < 2, a negative count or q
+ * outside (0, 1].
+ */
+BSA_API int bsa_interval_width_for_merge(const int32_t* hist_host, int nbins, double q, int* W_out);
+
+/*
+ * bsa_kept_to_intervals -- encode the kept lists as interval pairs of width W.
+ * Outputs intervals: device int32 [B,H,NB,W,2], each row's pairs ascending,
+ * pairs past its count set to (-1, -1); n_int: device int32 [B,H,NB] =
+ * min(runs, W); n_runs: device int32 [B,H,NB] (runs before merging) or NULL.
+ * A row with more than W runs is merged to exactly W intervals.  A malformed
+ * row gets n_int = 0 and all pairs (-1, -1).  1 <= W <= NB.
+ * Errors: BSA_EINVAL on null required or misaligned pointers or W out of
+ * range; BSA_ESHAPE; BSA_ENODEV; BSA_ECUDA.
+ */
+BSA_API int bsa_kept_to_intervals(bsa_shape s, const int32_t* kept_idx, const int32_t* kept_cnt, int W,
+                                  int32_t* intervals, int32_t* n_int, int32_t* n_runs, int32_t* status,
+                                  bsa_stream stream);
+
+/*
+ * bsa_intervals_to_kept -- decode interval pairs into the mask and kept lists
+ * that bsa_sparse_attn_fwd takes.
+ * Inputs intervals int32 [B,H,NB,W,2] and n_int int32 [B,H,NB] as
+ * bsa_kept_to_intervals writes them.  A row is well formed when
+ * 0 <= n_int <= W and its first n_int pairs satisfy 0 <= start < end <= NB
+ * and start >= the previous pair's end; a malformed row decodes as empty.
+ * Outputs mask uint8 [B,H,NB,NB] or NULL (1 = kept, whole row written),
+ * kept_idx int32 [B,H,NB,NB] (first kept_cnt entries ascending; the rest
+ * unspecified), kept_cnt int32 [B,H,NB].  1 <= W <= NB.
+ * Errors: as bsa_kept_to_intervals.
+ */
+BSA_API int bsa_intervals_to_kept(bsa_shape s, const int32_t* intervals, const int32_t* n_int, int W, uint8_t* mask,
+                                  int32_t* kept_idx, int32_t* kept_cnt, int32_t* status, bsa_stream stream);
+
+/*
  * bsa_sparse_attn_fwd -- block-sparse attention forward with an optional
  * fused correction epilogue.
  * Defines: computing the selected connections densely and skipping the

@@ -172,3 +172,50 @@ def test_elementwise_validation(lib):
     assert lib.bsa_refresh_refinement(Shape(1, 1, 10, 16, 0), FAKE, NULL, FAKE, NULL) == _lib.BSA_EINVAL
     assert lib.bsa_apply_correction(Shape(1, 1, 10, 16, 0), FAKE, FAKE, NULL, FAKE, NULL) == _lib.BSA_EINVAL
     assert lib.bsa_permute_tokens(Shape(1, 1, 10, 16, 0), FAKE, FAKE, FAKE, 0, NULL) == _lib.BSA_EINVAL  # x == y
+
+
+def test_interval_validation(lib):
+    s = Shape(1, 2, 1000, 128, 128)   # NB = 8
+    # runs: kept lists and n_runs required; hist optional
+    assert lib.bsa_interval_runs(s, NULL, FAKE, FAKE, NULL, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_interval_runs(s, FAKE, FAKE, NULL, FAKE, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_interval_runs(s, FAKE, FAKE, FAKE, MISALIGNED, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_interval_runs(Shape(1, 2, 1000, 128, 96), FAKE, FAKE, FAKE, NULL, NULL, NULL) == _lib.BSA_ESHAPE
+    # encode / decode: width in [1, NB]
+    for W in (0, -1, 9):
+        assert lib.bsa_kept_to_intervals(s, FAKE, FAKE, W, FAKE, FAKE, NULL, NULL, NULL) == _lib.BSA_EINVAL
+        assert lib.bsa_intervals_to_kept(s, FAKE, FAKE, W, NULL, FAKE, FAKE, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_kept_to_intervals(s, FAKE, FAKE, 3, NULL, FAKE, NULL, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_kept_to_intervals(s, FAKE, FAKE, 3, FAKE, FAKE, MISALIGNED, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_intervals_to_kept(s, FAKE, NULL, 3, NULL, FAKE, FAKE, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_intervals_to_kept(s, FAKE, FAKE, 3, MISALIGNED, FAKE, FAKE, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_intervals_to_kept(Shape(0, 2, 1000, 128, 128), FAKE, FAKE, 3, NULL, FAKE, FAKE, NULL,
+                                     NULL) == _lib.BSA_ESHAPE
+
+
+def _width(lib, hist, q):
+    arr = (ctypes.c_int32 * len(hist))(*hist)
+    w = ctypes.c_int(-7)
+    code = lib.bsa_interval_width_for_merge(arr, len(hist), q, ctypes.byref(w))
+    return code, w.value
+
+
+def test_interval_width_host_function_matches_oracle(lib):
+    """bsa_interval_width_for_merge is host code of the library: it runs here,
+    and agrees with the oracle on random and edge-case histograms."""
+    import numpy as np
+    from oracle import intervals as oint
+    rng = np.random.default_rng(7)
+    for _ in range(300):
+        nb = int(rng.integers(2, 40))
+        hist = rng.integers(0, 50, size=nb) * (rng.random(nb) < 0.6)
+        for q in (1e-9, 0.3, 0.5, 0.9, 0.95, 0.99, 1.0, float(rng.random())):
+            code, w = _width(lib, hist.tolist(), q)
+            assert code == _lib.BSA_OK and w == oint.width_for_merge(hist, q), (hist, q)
+    assert _width(lib, [0, 0, 0], 1.0) == (_lib.BSA_OK, 1)
+    assert _width(lib, [5], 1.0)[0] == _lib.BSA_EINVAL           # fewer than 2 bins
+    assert _width(lib, [1, -1, 3], 1.0)[0] == _lib.BSA_EINVAL      # negative count
+    for q in (0.0, -0.5, 1.5, float("nan")):
+        assert _width(lib, [1, 2, 3], q)[0] == _lib.BSA_EINVAL
+    w = ctypes.c_int(0)
+    assert lib.bsa_interval_width_for_merge(None, 3, 1.0, ctypes.byref(w)) == _lib.BSA_EINVAL
