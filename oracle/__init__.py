@@ -12,7 +12,8 @@ Sources (cited by page title and section in every function):
 
 * "RECAP: Reciprocal Sparse Attention and Hierarchical Caching for Efficient
   Video Diffusion" -- full text, sections 1, 3.2, 3.4 (block means, cached
-  dense refinement that corrects the sparse estimate, dense refreshes).
+  dense refinement that corrects the sparse estimate, dense refreshes; the
+  coarse tail of the omitted blocks and its reconstruction, section 3.2).
 * the head-wise adaptive top-p abstract (Temporal Mask Reuse / Error-guided
   Budgeted Calibration) and the GSRS abstract ("Top-p selection for adaptive
   sparsity control") -- online top-p block selection with per-head p.
@@ -36,6 +37,9 @@ Modules:
                  attention, refinement, exact kept attention mass)
   reuse       -- query-key drift of the block means, and scoring / selection
                  restricted to an earlier candidate set
+  tail        -- coarse estimate of the omitted attention tail (block means
+                 with the key-variance and value-key covariance corrections)
+                 and its reconstruction with a cached refinement
   intervals   -- interval (skip-list) encoding of the kept blocks, merging of
                  outlier rows to a width, the width for a merge percentage
 
@@ -43,4 +47,4 @@ Every function carries a "Pinned by" note naming the tests in
 ``tests/test_oracle.py`` that tie it to something other than itself.
 """
 
-from . import hilbert, scoring, topp, attention, correction, refresh, reuse, intervals  # noqa: F401
+from . import hilbert, scoring, topp, attention, correction, refresh, reuse, intervals, tail  # noqa: F401

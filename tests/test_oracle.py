@@ -23,6 +23,7 @@ from oracle import intervals as oint
 from oracle import refresh as oref
 from oracle import reuse as oreu
 from oracle import scoring as osco
+from oracle import tail as otail
 from oracle import topp as otop
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -678,6 +679,155 @@ def test_planted_mistake_inclusive_end_is_caught(monkeypatch):
     monkeypatch.setattr(oint, "runs_of", lambda kept: [(s, e - 1) for s, e in orig(kept)])
     with pytest.raises(AssertionError):
         test_intervals_golden_rows_and_widths()
+
+
+# ------------------------------------------------ coarse tail (RECAP section 3.2)
+
+def _random_lists(rng, B, H, NB, keep=0.4):
+    idx = np.full((B, H, NB, NB), -1, np.int32)
+    cnt = np.zeros((B, H, NB), np.int32)
+    for pos in np.ndindex(B, H, NB):
+        kept = np.flatnonzero(rng.random(NB) < keep)
+        idx[pos][: kept.size] = kept
+        cnt[pos] = kept.size
+    idx[0, 0, 0] = np.arange(NB)      # a row keeping everything (empty tail)
+    cnt[0, 0, 0] = NB
+    cnt[0, 0, 1] = 0                   # a row keeping nothing
+    return idx, cnt
+
+
+def test_tail_is_exact_for_constant_blocks():
+    """Keys and values constant within every block: zero key variance and zero
+    value-key covariance, so the coarse tail equals the exact tail (closed
+    form n_j exp(a . k_j) for the block masses)."""
+    rng = np.random.default_rng(31)
+    B, H, D, blk = 1, 2, 8, 16
+    L = 5 * blk + 7
+    NB = (L + blk - 1) // blk
+    kap = rng.standard_normal((B, H, NB, D))
+    nu = rng.standard_normal((B, H, NB, D))
+    blocks = np.minimum(np.arange(L) // blk, NB - 1)
+    k, v = kap[:, :, blocks], nu[:, :, blocks]
+    q = rng.standard_normal((B, H, L, D)) * 2.0
+    idx, cnt = _random_lists(rng, B, H, NB)
+    stats = otail.block_stats(k, v, blk)
+    assert np.all(stats[1] < 1e-24) and np.all(np.abs(stats[4]) < 1e-12)
+    lbar, obar = otail.coarse_tail(q, stats, idx, cnt, blk)
+    l_T, o_T = otail.exact_tail(q, k, v, idx, cnt, blk)
+    fin = np.isfinite(l_T)
+    assert np.array_equal(fin, np.isfinite(lbar))
+    assert np.allclose(lbar[fin], l_T[fin], rtol=0, atol=1e-10)
+    assert np.allclose(obar[fin], o_T[fin], rtol=0, atol=1e-10)
+    assert np.all(np.isneginf(lbar[0, 0, :blk])) and np.all(obar[0, 0, :blk] == 0)
+
+
+def _gaussian_block_case(seed):
+    """One large block of Gaussian keys (diagonal covariance) with values
+    v = M k + noise, followed by a short query block that keeps only itself,
+    so that its tail is exactly the large block."""
+    rng = np.random.default_rng(seed)
+    D, blk, nq = 4, 65536, 8
+    L = blk + nq
+    mu = np.array([0.3, -0.2, 0.5, 0.1])
+    sd = np.array([0.5, 0.8, 0.3, 0.6])
+    M = np.array([[1.0, 0.5, 0.0, -0.3], [0.2, -1.0, 0.4, 0.0], [0.0, 0.3, 0.8, 0.5], [-0.6, 0.0, 0.2, 1.0]])
+    k = np.empty((1, 1, L, D))
+    k[0, 0, :blk] = mu + sd * rng.standard_normal((blk, D))
+    k[0, 0, blk:] = rng.standard_normal((nq, D))
+    v = np.empty((1, 1, L, D))
+    v[0, 0] = k[0, 0] @ M.T + 0.3 * rng.standard_normal((L, D))
+    q = np.zeros((1, 1, L, D))
+    q[0, 0, blk:] = np.array([1.2, -0.9, 1.5, 0.8]) * (1 + 0.1 * rng.standard_normal((nq, D)))
+    idx = np.full((1, 1, 2, 2), -1, np.int32)
+    cnt = np.ones((1, 1, 2), np.int32)
+    idx[0, 0, 0, 0], idx[0, 0, 1, 0] = 0, 1     # block 0 keeps itself, block 1 keeps itself
+    return q, k, v, idx, cnt, blk, mu, sd, M
+
+
+def test_tail_mass_is_the_gaussian_limit():
+    """COBS reading: for Gaussian keys log mean_c exp(a . k_c) tends to
+    a . mu + 1/2 sum_d a_d^2 sd_d^2.  The coarse log-mass matches the exact
+    tail's within Monte Carlo error (~2e-3 at 65536 keys); dropping the
+    variance term or doubling it misses by ~0.15."""
+    q, k, v, idx, cnt, blk, mu, sd, M = _gaussian_block_case(41)
+    lbar, _ = otail.coarse_tail(q, otail.block_stats(k, v, blk), idx, cnt, blk)
+    l_T, _ = otail.exact_tail(q, k, v, idx, cnt, blk)
+    rows = slice(blk, None)
+    a = q[0, 0, rows] / 2.0
+    err = np.abs(lbar[0, 0, rows] - l_T[0, 0, rows])
+    assert err.max() < 0.02
+    half_var = 0.5 * (a * a) @ (sd * sd)
+    assert half_var.min() > 0.1                    # the variance term is not negligible here
+    limit = np.log(blk) + a @ mu + half_var        # the population-moment closed form
+    assert np.abs(l_T[0, 0, rows] - limit).max() < 0.03
+
+
+def test_tail_value_is_the_gaussian_limit():
+    """PISA reading: for jointly Gaussian keys and values the exp-weighted
+    value mean is vbar + Cov(v, k) a.  The coarse output matches the exact
+    tail output within Monte Carlo error; without C, or with C transposed, it
+    misses by more than 0.1."""
+    q, k, v, idx, cnt, blk, mu, sd, M = _gaussian_block_case(42)
+    stats = otail.block_stats(k, v, blk)
+    _, obar = otail.coarse_tail(q, stats, idx, cnt, blk)
+    _, o_T = otail.exact_tail(q, k, v, idx, cnt, blk)
+    rows = slice(blk, None)
+    a = q[0, 0, rows] / 2.0
+    assert np.abs(obar[0, 0, rows] - o_T[0, 0, rows]).max() < 0.03
+    comp = a @ (M @ np.diag(sd * sd)).T            # M Sigma a, the population closed form
+    assert np.abs(comp).max() > 0.1
+    assert np.abs(o_T[0, 0, rows] - (mu @ M.T + comp)).max() < 0.04
+    wrong = a @ (M @ np.diag(sd * sd))             # transposed covariance
+    assert np.abs(wrong - comp).max() > 0.1
+
+
+def test_reconstruction_with_same_step_refinement_is_dense():
+    """A refinement taken at the step itself makes the reconstructed tail exact,
+    so sparse part + tail is dense attention (the LSE merge of a partition of
+    the keys); a row keeping every block returns its sparse output."""
+    rng = np.random.default_rng(43)
+    B, H, D, blk = 1, 2, 16, 16
+    L = 6 * blk + 5
+    NB = (L + blk - 1) // blk
+    q, k, v = (rng.standard_normal((B, H, L, D)) for _ in range(3))
+    idx, cnt = _random_lists(rng, B, H, NB)
+    O_S, l_S = oatt.masked_attention(q, k, v, idx, cnt, blk)
+    lbar, obar = otail.coarse_tail(q, otail.block_stats(k, v, blk), idx, cnt, blk)
+    l_T, o_T = otail.exact_tail(q, k, v, idx, cnt, blk)
+    d_l, d_o = otail.refinement(l_T, o_T, lbar, obar)
+    O, lse = otail.reconstruct(l_S, O_S, lbar, obar, d_l, d_o)
+    O_d, l_d = oatt.dense_attention(q, k, v)
+    assert np.allclose(O, O_d, rtol=0, atol=1e-10) and np.allclose(lse, l_d, rtol=1e-12, atol=0)
+    assert np.array_equal(O[0, 0, :blk], O_S[0, 0, :blk])       # all kept: the tail is empty
+    # a stale refinement still leaves the all-kept row untouched and keeps the
+    # output a convex combination in weight (the weights sum to 1)
+    O2, lse2 = otail.reconstruct(l_S, O_S, lbar, obar, 0.5 * d_l, 0.5 * d_o)
+    assert np.array_equal(O2[0, 0, :blk], O_S[0, 0, :blk])
+    ws = np.exp(np.nan_to_num(l_S, neginf=-np.inf) - lse2)
+    wt = np.exp(lbar + 0.5 * d_l - lse2)
+    assert np.allclose(np.where(np.isneginf(l_S), 0, ws) + np.where(np.isneginf(lbar), 0, wt), 1.0, atol=1e-12)
+
+
+def test_planted_mistake_variance_factor_is_caught(monkeypatch):
+    orig = otail.block_stats
+
+    def doubled(k, v, blk):
+        kbar, s2, vbar, n, C = orig(k, v, blk)
+        return kbar, 2 * s2, vbar, n, C     # as if the second-order term had no 1/2
+    monkeypatch.setattr(otail, "block_stats", doubled)
+    with pytest.raises(AssertionError):
+        test_tail_mass_is_the_gaussian_limit()
+
+
+def test_planted_mistake_transposed_covariance_is_caught(monkeypatch):
+    orig = otail.block_stats
+
+    def transposed(k, v, blk):
+        kbar, s2, vbar, n, C = orig(k, v, blk)
+        return kbar, s2, vbar, n, np.swapaxes(C, -1, -2)
+    monkeypatch.setattr(otail, "block_stats", transposed)
+    with pytest.raises(AssertionError):
+        test_tail_value_is_the_gaussian_limit()
 
 
 # ------------------------------------------------- planted mistakes are caught
