@@ -14,10 +14,24 @@ from . import _lib
 from ._lib import Shape, check
 
 __all__ = [
-    "score_blocks", "select_topp_mask", "reorder_workspace_bytes", "reorder_tokens",
-    "permute_tokens", "sparse_attn_fwd", "refresh_refinement", "apply_correction",
-    "n_blocks", "version", "interval_runs", "interval_width_for_merge", "kept_to_intervals",
-    "intervals_to_kept", "max_intervals",
+    "n_blocks",
+    "version",
+    "score_blocks",
+    "score_blocks_gather",
+    "block_drift",
+    "select_topp_mask",
+    "max_intervals",
+    "interval_runs",
+    "interval_width_for_merge",
+    "kept_to_intervals",
+    "intervals_to_kept",
+    "reorder_workspace_bytes",
+    "reorder_tokens",
+    "permute_tokens",
+    "sparse_attn_fwd",
+    "sparse_attn_refresh",
+    "refresh_refinement",
+    "apply_correction",
 ]
 
 
