@@ -13,6 +13,8 @@
 // order while the running mass is still below T (a warp prefix scan).  All
 // sums are exact uint64 integer sums, so the result does not depend on the
 // order of summation and equals the sequential definition bit for bit.
+// Rows of up to 1024 blocks keep their keys and masses in registers
+// (select_reg_kernel); longer rows stage them in shared memory.
 //
 // Restricted form (GSRS abstract: later searches restricted to an early
 // candidate set): with a candidate mask the search runs over the candidate
@@ -166,11 +168,149 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ p
   if (lane == 0) kept_cnt[row] = count;
 }
 
+// Register-resident form of select_kernel for NB <= 32 R: lane l holds the
+// key and the fixed-point mass of blocks j = 32 r + l (r < R), so the 31-step
+// search reads no shared memory (the shared-memory form re-reads the whole
+// row at every step).  Same arithmetic and the same result bit for bit.
+template <int R>
+__global__ void __launch_bounds__(256) select_reg_kernel(const float* __restrict__ probs,
+                                                         const __grid_constant__ TopP tp,
+                                                         const uint8_t* __restrict__ cand,
+                                                         uint8_t* __restrict__ mask, int32_t* __restrict__ kept_idx,
+                                                         int32_t* __restrict__ kept_cnt, int H, int NB,
+                                                         long long rows) {
+  const int warps = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * warps + w;
+  if (row >= rows) return;
+  const int h = static_cast<int>((row / NB) % H);
+  const float p = tp.p[h];
+  const float* P = probs + row * NB;
+  uint8_t* mrow = mask + row * NB;
+  int32_t* irow = kept_idx + row * NB;
+  const uint8_t* crow = cand ? cand + row * NB : nullptr;
+  if (p == 1.0f && !crow) {
+    for (int j = lane; j < NB; j += 32) {
+      mrow[j] = 1;
+      irow[j] = j;
+    }
+    if (lane == 0) kept_cnt[row] = NB;
+    return;
+  }
+
+  uint32_t key[R];
+  uint64_t u[R];
+  uint64_t total = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int j = 32 * r + lane;
+    uint32_t kk = 0u;
+    if (j < NB && (!crow || crow[j])) kk = prob_key(__ldg(P + j));
+    key[r] = kk;
+    u[r] = fixed_mass(kk);
+    total += u[r];
+  }
+  total = warp_sum(total);
+  const uint64_t T = static_cast<uint64_t>(ceil(static_cast<double>(p) * static_cast<double>(total)));
+
+  uint32_t tau;
+  if (p == 1.0f) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int j = 32 * r + lane;
+      if (j < NB && crow[j]) key[r] = kSelected;
+    }
+    tau = kSelected - 1u;
+  } else if (T == 0) {
+    uint32_t best_key = 0;
+    int best_j = 0x7FFFFFFF;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int j = 32 * r + lane;
+      if (j >= NB || (crow && !crow[j])) continue;
+      if (key[r] > best_key || (key[r] == best_key && j < best_j)) {
+        best_key = key[r];
+        best_j = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint32_t ok = __shfl_xor_sync(0xffffffffu, best_key, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, best_j, o);
+      if (ok > best_key || (ok == best_key && oj < best_j)) {
+        best_key = ok;
+        best_j = oj;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (32 * r + lane == best_j) key[r] = kSelected;
+    tau = kSelected - 1u;
+  } else {
+    tau = 0;
+#pragma unroll 1
+    for (int b = 30; b >= 0; --b) {
+      const uint32_t c = tau | (1u << b);
+      uint64_t g = 0;
+#pragma unroll
+      for (int r = 0; r < R; ++r) g += key[r] >= c ? u[r] : 0ull;
+      if (warp_sum(g) >= T) tau = c;
+    }
+    uint64_t above = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) above += key[r] > tau ? u[r] : 0ull;
+    const uint64_t need = T - warp_sum(above);  // > 0 by maximality of tau
+    // blocks equal to tau, in ascending index order, while mass is short
+    uint64_t carry = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int j = 32 * r + lane;
+      const bool tie = j < NB && key[r] == tau;
+      const uint64_t val = tie ? u[r] : 0ull;
+      uint64_t incl = val;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (tie && carry + (incl - val) < need) key[r] = kSelected;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  // emit mask and the ascending kept list
+  int count = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int j = 32 * r + lane;
+    const bool sel = j < NB && key[r] > tau;
+    if (j < NB) mrow[j] = sel ? 1 : 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, sel);
+    if (sel) irow[count + __popc(bal & ((1u << lane) - 1u))] = j;
+    count += __popc(bal);
+  }
+  if (lane == 0) kept_cnt[row] = count;
+}
+
+template <int R>
+cudaError_t launch_select_reg(const float* probs, const TopP& p, const uint8_t* cand, uint8_t* mask, int32_t* idx,
+                              int32_t* cnt, int H, int NB, long long rows, cudaStream_t st) {
+  constexpr int kWarps = 8;
+  const long long grid = (rows + kWarps - 1) / kWarps;
+  select_reg_kernel<R><<<static_cast<unsigned>(grid), kWarps * 32, 0, st>>>(probs, p, cand, mask, idx, cnt, H, NB,
+                                                                          rows);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p, const uint8_t* cand, uint8_t* mask,
                           int32_t* idx, int32_t* cnt, cudaStream_t st) {
   const int NB = n_blocks(s.L, s.blk);
+  const long long rows = static_cast<long long>(s.B) * s.H * NB;
+  if (NB <= 32 * 8) return launch_select_reg<8>(probs, p, cand, mask, idx, cnt, s.H, NB, rows, st);
+  if (NB <= 32 * 20) return launch_select_reg<20>(probs, p, cand, mask, idx, cnt, s.H, NB, rows, st);
+  if (NB <= 32 * 32) return launch_select_reg<32>(probs, p, cand, mask, idx, cnt, s.H, NB, rows, st);
   const int nbp = (NB + 1) & ~1;
   const size_t per_warp = static_cast<size_t>(nbp) * 12;
   int warps = static_cast<int>((160 * 1024) / per_warp);
@@ -184,7 +324,6 @@ cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p,
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  const long long rows = static_cast<long long>(s.B) * s.H * NB;
   const long long grid = (rows + warps - 1) / warps;
   select_kernel<<<static_cast<unsigned>(grid), warps * 32, smem, st>>>(probs, p, cand, mask, idx, cnt, s.H, NB, rows,
                                                                        nbp);

@@ -83,7 +83,8 @@ def test_select_exact_on_oracle_scores_480p(p):
     _select_exact(P, np.array([p, p], np.float32), w.L, w.blk, w.D)
 
 
-@pytest.mark.parametrize("nb,ties", [(37, True), (37, False), (929, False), (1, False), (300, True)])
+@pytest.mark.parametrize("nb,ties", [(37, True), (37, False), (929, False), (1, False), (300, True), (256, False),
+                                     (257, True), (640, False), (641, True), (1024, False), (1100, True)])
 def test_select_exact_random_rows(nb, ties):
     P = random_probs(2, 3, nb, seed=nb + 10 * ties, temperature=2.0, ties=ties)
     _select_exact(P, np.array([0.9, 0.35, 1.0], np.float32), nb * 128, 128, 128)

@@ -68,10 +68,10 @@ def test_restricted_scoring_matches_oracle():
     assert np.all(Pg[cand == 0] == 0) and np.all(Pg[0, 0, 2] == 0)
 
 
-@pytest.mark.parametrize("seed", [60, 61])
-def test_restricted_selection_bit_exact(seed):
+@pytest.mark.parametrize("seed,NB", [(60, 45), (61, 45), (62, 600), (63, 1050)])
+def test_restricted_selection_bit_exact(seed, NB):
     rng = np.random.default_rng(seed)
-    B, H, NB, blk, D = 1, 4, 45, 128, 128
+    B, H, blk, D = 1, 4, 128, 128
     L = NB * blk
     P = rng.dirichlet(np.full(NB, 0.3), size=(B, H, NB)).astype(np.float32)
     P[0, 1, 5, ::3] = P[0, 1, 5, 0]     # ties
