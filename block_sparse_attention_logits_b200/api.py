@@ -270,9 +270,12 @@ def reorder_tokens(T, Hh, W, device="cuda", perm=None, inv=None, workspace=None)
     L = T * Hh * W
     perm = perm if perm is not None else torch.empty(L, dtype=torch.int32, device=device)
     inv = inv if inv is not None else torch.empty(L, dtype=torch.int32, device=device)
+    _need(perm, torch.int32, (L,), "perm")
+    _need(inv, torch.int32, (L,), "inv")
     nbytes = reorder_workspace_bytes(T, Hh, W)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=perm.device)
+    _need(workspace, torch.uint8, (workspace.numel(),), "workspace")
     check("bsa_reorder_tokens", _lib.load().bsa_reorder_tokens(
         T, Hh, W, _ptr(perm), _ptr(inv), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream()))
@@ -314,6 +317,8 @@ def sparse_attn_fwd(q, k, v, blk, kept_idx=None, kept_cnt=None, R=None, alpha=No
     lse = lse if lse is not None else torch.empty((B, H, L), dtype=torch.float32, device=q.device)
     _need(o, torch.bfloat16, (B, H, L, D), "o")
     _need(lse, torch.float32, (B, H, L), "lse")
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
     if out_rows is None:
         check("bsa_sparse_attn_fwd", _lib.load().bsa_sparse_attn_fwd(
             Shape(B, H, L, D, blk), _ptr(q), _ptr(k), _ptr(v), _ptr(kept_idx), _ptr(kept_cnt),
@@ -363,6 +368,8 @@ def sparse_attn_refresh(q, k, v, blk, kept_idx, kept_cnt, want_r=True, want_mass
         _need(R, torch.bfloat16, (B, H, L, D), "R")
     if mass is not None:
         _need(mass, torch.float32, (B, H, L), "kept_mass")
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
     check("bsa_sparse_attn_refresh", _lib.load().bsa_sparse_attn_refresh(
         Shape(B, H, L, D, blk), _ptr(q), _ptr(k), _ptr(v), _ptr(kept_idx), _ptr(kept_cnt),
         _ptr(o_d), _ptr(l_d), _ptr(o_s), _ptr(l_s), _ptr(R), _ptr(mass), _ptr(status), _stream()))
@@ -375,6 +382,7 @@ def refresh_refinement(o_dense, o_sparse, out=None):
     _need(o_dense, torch.bfloat16, (B, H, L, D), "o_dense")
     _need(o_sparse, torch.bfloat16, (B, H, L, D), "o_sparse")
     out = out if out is not None else torch.empty_like(o_dense)
+    _need(out, torch.bfloat16, (B, H, L, D), "out")
     check("bsa_refresh_refinement", _lib.load().bsa_refresh_refinement(
         Shape(B, H, L, D, 0), _ptr(o_dense), _ptr(o_sparse), _ptr(out), _stream()))
     return out
@@ -387,6 +395,7 @@ def apply_correction(o_sparse, R, alpha, out=None):
     _need(R, torch.bfloat16, (B, H, L, D), "R")
     _need(alpha, torch.float32, (H,), "alpha")
     out = out if out is not None else torch.empty_like(o_sparse)
+    _need(out, torch.bfloat16, (B, H, L, D), "out")
     check("bsa_apply_correction", _lib.load().bsa_apply_correction(
         Shape(B, H, L, D, 0), _ptr(o_sparse), _ptr(R), _ptr(alpha), _ptr(out), _stream()))
     return out
