@@ -13,6 +13,9 @@ namespace {
 using bsa::n_blocks;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// A 32-bit word the device reads or updates atomically (status, alpha):
+// null is allowed here, the callers decide whether it is required.
+bool word_ok(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 int check_device() {
   int dev = -1;
@@ -157,6 +160,7 @@ int bsa_interval_runs(bsa_shape s, const int32_t* kept_idx, const int32_t* kept_
   if (!kept_idx || !kept_cnt || !n_runs) return BSA_EINVAL;
   if (!aligned16(kept_idx) || !aligned16(kept_cnt) || !aligned16(n_runs) || (hist && !aligned16(hist)))
     return BSA_EINVAL;
+  if (!word_ok(status)) return BSA_EINVAL;
   if (int r = check_block_shape(s)) return r;
   if (int r = check_device()) return r;
   return from_cuda(bsa::launch_interval_encode(s, kept_idx, kept_cnt, 0, nullptr, nullptr, n_runs, hist, status,
@@ -189,7 +193,7 @@ int bsa_kept_to_intervals(bsa_shape s, const int32_t* kept_idx, const int32_t* k
                           int32_t* n_int, int32_t* n_runs, int32_t* status, bsa_stream stream) {
   if (!kept_idx || !kept_cnt || !intervals || !n_int) return BSA_EINVAL;
   if (!aligned16(kept_idx) || !aligned16(kept_cnt) || !aligned16(intervals) || !aligned16(n_int) ||
-      (n_runs && !aligned16(n_runs)))
+      (n_runs && !aligned16(n_runs)) || !word_ok(status))
     return BSA_EINVAL;
   if (int r = check_block_shape(s)) return r;
   if (W < 1 || W > n_blocks(s.L, s.blk)) return BSA_EINVAL;
@@ -202,7 +206,7 @@ int bsa_intervals_to_kept(bsa_shape s, const int32_t* intervals, const int32_t* 
                           int32_t* kept_idx, int32_t* kept_cnt, int32_t* status, bsa_stream stream) {
   if (!intervals || !n_int || !kept_idx || !kept_cnt) return BSA_EINVAL;
   if (!aligned16(intervals) || !aligned16(n_int) || !aligned16(kept_idx) || !aligned16(kept_cnt) ||
-      (mask && !aligned16(mask)))
+      (mask && !aligned16(mask)) || !word_ok(status))
     return BSA_EINVAL;
   if (int r = check_block_shape(s)) return r;
   if (W < 1 || W > n_blocks(s.L, s.blk)) return BSA_EINVAL;
@@ -258,6 +262,7 @@ int bsa_sparse_attn_fwd_scatter(bsa_shape s, const bsa_bf16* q, const bsa_bf16* 
   if ((kept_idx && !aligned16(kept_idx)) || (kept_cnt && !aligned16(kept_cnt)) || (R && !aligned16(R)))
     return BSA_EINVAL;
   if (out_rows && !aligned16(out_rows)) return BSA_EINVAL;
+  if (!word_ok(status) || !word_ok(alpha)) return BSA_EINVAL;
   if (int r = check_block_shape(s)) return r;
   if (out_rows && s.blk != 128) return BSA_ESHAPE;
   if (int r = check_device()) return r;
@@ -286,6 +291,7 @@ int bsa_sparse_attn_refresh(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, c
       !aligned16(o_dense) || !aligned16(lse_dense) || !aligned16(o_sparse) || !aligned16(lse_sparse))
     return BSA_EINVAL;
   if ((R && !aligned16(R)) || (kept_mass && !aligned16(kept_mass))) return BSA_EINVAL;
+  if (!word_ok(status)) return BSA_EINVAL;
   if (int r = check_block_shape(s)) return r;
   if (s.blk != 128) return BSA_ESHAPE;
   if (int r = check_device()) return r;
@@ -322,7 +328,7 @@ int bsa_refresh_refinement(bsa_shape s, const bsa_bf16* o_dense, const bsa_bf16*
 int bsa_apply_correction(bsa_shape s, const bsa_bf16* o_sparse, const bsa_bf16* R, const float* alpha, bsa_bf16* o,
                          bsa_stream stream) {
   if (!o_sparse || !R || !alpha || !o) return BSA_EINVAL;
-  if (!aligned16(o_sparse) || !aligned16(R) || !aligned16(o)) return BSA_EINVAL;
+  if (!aligned16(o_sparse) || !aligned16(R) || !aligned16(o) || !word_ok(alpha)) return BSA_EINVAL;
   if (int r = check_rows_shape(s)) return r;
   if (int r = check_device()) return r;
   return from_cuda(bsa::launch_correct(s, reinterpret_cast<const __nv_bfloat16*>(o_sparse),

@@ -16,7 +16,9 @@
  *     [B, H, L, D] (bsa_bf16 = raw bfloat16 bits).  NB = ceil(L / blk) blocks
  *     per sequence; the last block holds L - (NB-1)*blk tokens.
  *   - Every pointer argument is a DEVICE pointer unless its comment says
- *     "host".  Device pointers must be 16-byte aligned.  The caller owns and
+ *     "host".  Device pointers must be 16-byte aligned, except the optional
+ *     device `status` word and the per-head `alpha` array, which need 4-byte
+ *     alignment.  The caller owns and
  *     allocates every buffer (inputs, outputs, workspaces); the library never
  *     allocates, frees or synchronises.
  *   - Every call is asynchronous on `stream` (NULL = legacy default stream)

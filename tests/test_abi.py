@@ -219,3 +219,22 @@ def test_interval_width_host_function_matches_oracle(lib):
         assert _width(lib, [1, 2, 3], q)[0] == _lib.BSA_EINVAL
     w = ctypes.c_int(0)
     assert lib.bsa_interval_width_for_merge(None, 3, 1.0, ctypes.byref(w)) == _lib.BSA_EINVAL
+
+
+def test_status_and_alpha_need_word_alignment(lib):
+    s = Shape(1, 2, 1000, 128, 128)
+    odd = ctypes.c_void_p((1 << 20) + 2)      # not 4-byte aligned
+    qkv = (FAKE, FAKE, FAKE)
+    # status of the attention calls
+    assert lib.bsa_sparse_attn_fwd(s, *qkv, NULL, NULL, NULL, NULL, FAKE, FAKE, odd, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd_scatter(s, *qkv, NULL, NULL, NULL, NULL, NULL, FAKE, FAKE, odd,
+                                           NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_refresh(s, *qkv, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, NULL, odd,
+                                       NULL) == _lib.BSA_EINVAL
+    # alpha of the fused and the standalone correction
+    assert lib.bsa_sparse_attn_fwd(s, *qkv, NULL, NULL, FAKE, odd, FAKE, FAKE, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_apply_correction(Shape(1, 2, 10, 16, 0), FAKE, FAKE, odd, FAKE, NULL) == _lib.BSA_EINVAL
+    # status of the interval calls
+    assert lib.bsa_interval_runs(s, FAKE, FAKE, FAKE, NULL, odd, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_kept_to_intervals(s, FAKE, FAKE, 3, FAKE, FAKE, NULL, odd, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_intervals_to_kept(s, FAKE, FAKE, 3, NULL, FAKE, FAKE, odd, NULL) == _lib.BSA_EINVAL
