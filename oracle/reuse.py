@@ -3,7 +3,7 @@
 Sources:
 * head-wise adaptive top-p abstract: Temporal Mask Reuse skips mask
   prediction when the queries and keys have drifted little since the mask was
-  predicted ("based on query-key drift").
+  predicted, judged by how far queries and keys have drifted.
 * GSRS abstract: blocks selected early keep carrying most of the attention
   weight later, so later top-p searches are restricted to the early candidate
   set.

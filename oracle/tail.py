@@ -7,8 +7,8 @@ Efficient Video Diffusion", section 3.2:
   keys and values (initial estimates of value and normalisation mass);
 * the log-mass is refined by key variance through a second-order
   approximation (COBS), the value by a pooled value-key covariance through a
-  first-order compensation (PISA; related work: "block means and shared
-  first-order value compensation");
+  first-order compensation (PISA, which the related-work section describes as
+  block means plus a first-order value term common to all blocks);
 * the log of the summed block masses is the coarse log-mass lbar_T, the block
   values weighted by their normalised masses give the coarse output obar_T;
   both are recomputed at every sparse evaluation;
@@ -22,11 +22,11 @@ query q (one token of query block i), a = q / sqrt(D), K(i) the kept blocks
 and T(i) the omitted ones; per key block j with n_j tokens (the last block
 its own count):
   kbar_j   mean key;  s2_j  per-dimension key variance (population, the
-           block's own tokens)                     -- "key variance"
+           block's own tokens)                     -- the key variance
   vbar_j   mean value
   C        pooled within-block value-key covariance of the head,
            C[e, d] = (1/L) sum_j sum_{c in j} (v_c - vbar_j)[e] (k_c - kbar_j)[d]
-                                                   -- "pooled", "shared"
+                                                   -- pooled over the blocks
   coarse block log-mass  log n_j + a . kbar_j + 1/2 sum_d a_d^2 s2_j[d]
            (the second-order cumulant expansion of log mean_c exp(a . k_c);
            exact for Gaussian keys with diagonal covariance)
