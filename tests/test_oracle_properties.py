@@ -1,0 +1,91 @@
+"""Property-based checks of the oracle (CPU): random inputs drawn by
+hypothesis, each checked against what the definitions imply -- top-p
+selection is the shortest ordered prefix reaching the target, interval
+encoding decodes back and merging adds the fewest blocks, the drift does not
+depend on the scale of the means, and a refinement taken at the same step
+turns the coarse tail into the exact one."""
+
+import itertools
+
+import numpy as np
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+
+from oracle import attention as oatt
+from oracle import intervals as oint
+from oracle import reuse as oreu
+from oracle import tail as otail
+from oracle import topp as otop
+
+SETTINGS = settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+
+
+@SETTINGS
+@given(st.lists(st.floats(0.0, 1.0, width=32), min_size=1, max_size=40),
+       st.floats(0.0078125, 1.0, width=32))
+def test_topp_is_the_shortest_ordered_prefix(row, p):
+    P = np.asarray(row, np.float32)
+    kept, k = otop.select_row(P, np.float32(p))
+    assert k == len(kept) >= 1 and list(kept) == sorted(kept)
+    if np.float32(p) == 1:
+        assert k == P.size
+        return
+    u = otop.fixed_point_mass(otop.clamp_probs(P))
+    T = int(np.ceil(np.float64(np.float32(p)) * np.float64(int(u.sum()))))
+    order = sorted(range(P.size), key=lambda j: (-float(otop.clamp_probs(P)[j]), j))
+    assert sorted(order[:k]) == list(kept)              # a prefix of the order
+    if T > 0:
+        assert int(u[kept].sum()) >= T                   # reaches the target
+        assert int(u[order[:k - 1]].sum()) < T           # one block fewer does not
+
+
+@SETTINGS
+@given(st.integers(1, 48).flatmap(lambda nb: st.tuples(st.just(nb), st.sets(st.integers(0, nb - 1)),
+                                                       st.integers(1, nb))))
+def test_intervals_round_trip_and_fewest_added_blocks(args):
+    nb, kept_set, W = args
+    kept = sorted(kept_set)
+    runs = oint.runs_of(kept)
+    assert len(runs) <= oint.max_intervals(nb)
+    merged = oint.merge_runs(runs, W)
+    assert len(merged) == min(len(runs), W)
+    dec = oint.decode_row(merged)
+    assert set(kept) <= set(dec) and dec == sorted(set(dec))
+    if len(runs) <= W:
+        assert dec == kept
+    gaps = sorted(runs[r + 1][0] - runs[r][1] for r in range(len(runs) - 1))
+    assert len(dec) - len(kept) == sum(gaps[:max(0, len(runs) - W)])   # the smallest gaps are filled
+
+
+@SETTINGS
+@given(st.integers(0, 2 ** 31 - 1), st.floats(0.01, 100.0))
+def test_drift_does_not_depend_on_the_scale_of_the_means(seed, c):
+    rng = np.random.default_rng(seed)
+    ref_q, ref_k = rng.standard_normal((1, 2, 5, 8)), rng.standard_normal((1, 2, 5, 8))
+    q = ref_q + 0.1 * rng.standard_normal(ref_q.shape)
+    k = ref_k + 0.2 * rng.standard_normal(ref_k.shape)
+    d1 = oreu.block_drift(ref_q, ref_k, q, k)
+    d2 = oreu.block_drift(c * ref_q, c * ref_k, c * q, c * k)
+    assert np.allclose(d1, d2, rtol=1e-9, atol=0)
+
+
+@settings(max_examples=15, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(st.integers(0, 2 ** 31 - 1), st.integers(1, 5), st.integers(0, 15))
+def test_same_step_refinement_makes_the_tail_exact(seed, nblocks, ragged):
+    rng = np.random.default_rng(seed)
+    blk, D = 8, 4
+    L = nblocks * blk + ragged
+    NB = (L + blk - 1) // blk
+    q, k, v = (rng.standard_normal((1, 1, L, D)) for _ in range(3))
+    idx = np.full((1, 1, NB, NB), -1, np.int32)
+    cnt = np.zeros((1, 1, NB), np.int32)
+    for i in range(NB):
+        sel = np.flatnonzero(rng.random(NB) < 0.5)
+        idx[0, 0, i, :sel.size] = sel
+        cnt[0, 0, i] = sel.size
+    O_S, l_S = oatt.masked_attention(q, k, v, idx, cnt, blk)
+    lbar, obar = otail.coarse_tail(q, otail.block_stats(k, v, blk), idx, cnt, blk)
+    l_T, o_T = otail.exact_tail(q, k, v, idx, cnt, blk)
+    O, lse = otail.reconstruct(l_S, O_S, lbar, obar, *otail.refinement(l_T, o_T, lbar, obar))
+    O_d, l_d = oatt.dense_attention(q, k, v)
+    assert np.allclose(O, O_d, atol=1e-10) and np.allclose(lse, l_d, rtol=1e-12, atol=1e-12)
