@@ -89,3 +89,38 @@ def test_same_step_refinement_makes_the_tail_exact(seed, nblocks, ragged):
     O, lse = otail.reconstruct(l_S, O_S, lbar, obar, *otail.refinement(l_T, o_T, lbar, obar))
     O_d, l_d = oatt.dense_attention(q, k, v)
     assert np.allclose(O, O_d, atol=1e-10) and np.allclose(lse, l_d, rtol=1e-12, atol=1e-12)
+
+
+@SETTINGS
+@given(st.integers(1, 12), st.integers(1, 12), st.integers(1, 12))
+def test_hilbert_order_is_a_bijection_on_any_grid(T, Hh, W):
+    from oracle import hilbert as ohil
+    perm, inv = ohil.hilbert_perm(T, Hh, W)
+    L = T * Hh * W
+    assert sorted(perm.tolist()) == list(range(L))
+    assert np.array_equal(perm[inv], np.arange(L)) and np.array_equal(inv[perm], np.arange(L))
+    x = np.arange(L * 2, dtype=np.float64).reshape(1, L, 2)
+    assert np.array_equal(ohil.permute_rows(ohil.permute_rows(x, perm), perm, inverse=True), x)
+
+
+@settings(max_examples=15, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(st.integers(0, 2 ** 31 - 1), st.integers(1, 4), st.integers(0, 7))
+def test_refresh_kept_share_is_a_mixture_weight(seed, nblocks, ragged):
+    from oracle import refresh as oref
+    rng = np.random.default_rng(seed)
+    blk, D = 8, 4
+    L = nblocks * blk + ragged
+    NB = (L + blk - 1) // blk
+    q, k, v = (rng.standard_normal((1, 1, L, D)) for _ in range(3))
+    idx = np.full((1, 1, NB, NB), -1, np.int32)
+    cnt = np.zeros((1, 1, NB), np.int32)
+    for i in range(NB):
+        sel = np.flatnonzero(rng.random(NB) < 0.5)
+        idx[0, 0, i, :sel.size] = sel
+        cnt[0, 0, i] = sel.size
+    Od, Ld, Os, Ls, R, mass = oref.fused_refresh(q, k, v, idx, cnt, blk)
+    assert np.all((mass >= 0) & (mass <= 1 + 1e-12))
+    ci, cc = oref.complement_lists(idx, cnt, NB)
+    Oc, Lc = oatt.masked_attention(q, k, v, ci, cc, blk)
+    mix = mass[..., None] * np.nan_to_num(Os) + (1 - mass)[..., None] * np.nan_to_num(Oc)
+    assert np.allclose(mix, Od, atol=1e-10)
