@@ -15,6 +15,7 @@ EXPORTS = (
     "bsa_block_drift",
     "bsa_select_topp_mask", "bsa_select_topp_mask_restricted",
     "bsa_interval_runs", "bsa_interval_width_for_merge", "bsa_kept_to_intervals", "bsa_intervals_to_kept",
+    "bsa_wait_selftest",
     "bsa_reorder_workspace_bytes", "bsa_reorder_tokens", "bsa_reorder_tokens_noalloc", "bsa_permute_tokens",
     "bsa_sparse_attn_fwd", "bsa_sparse_attn_fwd_scatter", "bsa_sparse_attn_refresh", "bsa_refresh_refinement", "bsa_apply_correction",
 )
@@ -65,6 +66,7 @@ def load():
                                               ctypes.POINTER(ctypes.c_int)]),
         "bsa_kept_to_intervals": (_I, [Shape, _P, _P, _I, _P, _P, _P, _P, _P]),
         "bsa_intervals_to_kept": (_I, [Shape, _P, _P, _I, _P, _P, _P, _P, _P]),
+        "bsa_wait_selftest": (_I, [_P, ctypes.c_ulonglong, _P]),
         "bsa_reorder_workspace_bytes": (_SZ, [_I, _I, _I]),
         "bsa_reorder_tokens": (_I, [_I, _I, _I, _P, _P, _P, _SZ, _P]),
         "bsa_reorder_tokens_noalloc": (_I, [_I, _I, _I, _P, _P, _P]),

@@ -215,6 +215,13 @@ int bsa_intervals_to_kept(bsa_shape s, const int32_t* intervals, const int32_t* 
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int bsa_wait_selftest(int32_t* status, unsigned long long limit_ns, bsa_stream stream) {
+  if (!status || !word_ok(status)) return BSA_EINVAL;
+  if (limit_ns == 0 || limit_ns > 2000000000ull) return BSA_EINVAL;
+  if (int r = check_device()) return r;
+  return from_cuda(bsa::launch_wait_selftest(status, limit_ns, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t bsa_reorder_workspace_bytes(int T, int Hh, int W) { return bsa::hilbert_workspace_bytes(T, Hh, W); }
 
 int bsa_reorder_tokens(int T, int Hh, int W, int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes,

@@ -43,6 +43,8 @@ cudaError_t launch_interval_encode(const bsa_shape& s, const int32_t* kept_idx, 
 cudaError_t launch_interval_decode(const bsa_shape& s, const int32_t* intervals, const int32_t* n_int, int W,
                                    uint8_t* mask, int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
                                    cudaStream_t st);
+// one thread waits on an mbarrier nothing arrives at, for limit_ns
+cudaError_t launch_wait_selftest(int32_t* status, unsigned long long limit_ns, cudaStream_t st);
 size_t hilbert_workspace_bytes(int T, int Hh, int W);
 cudaError_t launch_hilbert(int T, int Hh, int W, int32_t* perm, int32_t* inv, void* ws, cudaStream_t st);
 cudaError_t launch_permute(const bsa_shape& s, const __nv_bfloat16* x, const int32_t* perm, __nv_bfloat16* y,

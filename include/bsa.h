@@ -299,6 +299,15 @@ BSA_API int bsa_intervals_to_kept(bsa_shape s, const int32_t* intervals, const i
                                   int32_t* kept_idx, int32_t* kept_cnt, int32_t* status, bsa_stream stream);
 
 /*
+ * bsa_wait_selftest -- exercises the bounded wait that every pipeline wait of
+ * the library uses: one thread waits on an mbarrier that nothing arrives at,
+ * gives up after limit_ns (1 ns .. 2 s) of the GPU's global timer, ORs
+ * BSA_DEV_TIMEOUT into *status (device int32, 4-byte aligned) and returns;
+ * the context stays usable.
+ */
+BSA_API int bsa_wait_selftest(int32_t* status, unsigned long long limit_ns, bsa_stream stream);
+
+/*
  * bsa_sparse_attn_fwd -- block-sparse attention forward with an optional
  * fused correction epilogue.
  * Defines: computing the selected connections densely and skipping the

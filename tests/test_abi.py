@@ -238,3 +238,10 @@ def test_status_and_alpha_need_word_alignment(lib):
     assert lib.bsa_interval_runs(s, FAKE, FAKE, FAKE, NULL, odd, NULL) == _lib.BSA_EINVAL
     assert lib.bsa_kept_to_intervals(s, FAKE, FAKE, 3, FAKE, FAKE, NULL, odd, NULL) == _lib.BSA_EINVAL
     assert lib.bsa_intervals_to_kept(s, FAKE, FAKE, 3, NULL, FAKE, FAKE, odd, NULL) == _lib.BSA_EINVAL
+
+
+def test_wait_selftest_validation(lib):
+    assert lib.bsa_wait_selftest(NULL, 1000, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_wait_selftest(ctypes.c_void_p((1 << 20) + 2), 1000, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_wait_selftest(FAKE, 0, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_wait_selftest(FAKE, 3_000_000_000, NULL) == _lib.BSA_EINVAL
