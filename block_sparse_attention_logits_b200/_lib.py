@@ -23,6 +23,7 @@ EXPORTS = (
 BSA_OK, BSA_EINVAL, BSA_ESHAPE, BSA_ENODEV, BSA_ECUDA, BSA_EWORKSPACE = range(6)
 BSA_DEV_TIMEOUT = 1
 BSA_DEV_BAD_INDEX = 2
+BSA_DEV_SCHED_CONFLICT = 4
 
 
 class Shape(ctypes.Structure):

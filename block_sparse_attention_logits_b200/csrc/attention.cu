@@ -636,13 +636,8 @@ bool make_map(CUtensorMap* m, const void* base, int D, int L, int BH, int box_ro
 template <int D, int BN>
 int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   using C = Cfg<D, BN>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(sparse_attn_kernel<D, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
-      return BSA_ECUDA;
-    configured = true;
-  }
+  if (smem_opt_in(reinterpret_cast<const void*>(sparse_attn_kernel<D, BN>), C::SMEM_BYTES) != cudaSuccess)
+    return BSA_ECUDA;
   const int BH = s.B * s.H;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, a.q, D, s.L, BH, BM) || !make_map(&mk, a.k, D, s.L, BH, BN) ||

@@ -90,15 +90,25 @@ constexpr int kRegsSoftmax = 168;   // two warpgroups
 constexpr int kRegsEpilogue = 120;
 static_assert(128 * kRegsCtl + 256 * kRegsSoftmax + 128 * kRegsEpilogue <= 512 * 128, "register split exceeds launch");
 
-// Work counters, one per launch in flight (round robin).  Zero at module
-// load; every launch leaves its slot at zero again.
-constexpr int kSchedSlots = 64;
+// Work counters.  Each launch draws its work items from one slot of a ring,
+// the host assigning slots round robin, one per launch.  A slot is owned by
+// one launch from its first CTA to its last: the state word holds the owner's
+// tag (from %gridid, so two replays of one captured graph differ), how many of
+// its CTAs joined and how many have left.  The last CTA to leave returns the
+// counter to zero and frees the slot, so a launch needs no memset and the call
+// allocates nothing.  A CTA that finds its slot owned by another launch (more
+// than kSchedSlots launches executing at once, or one captured graph replayed
+// on two streams at the same time) does no work and flags
+// BSA_DEV_SCHED_CONFLICT; the slot stays consistent for later launches.
+constexpr int kSchedSlots = 256;
 struct SchedSlot {
-  unsigned int next;
-  unsigned int done;
-  unsigned int pad[30];
+  unsigned long long state;  // tag << 32 | joined << 16 | left; 0 = free
+  unsigned int next;         // next work item; 0 whenever the slot is free
+  unsigned int last_tag;     // tag of the last launch that freed the slot
+  unsigned int pad[28];
 };
 __device__ SchedSlot g_sched[kSchedSlots];
+constexpr int kCasTries = 1 << 16;
 
 struct Params {
   const int32_t* kept_idx;
@@ -151,11 +161,69 @@ struct Shared {
   int items[kQueue];
   uint32_t tmem_base;
   volatile int abort_flag;
+  int joined;  // this CTA fetches work from its scheduler slot
 };
 static_assert(sizeof(Shared) <= 512, "misc region too small");
 
 __device__ __forceinline__ void flag_status(const Params& prm, int bits) {
   if (prm.status) atomicOr(prm.status, bits);
+}
+
+__device__ __forceinline__ uint32_t launch_tag() {
+  uint64_t g;
+  asm volatile("mov.u64 %0, %%gridid;" : "=l"(g));
+  return (static_cast<uint32_t>(g) << 1) | 1u;  // never 0 (0 marks a free slot)
+}
+
+// Joins this CTA to its launch's use of the slot; false: fetch no work (the
+// slot belongs to another launch, or this launch has already finished).
+__device__ bool sched_join(SchedSlot* s, uint32_t tag, const Params& prm) {
+  unsigned long long cur = atomicAdd(&s->state, 0ull);
+  for (int t = 0; t < kCasTries; ++t) {
+    const uint32_t owner = static_cast<uint32_t>(cur >> 32);
+    const uint32_t joined = static_cast<uint32_t>(cur >> 16) & 0xffffu, left = static_cast<uint32_t>(cur) & 0xffffu;
+    unsigned long long want;
+    if (owner == 0) {
+      if (atomicAdd(&s->last_tag, 0u) == tag) return false;  // this launch already finished
+      want = (static_cast<unsigned long long>(tag) << 32) | (1ull << 16);
+    } else if (owner == tag) {
+      if (joined != 0 && left == joined) return false;  // finishing: nothing left to fetch
+      want = cur + (1ull << 16);
+    } else {
+      flag_status(prm, BSA_DEV_SCHED_CONFLICT);
+      return false;
+    }
+    const unsigned long long got = atomicCAS(&s->state, cur, want);
+    if (got == cur) {
+      __threadfence();
+      return true;
+    }
+    cur = got;
+  }
+  flag_status(prm, BSA_DEV_SCHED_CONFLICT);
+  return false;
+}
+
+// Leaves the slot after this CTA's last fetch; the last CTA to leave resets
+// the counter and frees the slot.
+__device__ void sched_leave(SchedSlot* s, uint32_t tag, const Params& prm) {
+  __threadfence();
+  unsigned long long cur = atomicAdd(&s->state, 0ull);
+  for (int t = 0; t < kCasTries; ++t) {
+    const unsigned long long want = cur + 1ull;
+    const unsigned long long got = atomicCAS(&s->state, cur, want);
+    if (got == cur) {
+      if ((static_cast<uint32_t>(want >> 16) & 0xffffu) == (static_cast<uint32_t>(want) & 0xffffu)) {
+        atomicExch(&s->next, 0u);
+        atomicExch(&s->last_tag, tag);
+        __threadfence();
+        atomicExch(&s->state, 0ull);
+      }
+      return;
+    }
+    cur = got;
+  }
+  flag_status(prm, BSA_DEV_SCHED_CONFLICT);
 }
 
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Shared* sh, const Params& prm) {
@@ -299,6 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh->drain[j], 1);
     }
     sh->abort_flag = 0;
+    sh->joined = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -320,6 +389,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
       // ---------------------------------- item queue, TMA: Q and the K ring
       SchedSlot* sched = &g_sched[prm.sched_slot];
+      const uint32_t tag = launch_tag();
+      int joined = 0;
+      if (lane == 0) {
+        joined = sched_join(sched, tag, prm) ? 1 : 0;
+        sh->joined = joined;
+      }
+      joined = __shfl_sync(0xffffffffu, joined, 0);
       int u = 0;
       bool ok = true;
       for (int i = 0;; ++i) {
@@ -327,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i >= kQueue && !(ok = warp_wait(&sh->item_empty[qs], ((i / kQueue) - 1) & 1, sh, prm))) break;
         int w = 0;
         if (lane == 0) {
-          w = static_cast<int>(atomicAdd(&sched->next, 1u));
+          w = joined ? static_cast<int>(atomicAdd(&sched->next, 1u)) : -1;
           if (w >= prm.n_work) w = -1;
           sh->items[qs] = w;
           mbar_arrive(&sh->item_full[qs]);
@@ -810,16 +886,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (threadIdx.x == 0) {
-    // the last CTA of the launch leaves the work counter at zero for reuse;
-    // every CTA has made its final fetch before it counts itself done
-    SchedSlot* sched = &g_sched[prm.sched_slot];
-    __threadfence();
-    if (atomicAdd(&sched->done, 1u) == gridDim.x - 1) {
-      atomicExch(&sched->next, 0u);
-      atomicExch(&sched->done, 0u);
-      __threadfence();
-    }
+  if (threadIdx.x == 0 && sh->joined) {
+    // this CTA has made its final fetch (or given up): leave the slot
+    sched_leave(&g_sched[prm.sched_slot], launch_tag(), prm);
   }
 }
 
@@ -854,26 +923,11 @@ bool make_map(CUtensorMap* m, const void* base, int D, int L, int BH, int box_ro
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  }
-  return n;
-}
-
 template <int D, bool kFused>
 int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   using C = Cfg<D>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(sparse_attn_tile_kernel<D, kFused>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
-      return BSA_ECUDA;
-    configured = true;
-  }
+  if (smem_opt_in(reinterpret_cast<const void*>(sparse_attn_tile_kernel<D, kFused>), C::SMEM_BYTES) != cudaSuccess)
+    return BSA_ECUDA;
   const int BH = s.B * s.H;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, a.q, D, s.L, BH, BM) || !make_map(&mk, a.k, D, s.L, BH, BN) ||
@@ -901,7 +955,8 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   prm.dense = a.kept_idx == nullptr;
   static std::atomic<unsigned int> launches{0};
   prm.sched_slot = static_cast<int>(launches.fetch_add(1u) % kSchedSlots);
-  const int grid = prm.n_work < num_sms() ? prm.n_work : num_sms();
+  const int sms = sm_count();
+  const int grid = prm.n_work < sms ? prm.n_work : sms;
   sparse_attn_tile_kernel<D, kFused><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ECUDA;
 }

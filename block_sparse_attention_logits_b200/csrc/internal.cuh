@@ -19,6 +19,15 @@ struct TopP {
 
 inline int n_blocks(int L, int blk) { return (L + blk - 1) / blk; }
 
+// Per-device host state (host_state.cu), valid for the context it was made in:
+// raise a kernel's dynamic shared-memory limit to `bytes` on the current device
+// (no-op up to 48 KB, once per kernel and context); the current device's SM
+// count; the current device's address of one of the library's __device__
+// arrays (BSA_OK, BSA_ENODEV or BSA_ECUDA).
+cudaError_t smem_opt_in(const void* func, size_t bytes);
+int sm_count();
+int symbol_address(const void* symbol, void** out);
+
 // launchers (return cudaSuccess or the launch error)
 // perm (nullable): gather form -- token t is input row perm[t]; the gathered
 // rows are also written to q_out / k_out

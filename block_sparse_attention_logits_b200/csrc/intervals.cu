@@ -237,16 +237,6 @@ __global__ void __launch_bounds__(256) interval_decode_kernel(const int32_t* __r
   if (lane == 0) kept_cnt[row] = total;
 }
 
-template <typename Kern>
-cudaError_t smem_opt_in(Kern k, size_t smem, size_t& configured) {
-  if (smem > 48 * 1024 && smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured = smem;
-  }
-  return cudaSuccess;
-}
-
 }  // namespace
 
 int max_intervals(int NB) { return (NB + 1) / 2; }
@@ -265,8 +255,7 @@ cudaError_t launch_interval_encode(const bsa_shape& s, const int32_t* kept_idx, 
     return cudaGetLastError();
   }
   const size_t smem = static_cast<size_t>(warps) * 2 * cap * sizeof(int32_t);
-  static size_t configured = 0;
-  if (cudaError_t e = smem_opt_in(interval_encode_kernel<true>, smem, configured)) return e;
+  if (cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(interval_encode_kernel<true>), smem)) return e;
   interval_encode_kernel<true><<<static_cast<unsigned>(grid), warps * 32, smem, st>>>(
       kept_idx, kept_cnt, NB, rows, W, cap, intervals, n_int, n_runs, nullptr, status);
   return cudaGetLastError();

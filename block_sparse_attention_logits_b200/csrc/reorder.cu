@@ -10,7 +10,6 @@
 // Ranks come from a two-pass stream compaction over chunks of the index
 // range: pass 1 counts grid points per chunk into the caller's workspace,
 // pass 2 adds up the counts of the preceding chunks and writes perm / inv.
-#include <mutex>
 
 #include "internal.cuh"
 
@@ -239,28 +238,6 @@ cudaError_t launch_permute(const bsa_shape& s, const __nv_bfloat16* x, const int
 constexpr int kNoAllocChunks = 4096;
 static __device__ __align__(256) int g_reorder_counts[kNoAllocChunks];
 
-namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_counts_mu;
-void* g_counts_addr[kMaxDevices] = {};
-
-// Device address of g_reorder_counts on the current device, looked up once per
-// device (the first call on a device does it; make that call before any stream
-// capture).  In host code the array's name is only a host-side stand-in.
-int counts_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ENODEV;
-  std::lock_guard<std::mutex> lock(g_counts_mu);
-  if (g_counts_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_reorder_counts) != cudaSuccess || p == nullptr) return BSA_ECUDA;
-    g_counts_addr[dev] = p;
-  }
-  *out = g_counts_addr[dev];
-  return BSA_OK;
-}
-}  // namespace
-
 }  // namespace bsa
 
 extern "C" int bsa_reorder_tokens_noalloc(int T, int Hh, int W, int32_t* perm, int32_t* inv, bsa_stream stream) {
@@ -272,8 +249,12 @@ extern "C" int bsa_reorder_tokens_noalloc(int T, int Hh, int W, int32_t* perm, i
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10)
     return BSA_ENODEV;
+  // Device address of g_reorder_counts on the current device: in host code
+  // the array's name is only a host-side stand-in.  Looked up by the first
+  // call on each device (make that call before any stream capture) and again
+  // whenever the device's context has changed (after cudaDeviceReset).
   void* counts = nullptr;
-  if (int r = bsa::counts_address(&counts)) return r;
+  if (int r = bsa::symbol_address(reinterpret_cast<const void*>(&bsa::g_reorder_counts), &counts)) return r;
   return bsa::launch_hilbert(T, Hh, W, perm, inv, counts, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? BSA_OK
              : BSA_ECUDA;

@@ -215,17 +215,11 @@ cudaError_t launch_block_softmax(const bsa_shape& s, const float* qp, const floa
   const int NB = n_blocks(s.L, s.blk);
   dim3 grid((NB + kTile - 1) / kTile, s.B * s.H);
   const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(s.D)));
-  static bool configured = false;
-  if (!configured) {
-    // 69.6 KB of transposed tiles at D = 128: above the default 48 KB
-    cudaError_t e = cudaFuncSetAttribute(block_softmax_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         2 * 128 * kPad * 4);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(block_softmax_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               2 * 64 * kPad * 4);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // 69.6 KB of transposed tiles at D = 128: above the default 48 KB
+  if (cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(block_softmax_kernel<128>), 2 * 128 * kPad * 4))
+    return e;
+  if (cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(block_softmax_kernel<64>), 2 * 64 * kPad * 4))
+    return e;
   if (s.D == 128)
     block_softmax_kernel<128><<<grid, 256, 2 * 128 * kPad * 4, st>>>(qp, kp, probs, cand, NB, scale);
   else

@@ -317,13 +317,7 @@ cudaError_t launch_select(const bsa_shape& s, const float* probs, const TopP& p,
   if (warps > 8) warps = 8;
   if (warps < 1) warps = 1;
   const size_t smem = per_warp * warps;
-  static size_t configured = 0;
-  if (smem > 48 * 1024 && smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured = smem;
-  }
+  if (cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(select_kernel), smem)) return e;
   const long long grid = (rows + warps - 1) / warps;
   select_kernel<<<static_cast<unsigned>(grid), warps * 32, smem, st>>>(probs, p, cand, mask, idx, cnt, s.H, NB, rows,
                                                                        nbp);

@@ -1,0 +1,74 @@
+"""One pass of the hot path over one batch, as the benchmark times it.
+
+The pass (DFSAttn abstract: Hilbert reorder, block scoring; head-wise top-p
+and GSRS abstracts: cumulative top-p selection per query block; CalibAtt
+Fig. 5(b): attention over the kept blocks only; RECAP section 1: the cached
+refinement scaled per head):
+
+  with a latent grid (Hilbert order):
+    score_blocks_gather  Q, K gathered into curve order inside the pooling pass
+    permute_tokens       V gathered into curve order
+    select_topp_mask     kept lists from the GPU's own block scores
+    sparse_attn_fwd      attention with the fused O + alpha*R epilogue, writing
+                         O and LSE straight back to grid order (row map = perm)
+  without one:
+    score_blocks -> select_topp_mask -> sparse_attn_fwd (+ alpha*R)
+
+Every call is one of this library's C calls (api.py); nothing here computes.
+`run_step` works on a dict of caller-owned buffers, so a head chunk of a
+larger job can run the same pass on slices of the full buffers.
+"""
+
+import torch
+
+from . import api
+
+
+def alloc_buffers(B, H, L, D, blk, device):
+    """Device buffers of one pass: curve-order copies, scores, lists, outputs."""
+    nb = api.n_blocks(L, blk)
+    dev = torch.device(device)
+    bf = dict(dtype=torch.bfloat16, device=dev)
+    return dict(
+        qh=torch.empty((B, H, L, D), **bf), kh=torch.empty((B, H, L, D), **bf), vh=torch.empty((B, H, L, D), **bf),
+        qp=torch.empty((B, H, nb, D), dtype=torch.float32, device=dev),
+        kp=torch.empty((B, H, nb, D), dtype=torch.float32, device=dev),
+        probs=torch.empty((B, H, nb, nb), dtype=torch.float32, device=dev),
+        mask=torch.empty((B, H, nb, nb), dtype=torch.uint8, device=dev),
+        idx=torch.empty((B, H, nb, nb), dtype=torch.int32, device=dev),
+        cnt=torch.empty((B, H, nb), dtype=torch.int32, device=dev),
+        oh=torch.empty((B, H, L, D), **bf),
+        o=torch.empty((B, H, L, D), **bf),
+        lse=torch.empty((B, H, L), dtype=torch.float32, device=dev),
+    )
+
+
+def run_step(b, q, k, v, blk, p, perm=None, R=None, alpha=None, status=None, events=None):
+    """One pass on buffers `b` (from alloc_buffers, or slices of them).
+
+    q, k, v: bf16 [B,H,L,D] in grid order.  perm: the Hilbert order (int32
+    [L], from api.reorder_tokens) or None for no reorder.  p: top-p, one float
+    or one per head.  R (bf16 [B,H,L,D], in the order the attention reads:
+    curve order when perm is given) and alpha (float32 [H]) enable the fused
+    correction.  events: optional three CUDA events recorded before scoring,
+    after selection and after attention.
+    Returns (o, lse) in grid order.
+    """
+    B, H, L, D = q.shape
+    if events:
+        events[0].record()
+    if perm is not None:
+        api.score_blocks_gather(q, k, perm, blk, b["qh"], b["kh"], b["qp"], b["kp"], b["probs"])
+        api.permute_tokens(v, perm, out=b["vh"])
+        qs, ks, vs = b["qh"], b["kh"], b["vh"]
+    else:
+        qs, ks, vs = q, k, v
+        api.score_blocks(qs, ks, blk, b["qp"], b["kp"], b["probs"])
+    api.select_topp_mask(b["probs"], p, L, blk, D, b["mask"], b["idx"], b["cnt"])
+    if events:
+        events[1].record()
+    o = b["o"] if perm is not None else b["oh"]
+    api.sparse_attn_fwd(qs, ks, vs, blk, b["idx"], b["cnt"], R, alpha, o, b["lse"], status=status, out_rows=perm)
+    if events:
+        events[2].record()
+    return o, b["lse"]

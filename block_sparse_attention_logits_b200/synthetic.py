@@ -44,10 +44,12 @@ def _head_field(coords, D, fp, h):
     return (fp.amp * phi).astype(np.float32)
 
 
-def make_qkv(B, H, grid, D, fp, with_v=True, out=None):
+def make_qkv(B, H, grid, D, fp, with_v=True, out=None, h0=0):
     """Q, K (and V) as bf16 CPU tensors [B, H, L, D] in grid (row-major) order.
 
     `out` may pass preallocated bf16 tensors (e.g. pinned) to fill in place.
+    h0: index of the first head, so that heads h0 .. h0+H-1 of a larger
+    workload (one rank's head shard) get exactly that workload's values.
     """
     T, Hh, W = grid
     L = T * Hh * W
@@ -55,7 +57,8 @@ def make_qkv(B, H, grid, D, fp, with_v=True, out=None):
     names = ("q", "k", "v") if with_v else ("q", "k")
     if out is None:
         out = {n: torch.empty((B, H, L, D), dtype=torch.bfloat16) for n in names}
-    for h in range(H):
+    for hl in range(H):
+        h = h0 + hl
         field = _head_field(coords, D, fp, h)
         for b in range(B):
             rng = np.random.default_rng([fp.seed, 7919, b, h])
@@ -65,7 +68,7 @@ def make_qkv(B, H, grid, D, fp, with_v=True, out=None):
                     val = noise
                 else:
                     val = field + np.float32(fp.sigma) * noise
-                out[n][b, h].copy_(torch.from_numpy(val))
+                out[n][b, hl].copy_(torch.from_numpy(val))
     return out
 
 

@@ -62,6 +62,7 @@ typedef enum {
 /* Bits a kernel may OR into a device status word. */
 #define BSA_DEV_TIMEOUT 1   /* an internal pipeline wait exceeded its time limit */
 #define BSA_DEV_BAD_INDEX 2 /* a kept index or count was out of range and was skipped */
+#define BSA_DEV_SCHED_CONFLICT 4 /* an attention launch found its work counter in use (see below) */
 
 typedef struct {
   int B;   /* batch */
@@ -327,6 +328,15 @@ BSA_API int bsa_wait_selftest(int32_t* status, unsigned long long limit_ns, bsa_
  * status: optional device int32 that receives BSA_DEV_* bits (OR-ed; the
  * caller zeroes it); NULL to skip.  Kept indices outside [0, NB) and counts
  * outside [0, NB] are skipped/clamped and flagged, never dereferenced.
+ * Work distribution (blk = 128): the launch's CTAs draw query blocks from a
+ * work counter in a ring of 256 counters inside the library, one per launch,
+ * assigned round robin and released by the launch's last CTA, so no scratch
+ * is needed.  A launch that finds its counter still owned by another launch
+ * -- more than 256 attention launches (of this call, the scatter form and
+ * bsa_sparse_attn_refresh) executing at the same time, or one captured CUDA
+ * graph holding an attention call replayed on two streams at once -- leaves
+ * (part of) its output unwritten and sets BSA_DEV_SCHED_CONFLICT; do not
+ * replay such a graph concurrently with itself.
  * Errors: BSA_EINVAL on null/misaligned pointers or exactly one of
  * kept_idx/kept_cnt (or R/alpha) NULL; BSA_ESHAPE; BSA_ENODEV; BSA_ECUDA.
  */

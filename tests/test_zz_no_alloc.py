@@ -4,10 +4,13 @@ For callers that cannot allocate device memory (their memory belongs to a
 host framework's allocator that hands over only input/output buffers, HBM is
 already reserved, or cudaMalloc's implicit synchronisation is unacceptable),
 the library keeps the reorder's scratch in a fixed array of its own.  This
-test calls the new entry point through the C ABI, twice in a row on
+test calls the new entry point through the C ABI, several times in a row on
 different grids (the shared array keeps the previous call's contents), and
 checks each result against the workspace-taking bsa_reorder_tokens on the
-same grid: permutations are integers, so they must match bit for bit.
+same grid and against the oracle's Hilbert order: permutations are
+integers, so they must match bit for bit.  One grid, (2, 3, 200), has a
+longest side between 129 and 256, so its 2^24-cell cube uses every one of
+the array's 4096 chunk counts.
 
 This file is collected last so that a run stopping at the first failure has
 already run every other test; it also passes alone in a fresh process (the
@@ -16,10 +19,12 @@ first call on the device performs the array's address look-up).
 
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
 from block_sparse_attention_logits_b200 import _lib
+from oracle import hilbert as ohil
 
 pytestmark = pytest.mark.gpu
 
@@ -51,13 +56,17 @@ def _no_alloc(lib, grid, stream):
 def test_noalloc_reorder_matches_workspace_reorder_twice():
     lib = _lib.load()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    # a large grid first, then a smaller one that reuses (part of) the array
-    for grid in [(21, 45, 80), (3, 5, 7)]:
+    # a large grid, one that fills the whole array, then a small one that
+    # reuses part of it
+    for grid in [(21, 45, 80), (2, 3, 200), (3, 5, 7)]:
         ref_perm, ref_inv = _with_workspace(lib, grid, stream)
         perm, inv = _no_alloc(lib, grid, stream)
         torch.cuda.synchronize()
         assert torch.equal(perm, ref_perm), grid
         assert torch.equal(inv, ref_inv), grid
+        o_perm, o_inv = ohil.hilbert_perm(*grid)
+        assert np.array_equal(perm.cpu().numpy(), o_perm), grid
+        assert np.array_equal(inv.cpu().numpy(), o_inv), grid
 
 
 def test_noalloc_reorder_rejects_grids_beyond_its_limit():
