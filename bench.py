@@ -305,6 +305,39 @@ def interval_timings(idx, cnt, L, blk, D, barrier, q=0.95):
             "interval_bytes_max": rows * Wmax * 8 + rows * 4, "status": int(st.item())}
 
 
+def tail_timings(q, k, v, mask, idx, cnt, blk, barrier):
+    """The coarse tail of the omitted blocks on a step's inputs: statistics
+    (block moments and pooled covariance), the tail, the refinement at a
+    refresh (with the exact tail over the complement lists) and the
+    reconstruction; ms per call."""
+    from block_sparse_attention_logits_b200 import api
+    L = q.shape[2]
+    st = torch.zeros(1, dtype=torch.int32, device=q.device)
+    o_S, l_S = api.sparse_attn_fwd(q, k, v, blk, idx, cnt, status=st)
+    ci, cc = api.complement_lists(mask, L, blk)
+    o_T, l_T = api.sparse_attn_fwd(q, k, v, blk, ci, cc, status=st)
+    _, _, _, _, ws = api.tail_stats(k, v, blk, status=st)
+    lbar, obar = api.coarse_tail(q, mask, blk, ws, status=st)
+    d_l, d_o = api.tail_refinement(l_T, o_T, lbar, obar)
+    calls = (("stats", lambda: api.tail_stats(k, v, blk, ws=ws, status=st)),
+             ("coarse_tail", lambda: api.coarse_tail(q, mask, blk, ws, status=st)),
+             ("refinement", lambda: api.tail_refinement(l_T, o_T, lbar, obar)),
+             ("reconstruct", lambda: api.tail_reconstruct(l_S, o_S, lbar, obar, d_l, d_o)))
+    ms = {}
+    for name, fn in calls:
+        fn()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(5):
+            fn()
+        a1.record()
+        barrier()
+        ms[name + "_ms"] = round(a0.elapsed_time(a1) / 5, 4)
+    ms["status"] = int(st.item())
+    return ms
+
+
 def run_ours(args, w, world, rank, local):
     from block_sparse_attention_logits_b200 import api, _lib
     from block_sparse_attention_logits_b200 import build as bsa_build
@@ -529,6 +562,15 @@ def run_ours(args, w, world, rank, local):
         except Exception as e:  # noqa: BLE001
             intervals = {"error": f"{type(e).__name__}: {e}"}
 
+    # the coarse tail of the omitted blocks (D = 128, 128-token blocks)
+    tail = None
+    if not args.no_refresh and D == 128 and blk == 128:
+        try:
+            qs_, ks_, vs_ = (bufs["qh"], bufs["kh"], bufs["vh"]) if w.hilbert else (q, k, v)
+            tail = tail_timings(qs_, ks_, vs_, bufs["mask"], bufs["idx"], bufs["cnt"], blk, barrier)
+        except Exception as e:  # noqa: BLE001
+            tail = {"error": f"{type(e).__name__}: {e}"}
+
     # the elementwise calls (refinement at a refresh, standalone correction):
     # HBM-bound, three [B,H,L,D] bf16 streams each
     elementwise = None
@@ -639,7 +681,7 @@ def run_ours(args, w, world, rank, local):
         "stages_ms": {"gather_score_and_select": round(float(np.mean(sel_ms)), 4), "attention": round(attn_avg_ms, 4),
                       "rest": round(ms_step - attn_avg_ms - float(np.mean(sel_ms)), 4)},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "refresh": refresh, "reuse": reuse,
-        "elementwise": elementwise, "sweep": sweep, "intervals": intervals,
+        "elementwise": elementwise, "sweep": sweep, "intervals": intervals, "tail": tail,
         "gpu_launches": LAUNCHES_PER_STEP * K if w.hilbert else (LAUNCHES_PER_STEP - 1) * K,
         "clocks": clk,
     }

@@ -15,6 +15,8 @@ EXPORTS = (
     "bsa_block_drift",
     "bsa_select_topp_mask", "bsa_select_topp_mask_restricted",
     "bsa_interval_runs", "bsa_interval_width_for_merge", "bsa_kept_to_intervals", "bsa_intervals_to_kept",
+    "bsa_tail_workspace_bytes", "bsa_tail_stats", "bsa_coarse_tail", "bsa_tail_refinement", "bsa_tail_reconstruct",
+    "bsa_complement_lists",
     "bsa_wait_selftest",
     "bsa_reorder_workspace_bytes", "bsa_reorder_tokens", "bsa_reorder_tokens_noalloc", "bsa_permute_tokens",
     "bsa_sparse_attn_fwd", "bsa_sparse_attn_fwd_scatter", "bsa_sparse_attn_refresh", "bsa_refresh_refinement", "bsa_apply_correction",
@@ -68,6 +70,12 @@ def load():
         "bsa_kept_to_intervals": (_I, [Shape, _P, _P, _I, _P, _P, _P, _P, _P]),
         "bsa_intervals_to_kept": (_I, [Shape, _P, _P, _I, _P, _P, _P, _P, _P]),
         "bsa_wait_selftest": (_I, [_P, ctypes.c_ulonglong, _P]),
+        "bsa_tail_workspace_bytes": (_SZ, [Shape]),
+        "bsa_tail_stats": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
+        "bsa_coarse_tail": (_I, [Shape, _P, _P, _P, _SZ, _P, _P, _P, _P]),
+        "bsa_tail_refinement": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P]),
+        "bsa_tail_reconstruct": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "bsa_complement_lists": (_I, [Shape, _P, _P, _P, _P]),
         "bsa_reorder_workspace_bytes": (_SZ, [_I, _I, _I]),
         "bsa_reorder_tokens": (_I, [_I, _I, _I, _P, _P, _P, _SZ, _P]),
         "bsa_reorder_tokens_noalloc": (_I, [_I, _I, _I, _P, _P, _P]),

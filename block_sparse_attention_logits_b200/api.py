@@ -25,6 +25,12 @@ __all__ = [
     "interval_width_for_merge",
     "kept_to_intervals",
     "intervals_to_kept",
+    "tail_workspace_bytes",
+    "tail_stats",
+    "coarse_tail",
+    "tail_refinement",
+    "tail_reconstruct",
+    "complement_lists",
     "reorder_workspace_bytes",
     "reorder_tokens",
     "permute_tokens",
@@ -259,6 +265,92 @@ def intervals_to_kept(intervals, n_int, L, blk, D=128, mask=None, kept_idx=None,
         Shape(B, H, L, D, blk), _ptr(intervals), _ptr(n_int), int(W), _ptr(mask), _ptr(kept_idx), _ptr(kept_cnt),
         _ptr(status), _stream()))
     return mask, kept_idx, kept_cnt
+
+
+def tail_workspace_bytes(B, H, L, D, blk):
+    """Device bytes of the workspace tail_stats and coarse_tail share."""
+    return _lib.load().bsa_tail_workspace_bytes(Shape(B, H, L, D, blk))
+
+
+def tail_stats(k, v, blk, ws=None, status=None):
+    """Block moments and pooled covariance of K and V (D = 128).  Returns
+    (kbar, s2, vbar float32 [B,H,NB,D], C float32 [B,H,D,D], ws); ws holds the
+    operand tables coarse_tail reads."""
+    B, H, L, D = k.shape
+    nb = n_blocks(L, blk)
+    _need(k, torch.bfloat16, (B, H, L, D), "k")
+    _need(v, torch.bfloat16, (B, H, L, D), "v")
+    dev = k.device
+    nbytes = tail_workspace_bytes(B, H, L, D, blk)
+    if nbytes == 0:
+        raise ValueError("unsupported shape for the coarse tail (D must be 128)")
+    ws = ws if ws is not None else torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _need(ws, torch.uint8, (ws.numel(),), "ws")
+    kbar, s2, vbar = (torch.empty((B, H, nb, D), dtype=torch.float32, device=dev) for _ in range(3))
+    C = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
+    check("bsa_tail_stats", _lib.load().bsa_tail_stats(
+        Shape(B, H, L, D, blk), _ptr(k), _ptr(v), _ptr(kbar), _ptr(s2), _ptr(vbar), _ptr(C), _ptr(ws), ws.numel(),
+        _ptr(status), _stream()))
+    return kbar, s2, vbar, C, ws
+
+
+def coarse_tail(q, mask, blk, ws, status=None):
+    """(lbar float32 [B,H,L], obar bf16 [B,H,L,D]) over the blocks each query
+    block omits (mask uint8 [B,H,NB,NB], 1 = kept); ws from tail_stats."""
+    B, H, L, D = q.shape
+    nb = n_blocks(L, blk)
+    _need(q, torch.bfloat16, (B, H, L, D), "q")
+    _need(mask, torch.uint8, (B, H, nb, nb), "mask")
+    _need(ws, torch.uint8, (ws.numel(),), "ws")
+    lbar = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    obar = torch.empty_like(q)
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
+    check("bsa_coarse_tail", _lib.load().bsa_coarse_tail(
+        Shape(B, H, L, D, blk), _ptr(q), _ptr(mask), _ptr(ws), ws.numel(), _ptr(lbar), _ptr(obar), _ptr(status),
+        _stream()))
+    return lbar, obar
+
+
+def tail_refinement(l_T, o_T, lbar, obar):
+    """(d_l float32 [B,H,L], d_o bf16 [B,H,L,D]) cached at a dense refresh."""
+    B, H, L, D = o_T.shape
+    _need(l_T, torch.float32, (B, H, L), "l_T")
+    _need(o_T, torch.bfloat16, (B, H, L, D), "o_T")
+    _need(lbar, torch.float32, (B, H, L), "lbar")
+    _need(obar, torch.bfloat16, (B, H, L, D), "obar")
+    d_l, d_o = torch.empty_like(lbar), torch.empty_like(obar)
+    check("bsa_tail_refinement", _lib.load().bsa_tail_refinement(
+        Shape(B, H, L, D, 0), _ptr(l_T), _ptr(o_T), _ptr(lbar), _ptr(obar), _ptr(d_l), _ptr(d_o), _stream()))
+    return d_l, d_o
+
+
+def tail_reconstruct(l_S, o_S, lbar, obar, d_l, d_o):
+    """(o bf16 [B,H,L,D], lse float32 [B,H,L]): the sparse part merged with the
+    reconstructed tail."""
+    B, H, L, D = o_S.shape
+    for name, t in (("l_S", l_S), ("lbar", lbar), ("d_l", d_l)):
+        _need(t, torch.float32, (B, H, L), name)
+    for name, t in (("o_S", o_S), ("obar", obar), ("d_o", d_o)):
+        _need(t, torch.bfloat16, (B, H, L, D), name)
+    o, lse = torch.empty_like(o_S), torch.empty_like(l_S)
+    check("bsa_tail_reconstruct", _lib.load().bsa_tail_reconstruct(
+        Shape(B, H, L, D, 0), _ptr(l_S), _ptr(o_S), _ptr(lbar), _ptr(obar), _ptr(d_l), _ptr(d_o), _ptr(o),
+        _ptr(lse), _stream()))
+    return o, lse
+
+
+def complement_lists(mask, L, blk, D=128):
+    """The blocks each row does not keep: (idx int32 [B,H,NB,NB], cnt int32 [B,H,NB])."""
+    B, H, nb, _ = mask.shape
+    _need(mask, torch.uint8, (B, H, nb, nb), "mask")
+    idx = torch.empty((B, H, nb, nb), dtype=torch.int32, device=mask.device)
+    cnt = torch.empty((B, H, nb), dtype=torch.int32, device=mask.device)
+    check("bsa_complement_lists", _lib.load().bsa_complement_lists(
+        Shape(B, H, L, D, blk), _ptr(mask), _ptr(idx), _ptr(cnt), _stream()))
+    return idx, cnt
 
 
 def reorder_workspace_bytes(T, Hh, W):

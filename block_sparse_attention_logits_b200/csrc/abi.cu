@@ -215,6 +215,75 @@ int bsa_intervals_to_kept(bsa_shape s, const int32_t* intervals, const int32_t* 
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t bsa_tail_workspace_bytes(bsa_shape s) {
+  if (check_block_shape(s) != BSA_OK || s.D != 128) return 0;
+  return bsa::tail_workspace_bytes(s);
+}
+
+int bsa_tail_stats(bsa_shape s, const bsa_bf16* k, const bsa_bf16* v, float* kbar, float* s2, float* vbar, float* C,
+                   void* ws, size_t ws_bytes, int32_t* status, bsa_stream stream) {
+  if (!k || !v || !kbar || !s2 || !vbar || !C) return BSA_EINVAL;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kbar) || !aligned16(s2) || !aligned16(vbar) || !aligned16(C) ||
+      !word_ok(status))
+    return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (s.D != 128) return BSA_ESHAPE;
+  if (!ws || ws_bytes < bsa::tail_workspace_bytes(s)) return BSA_EWORKSPACE;
+  if (!aligned16(ws)) return BSA_EINVAL;
+  if (int r = check_device()) return r;
+  return bsa::launch_tail_stats(s, reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v),
+                                kbar, s2, vbar, C, ws, status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bsa_coarse_tail(bsa_shape s, const bsa_bf16* q, const uint8_t* mask, const void* ws, size_t ws_bytes, float* lbar,
+                    bsa_bf16* obar, int32_t* status, bsa_stream stream) {
+  if (!q || !mask || !lbar || !obar) return BSA_EINVAL;
+  if (!aligned16(q) || !aligned16(mask) || !aligned16(lbar) || !aligned16(obar) || !word_ok(status))
+    return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (s.D != 128 || s.blk != 128) return BSA_ESHAPE;
+  if (!ws || ws_bytes < bsa::tail_workspace_bytes(s)) return BSA_EWORKSPACE;
+  if (!aligned16(ws)) return BSA_EINVAL;
+  if (int r = check_device()) return r;
+  return bsa::launch_coarse_tail(s, reinterpret_cast<const __nv_bfloat16*>(q), mask, ws, lbar,
+                                 reinterpret_cast<__nv_bfloat16*>(obar), status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bsa_tail_refinement(bsa_shape s, const float* l_T, const bsa_bf16* o_T, const float* lbar, const bsa_bf16* obar,
+                        float* d_l, bsa_bf16* d_o, bsa_stream stream) {
+  if (!l_T || !o_T || !lbar || !obar || !d_l || !d_o) return BSA_EINVAL;
+  if (!aligned16(l_T) || !aligned16(o_T) || !aligned16(lbar) || !aligned16(obar) || !aligned16(d_l) ||
+      !aligned16(d_o))
+    return BSA_EINVAL;
+  if (int r = check_rows_shape(s)) return r;
+  if (int r = check_device()) return r;
+  return bsa::launch_tail_refine(s, l_T, reinterpret_cast<const __nv_bfloat16*>(o_T), lbar,
+                                 reinterpret_cast<const __nv_bfloat16*>(obar), d_l,
+                                 reinterpret_cast<__nv_bfloat16*>(d_o), reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bsa_tail_reconstruct(bsa_shape s, const float* l_S, const bsa_bf16* o_S, const float* lbar, const bsa_bf16* obar,
+                         const float* d_l, const bsa_bf16* d_o, bsa_bf16* o, float* lse, bsa_stream stream) {
+  if (!l_S || !o_S || !lbar || !obar || !d_l || !d_o || !o || !lse) return BSA_EINVAL;
+  if (!aligned16(l_S) || !aligned16(o_S) || !aligned16(lbar) || !aligned16(obar) || !aligned16(d_l) ||
+      !aligned16(d_o) || !aligned16(o) || !aligned16(lse))
+    return BSA_EINVAL;
+  if (int r = check_rows_shape(s)) return r;
+  if (int r = check_device()) return r;
+  return bsa::launch_tail_merge(s, l_S, reinterpret_cast<const __nv_bfloat16*>(o_S), lbar,
+                                reinterpret_cast<const __nv_bfloat16*>(obar), d_l,
+                                reinterpret_cast<const __nv_bfloat16*>(d_o), reinterpret_cast<__nv_bfloat16*>(o), lse,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bsa_complement_lists(bsa_shape s, const uint8_t* mask, int32_t* idx, int32_t* cnt, bsa_stream stream) {
+  if (!mask || !idx || !cnt) return BSA_EINVAL;
+  if (!aligned16(mask) || !aligned16(idx) || !aligned16(cnt)) return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (int r = check_device()) return r;
+  return bsa::launch_complement(s, mask, idx, cnt, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int bsa_wait_selftest(int32_t* status, unsigned long long limit_ns, bsa_stream stream) {
   if (!status || !word_ok(status)) return BSA_EINVAL;
   if (limit_ns == 0 || limit_ns > 2000000000ull) return BSA_EINVAL;

@@ -19,13 +19,14 @@
 // round robin); the last CTA of a launch resets its slot, so each launch finds
 // its slot at zero as long as fewer than kSchedSlots launches overlap.
 //
-// Tensor memory (512 columns): S0 | S1 | O0 | O1.  S is double buffered, so
-// the tensor core computes S for block n+1 while the softmax works on block
-// n; O is double buffered across work items, so the epilogue of one item
-// overlaps the next.  All MMAs are M=128, N=128 (or N=D), K=16: full-rate
-// shapes.  P of block n (bf16 pairs) overwrites the first 64 columns of its S
-// buffer; S of block n+2 reuses the buffer only after the PV of block n has
-// completed.
+// Tensor memory (512 columns): S0 | S1 | S2 | O at D = 128 (S0 | S1 | S2 |
+// O0 | O1 at D = 64).  S is triple buffered, so the tensor core can compute S
+// for blocks n+1 and n+2 while the softmax works on block n, and the S of
+// block n+3 waits only for the PV of block n.  P of block n (bf16 pairs)
+// overwrites the first 64 columns of its S buffer.  With one O buffer the
+// first PV of an item waits until the epilogue has read the previous item's
+// O out; the S MMAs and the softmax of the new item's first blocks run
+// meanwhile.  All MMAs are M=128, N=128 (or N=D), K=16: full-rate shapes.
 //
 // Warp roles (16 warps):
 //   warp 0       item queue; TMA: Q of every item (double buffered), K ring
@@ -47,9 +48,10 @@
 // the same reference.
 //
 // Fused refresh (kFused).  Every key block is visited once; the PV of a kept
-// block accumulates into OK, that of any other block into OR (TMEM: S0 | S1 |
-// OK | OR, so O is single-buffered across items and the PV of an item waits
-// until the epilogue has read the previous item's O).  One shared reference
+// block accumulates into OK, that of any other block into OR (TMEM at D = 128:
+// S0 | S1 | OK | OR, so S is double buffered and O single buffered across
+// items, and the PV of an item waits until the epilogue has read the previous
+// item's O).  One shared reference
 // max serves both; the softmax keeps the total row sum and the kept row sum.
 // The epilogue writes the dense output (OK + OR) / l, the sparse output
 // OK / l_kept, both LSEs, R = bf16(bf16(O_dense) - bf16(O_sparse)) and the kept
@@ -146,14 +148,13 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_STATS + STATS_BYTES;
   static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
   static constexpr int COL_S = 0;        // S[b] at b*BN
-  static constexpr int COL_O = 2 * BN;   // O[j] at COL_O + j*D
   static constexpr int PANELS = D / 64;
 };
 
 struct Shared {
   uint64_t full_k[4], empty_k[4], full_v[4], empty_v[4];
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t s_full[3], p_full[3], pv_done[3];
   uint64_t o_full[2], o_empty[2];
   uint64_t stats_full[2], stats_free[2];
   uint64_t drain[2];
@@ -328,8 +329,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const Params prm) {
   using C = Cfg<D>;
-  constexpr int OB = kFused ? 1 : 2;          // O buffers across items
+  // TMEM (512 columns): NS buffers of S (128 columns each) then OB buffers of
+  // the accumulator(s) of an item (D columns each; the fused refresh keeps two
+  // per item, OK and OR).  D = 128: S0|S1|S2|O, fused S0|S1|OK|OR.
   constexpr int OB_RESCALE = kFused ? 2 : 1;  // accumulators per item
+  constexpr int NS = kFused ? (512 - 2 * D) / BN : 3;
+  constexpr int OB_FIT = (512 - NS * BN) / (OB_RESCALE * D);
+  constexpr int OB = OB_FIT > 2 ? 2 : OB_FIT;  // O buffers across items
+  constexpr int COL_O = NS * BN;
+  static_assert(NS >= 2 && NS <= 3 && OB >= 1, "TMEM layout");
   constexpr int NSK = C::NSK;
   constexpr int NSV = C::NSV;
   extern __shared__ uint8_t smem_raw[];
@@ -354,12 +362,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh->item_full[s], 1);
       mbar_init(&sh->item_empty[s], kItemReaders);
     }
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(&sh->q_full[j], 1);
-      mbar_init(&sh->q_empty[j], 1);
+    for (int j = 0; j < 3; ++j) {
       mbar_init(&sh->s_full[j], 1);
       mbar_init(&sh->p_full[j], 256);
       mbar_init(&sh->pv_done[j], 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&sh->q_full[j], 1);
+      mbar_init(&sh->q_empty[j], 1);
       mbar_init(&sh->o_full[j], 1);
       mbar_init(&sh->o_empty[j], 128);
       mbar_init(&sh->stats_full[j], 256);
@@ -487,9 +497,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int n = 0; n < it.cnt; ++n) {
           if (entry_kb(it, n, NB) < 0) continue;
           const int sk = u % NSK;
-          const int b = u & 1;
+          const int b = u % NS;
           if (!(ok = warp_wait(&sh->full_k[sk], (u / NSK) & 1, sh, prm))) break;
-          if (u >= 2 && !(ok = warp_wait(&sh->pv_done[b], ((u - 2) >> 1) & 1, sh, prm))) break;
+          // S[b] held P of block u - NS: its PV must have read it
+          if (u >= NS && !(ok = warp_wait(&sh->pv_done[b], ((u - NS) / NS) & 1, sh, prm))) break;
           tc_fence_after();
           if (lane == 0) {
             const uint32_t ka = k_base + sk * C::KV_BYTES;
@@ -525,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int w = next_item(i, sh, prm);
         if (w < 0) break;
         const Item it = item_of<kFused>(w, prm);
-        const int ob = kFused ? 0 : (i & 1);
+        const int ob = i % OB;
         if (i >= OB && !(ok = warp_wait(&sh->o_empty[ob], ((i - OB) / OB) & 1, sh, prm))) break;
         bool first = true, first_rest = true;
         int kp = 0;
@@ -535,14 +546,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kb < 0) continue;
           const bool kept = !kFused || kept_at(it, kb, kp, bad);
           const int sv = u % NSV;
-          const int b = u & 1;
-          if (!(ok = warp_wait(&sh->p_full[b], (u >> 1) & 1, sh, prm))) break;
+          const int b = u % NS;
+          if (!(ok = warp_wait(&sh->p_full[b], (u / NS) & 1, sh, prm))) break;
           if (!(ok = warp_wait(&sh->full_v[sv], (u / NSV) & 1, sh, prm))) break;
           tc_fence_after();
           const bool fresh = kept ? first : first_rest;
           if (lane == 0) {
             const uint32_t va = v_base + sv * C::KV_BYTES;
-            const uint32_t dst = tmem + C::COL_O + (kFused ? (kept ? 0 : D) : ob * D);
+            const uint32_t dst = tmem + COL_O + (kFused ? (kept ? 0 : D) : ob * D);
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)
               mma_ts(dst, tmem + C::COL_S + b * BN + kk * 8, sdesc_sw128(va + kk * 2048, BN * 128, 1024), idPV,
@@ -584,9 +595,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int w = next_item(i, sh, prm);
       if (w < 0) break;
       const Item it = item_of<kFused>(w, prm);
-      const int ob = kFused ? 0 : (i & 1);
+      const int ob = i % OB;
       const int sb = i & 1;  // statistics buffer
-      const uint32_t tO = tmem + lane_off + C::COL_O + ob * D;
+      const uint32_t tO = tmem + lane_off + COL_O + ob * D;
       float mA = -INFINITY, mB = -INFINITY;  // reference max of rows rA, rA+8 (log2 units)
       float lA = 0.f, lB = 0.f;              // this thread's share of the row sums
       float kA = 0.f, kB = 0.f;              // fused refresh: the same over the kept blocks
@@ -597,9 +608,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kb = entry_kb(it, n, NB);
         if (kb < 0) continue;
         const bool kept = !kFused || kept_at(it, kb, kp, bad);
-        const int b = u & 1;
+        const int b = u % NS;
         const uint32_t tS = tmem + lane_off + C::COL_S + b * BN;
-        if (!(ok = warp_wait(&sh->s_full[b], (u >> 1) & 1, sh, prm))) break;
+        if (!(ok = warp_wait(&sh->s_full[b], (u / NS) & 1, sh, prm))) break;
         tc_fence_after();
         // s[chunk][0..1]: row rA, keys 8*chunk + 2*j4 + {0,1}; s[chunk][2..3]: row rA+8
         uint32_t sr[2][32];
@@ -652,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (nt > 0 && __any_sync(0xffffffffu, rsA || rsB)) {
           // O must hold the previous block's PV before it is rescaled
-          if (!(ok = warp_wait(&sh->pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1, sh, prm))) break;
+          if (!(ok = warp_wait(&sh->pv_done[(u - 1) % NS], ((u - 1) / NS) & 1, sh, prm))) break;
           tc_fence_after();
 #pragma unroll
           for (int cc = 0; cc < OB_RESCALE * D / 64; ++cc) {  // fused: OK and OR
@@ -747,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int w = next_item(i, sh, prm);
       if (w < 0) break;
       const Item it = item_of<kFused>(w, prm);
-      const int ob = kFused ? 0 : (i & 1);
+      const int ob = i % OB;
       const int sb = i & 1;
       if (!(ok = warp_wait(&sh->o_full[ob], (i / OB) & 1, sh, prm))) break;
       if (!(ok = warp_wait(&sh->stats_full[sb], (i >> 1) & 1, sh, prm))) break;
@@ -769,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const size_t row_elem = (static_cast<size_t>(it.bh) * L + (store ? grow : 0)) * D;
       const size_t out_elem = (static_cast<size_t>(it.bh) * L + (store ? orow : 0)) * D;
-      const uint32_t tO = tmem + lane_off + C::COL_O + ob * D;
+      const uint32_t tO = tmem + lane_off + COL_O + ob * D;
       if constexpr (kFused) {
         // dense = (OK + OR) / l, sparse = OK / l_kept.  OK holds data only if
         // some block was kept (l_kept > 0), OR only if some block was not,

@@ -54,6 +54,19 @@ cudaError_t launch_interval_decode(const bsa_shape& s, const int32_t* intervals,
                                    cudaStream_t st);
 // one thread waits on an mbarrier nothing arrives at, for limit_ns
 cudaError_t launch_wait_selftest(int32_t* status, unsigned long long limit_ns, cudaStream_t st);
+// coarse tail (D = 128): moments and pooled covariance, then the tail itself;
+// `ws` holds the centred transposed K/V and the operand tables between them
+size_t tail_workspace_bytes(const bsa_shape& s);
+int launch_tail_stats(const bsa_shape& s, const __nv_bfloat16* k, const __nv_bfloat16* v, float* kbar, float* s2,
+                      float* vbar, float* C, void* ws, int32_t* status, cudaStream_t st);
+int launch_coarse_tail(const bsa_shape& s, const __nv_bfloat16* q, const uint8_t* mask, const void* ws,
+                       float* lbar, __nv_bfloat16* obar, int32_t* status, cudaStream_t st);
+int launch_tail_refine(const bsa_shape& s, const float* l_T, const __nv_bfloat16* o_T, const float* lbar,
+                       const __nv_bfloat16* obar, float* d_l, __nv_bfloat16* d_o, cudaStream_t st);
+int launch_tail_merge(const bsa_shape& s, const float* l_S, const __nv_bfloat16* o_S, const float* lbar,
+                      const __nv_bfloat16* obar, const float* d_l, const __nv_bfloat16* d_o, __nv_bfloat16* o,
+                      float* lse, cudaStream_t st);
+int launch_complement(const bsa_shape& s, const uint8_t* mask, int32_t* idx, int32_t* cnt, cudaStream_t st);
 size_t hilbert_workspace_bytes(int T, int Hh, int W);
 cudaError_t launch_hilbert(int T, int Hh, int W, int32_t* perm, int32_t* inv, void* ws, cudaStream_t st);
 cudaError_t launch_permute(const bsa_shape& s, const __nv_bfloat16* x, const int32_t* perm, __nv_bfloat16* y,

@@ -185,6 +185,14 @@ __device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_
       BSA_W8(0), BSA_W8(8), BSA_W8(16), BSA_W8(24)
       : "memory");
 }
+// 8 chunks of 4 columns = 32 columns, 16 registers
+__device__ __forceinline__ void tmem_st_16x128b_x8(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      BSA_W8(0), BSA_W8(8)
+      : "memory");
+}
 // 16 chunks of 4 columns = 64 columns, 32 registers
 __device__ __forceinline__ void tmem_st_16x128b_x16(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(

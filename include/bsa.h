@@ -300,6 +300,62 @@ BSA_API int bsa_intervals_to_kept(bsa_shape s, const int32_t* intervals, const i
                                   int32_t* kept_idx, int32_t* kept_cnt, int32_t* status, bsa_stream stream);
 
 /*
+ * Coarse tail of the omitted blocks and its reconstruction (RECAP, section
+ * 3.2).  Per head, with a = q / sqrt(D) and T(i) the blocks query block i does
+ * NOT keep:
+ *   block log-mass  log n_j + a . kbar_j + 1/2 sum_d a_d^2 s2_j[d]
+ *   lbar  = log sum_{j in T(i)} exp(block log-mass)          (-inf if T(i) is empty)
+ *   obar  = sum_{j in T(i)} w_j vbar_j + C a                   (0 if T(i) is empty)
+ * kbar_j, s2_j, vbar_j: the block's key mean, per-dimension key variance
+ * (population) and value mean; w_j the normalised block masses; C[e][d] =
+ * (1/L) sum over all tokens of (v - vbar_block)[e] (k - kbar_block)[d], the
+ * pooled within-block value-key covariance.  At a dense refresh the cached
+ * refinement is d = (l_T - lbar, o_T - obar) with (l_T, o_T) the exact
+ * attention over T(i); a later sparse step returns
+ *   LSE = logaddexp(l_S, lbar + d_l),  O = w_S O_S + w_T (obar + d_o).
+ * D must be 128 for the statistics and the tail.
+ */
+
+/* Workspace bytes that bsa_tail_stats and bsa_coarse_tail share (0 for an
+ * unsupported shape). */
+BSA_API size_t bsa_tail_workspace_bytes(bsa_shape s);
+
+/*
+ * bsa_tail_stats -- block moments and the pooled covariance of K and V.
+ * Outputs kbar, s2, vbar float32 [B,H,NB,D], C float32 [B,H,D,D]; ws (device,
+ * bsa_tail_workspace_bytes) receives the operand tables bsa_coarse_tail reads.
+ * Errors: BSA_EINVAL, BSA_ESHAPE (D != 128), BSA_EWORKSPACE, BSA_ENODEV,
+ * BSA_ECUDA.
+ */
+BSA_API int bsa_tail_stats(bsa_shape s, const bsa_bf16* k, const bsa_bf16* v, float* kbar, float* s2, float* vbar,
+                           float* C, void* ws, size_t ws_bytes, int32_t* status, bsa_stream stream);
+
+/*
+ * bsa_coarse_tail -- lbar float32 [B,H,L] and obar bf16 [B,H,L,D] over the
+ * blocks each query block omits.  mask: uint8 [B,H,NB,NB] (1 = kept), as
+ * bsa_select_topp_mask writes it; ws as written by bsa_tail_stats for the same
+ * K and V.  s.blk must be 128 and s.D 128.
+ */
+BSA_API int bsa_coarse_tail(bsa_shape s, const bsa_bf16* q, const uint8_t* mask, const void* ws, size_t ws_bytes,
+                            float* lbar, bsa_bf16* obar, int32_t* status, bsa_stream stream);
+
+/* bsa_tail_refinement -- d_l = l_T - lbar, d_o = bf16(o_T - obar) (both 0
+ * where the tail is empty); l_T, o_T: the exact attention over the omitted
+ * blocks (bsa_sparse_attn_fwd with bsa_complement_lists). */
+BSA_API int bsa_tail_refinement(bsa_shape s, const float* l_T, const bsa_bf16* o_T, const float* lbar,
+                                const bsa_bf16* obar, float* d_l, bsa_bf16* d_o, bsa_stream stream);
+
+/* bsa_tail_reconstruct -- the sparse part (l_S, o_S) merged with the
+ * reconstructed tail (lbar + d_l, obar + d_o): o bf16 [B,H,L,D], lse float32. */
+BSA_API int bsa_tail_reconstruct(bsa_shape s, const float* l_S, const bsa_bf16* o_S, const float* lbar,
+                                 const bsa_bf16* obar, const float* d_l, const bsa_bf16* d_o, bsa_bf16* o,
+                                 float* lse, bsa_stream stream);
+
+/* bsa_complement_lists -- the blocks each row does not keep (mask 0), as
+ * ascending lists in the layout of bsa_select_topp_mask. */
+BSA_API int bsa_complement_lists(bsa_shape s, const uint8_t* mask, int32_t* idx, int32_t* cnt, bsa_stream stream);
+
+/*
  * bsa_wait_selftest -- exercises the bounded wait that every pipeline wait of
  * the library uses: one thread waits on an mbarrier that nothing arrives at,
  * gives up after limit_ns (1 ns .. 2 s) of the GPU's global timer, ORs

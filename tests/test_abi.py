@@ -245,3 +245,31 @@ def test_wait_selftest_validation(lib):
     assert lib.bsa_wait_selftest(ctypes.c_void_p((1 << 20) + 2), 1000, NULL) == _lib.BSA_EINVAL
     assert lib.bsa_wait_selftest(FAKE, 0, NULL) == _lib.BSA_EINVAL
     assert lib.bsa_wait_selftest(FAKE, 3_000_000_000, NULL) == _lib.BSA_EINVAL
+
+
+def test_tail_validation(lib):
+    s = Shape(1, 2, 1000, 128, 128)
+    need = lib.bsa_tail_workspace_bytes(s)
+    assert need > 0 and lib.bsa_tail_workspace_bytes(Shape(1, 2, 1000, 64, 128)) == 0
+    # statistics: every output required, D = 128, the workspace big enough
+    assert lib.bsa_tail_stats(s, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, FAKE, need, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_tail_stats(Shape(1, 2, 1000, 64, 128), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, NULL,
+                              NULL) == _lib.BSA_ESHAPE
+    assert lib.bsa_tail_stats(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, NULL,
+                              NULL) == _lib.BSA_EWORKSPACE
+    assert lib.bsa_tail_stats(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, need, NULL, NULL) == _lib.BSA_EWORKSPACE
+    # the tail: 128-token blocks, D = 128, word-aligned status
+    assert lib.bsa_coarse_tail(Shape(1, 2, 1000, 128, 64), FAKE, FAKE, FAKE, need, FAKE, FAKE, NULL,
+                               NULL) == _lib.BSA_ESHAPE
+    assert lib.bsa_coarse_tail(s, FAKE, FAKE, FAKE, need - 1, FAKE, FAKE, NULL, NULL) == _lib.BSA_EWORKSPACE
+    assert lib.bsa_coarse_tail(s, FAKE, NULL, FAKE, need, FAKE, FAKE, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_coarse_tail(s, FAKE, FAKE, FAKE, need, FAKE, FAKE, ctypes.c_void_p((1 << 20) + 2),
+                               NULL) == _lib.BSA_EINVAL
+    # elementwise refinement / reconstruction and the complement lists
+    e = Shape(1, 2, 100, 12, 0)
+    assert lib.bsa_tail_refinement(e, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, NULL) == _lib.BSA_ESHAPE
+    assert lib.bsa_tail_refinement(Shape(1, 2, 100, 16, 0), FAKE, FAKE, NULL, FAKE, FAKE, FAKE,
+                                   NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_tail_reconstruct(Shape(1, 2, 100, 16, 0), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, FAKE,
+                                    NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_complement_lists(s, FAKE, NULL, FAKE, NULL) == _lib.BSA_EINVAL
