@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wan2.1-14b-720p", choices=sorted(configs.ALL))
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
+    ap.add_argument("--top-p", type=float, default=0.0,
+                    help="top-p threshold for every head (default: the workload's first value)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run only the first N heads of the workload (small profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -711,7 +713,8 @@ def run_reference(args, w, world, rank):
     out = {
         "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(sec / args.steps * 1e3, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "scaling": "strong" if (world > 1 and args.shard == "heads") else "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "D": w.D, "blk": w.blk,
                    "grid": list(w.grid), "hilbert": w.hilbert, "top_p": p,
                    "parallelism": "CPU oracle on rank 0"},
@@ -731,6 +734,9 @@ def main():
     if args.heads:
         import dataclasses
         w = dataclasses.replace(w, H=min(args.heads, w.H))
+    if args.top_p:
+        import dataclasses
+        w = dataclasses.replace(w, p=(float(args.top_p),))
     if args.impl == "reference":
         run_reference(args, w, world, rank)
     else:

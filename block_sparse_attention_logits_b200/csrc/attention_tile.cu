@@ -84,6 +84,16 @@ constexpr int BM = 128;                         // query rows per work item
 constexpr int BN = 128;                         // keys per block
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
 constexpr float kRescaleThreshold = 8.0f;       // log2 units
+// Key pairs whose exponentials are evaluated on the FMA pipe by exp2_poly
+// instead of the exp unit: bit 2k is row rA's pair in 8-key chunk k of the 16 a
+// softmax thread handles per block, bit 2k+1 row rA+8's
+constexpr uint32_t kPolyPairs = 0x0000C000u;
+// Q tiles in shared memory across items: one leaves room for a third K slot
+constexpr int kQBuffers = 1;
+// S of a block read by one 128-column TMEM load per warp instead of two
+constexpr bool kWideLoad = false;
+// cycles by which the second softmax group starts after the first (0: none)
+constexpr int kGroupOffset = 500;
 constexpr int kQueue = 4;                       // item queue depth
 constexpr int kItemReaders = 32 * 3 + 256 + 128;  // threads of the roles that read the queue
 // registers per thread: launch 65536 / 512 = 128, then re-balanced per warpgroup
@@ -134,15 +144,16 @@ struct Params {
 template <int D>
 struct Cfg {
   static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int NQ = kQBuffers;            // Q buffers across items
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int STATS_BYTES = 2 * 3 * BM * 4;  // [item parity][l, m, l_kept][row]
   static constexpr int MISC_BYTES = 512;
-  static constexpr int SLOTS = (227 * 1024 - 1024 - 2 * Q_BYTES - STATS_BYTES - MISC_BYTES) / KV_BYTES;
+  static constexpr int SLOTS = (227 * 1024 - 1024 - NQ * Q_BYTES - STATS_BYTES - MISC_BYTES) / KV_BYTES;
   static constexpr int NSK = ((SLOTS + 1) / 2) > 4 ? 4 : (SLOTS + 1) / 2;
   static constexpr int NSV = (SLOTS / 2) > 4 ? 4 : SLOTS / 2;
   static_assert(NSK >= 2 && NSV >= 2, "shared memory too small for double-buffered K and V");
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = 2 * Q_BYTES;
+  static constexpr int OFF_K = NQ * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
   static constexpr int OFF_STATS = OFF_V + NSV * KV_BYTES;
   static constexpr int OFF_MISC = OFF_STATS + STATS_BYTES;
@@ -225,6 +236,32 @@ __device__ void sched_leave(SchedSlot* s, uint32_t tag, const Params& prm) {
     cur = got;
   }
   flag_status(prm, BSA_DEV_SCHED_CONFLICT);
+}
+
+// 2^x for a pair of floats (x <= 127) on the FMA and integer pipes, without
+// the exp unit: x = j + f with j the nearest integer and f in [-1/2, 1/2]
+// (adding 1.5 * 2^23 rounds x to an integer, whose value lands in the low
+// mantissa bits); 2^f by a degree-3 polynomial fitted to a relative error of
+// 7.5e-5 on that interval, far below the bf16 rounding of P; 2^j added to the
+// exponent field.  x below -125 gives 2^-125 (about 2e-38) instead of ~0.
+__device__ __forceinline__ uint64_t exp2_poly(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  const uint64_t xc = f2_pack(x0, x1);
+  const uint64_t t = f2_add(xc, f2_pack(12582912.f, 12582912.f));
+  const uint64_t j = f2_add(t, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t fr = f2_fma(j, f2_pack(-1.f, -1.f), xc);
+  uint64_t p = f2_fma(f2_pack(0.055171772837638855f, 0.055171772837638855f), fr,
+                      f2_pack(0.24261115491390228f, 0.24261115491390228f));
+  p = f2_fma(p, fr, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, fr, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }
 
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Shared* sh, const Params& prm) {
@@ -422,8 +459,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (w < 0) break;
         const Item it = item_of<kFused>(w, prm);
         if (it.bad_cnt && lane == 0) flag_status(prm, BSA_DEV_BAD_INDEX);
-        const int qb = i & 1;
-        if (i >= 2 && !(ok = warp_wait(&sh->q_empty[qb], ((i - 2) >> 1) & 1, sh, prm))) break;
+        const int qb = i % C::NQ;
+        if (i >= C::NQ && !(ok = warp_wait(&sh->q_empty[qb], ((i - C::NQ) / C::NQ) & 1, sh, prm))) break;
         if (lane == 0) {
           mbar_arrive_expect_tx(&sh->q_full[qb], C::Q_BYTES);
           for (int pnl = 0; pnl < C::PANELS; ++pnl)
@@ -491,8 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int w = next_item(i, sh, prm);
         if (w < 0) break;
         const Item it = item_of<kFused>(w, prm);
-        const int qb = i & 1;
-        if (!(ok = warp_wait(&sh->q_full[qb], (i >> 1) & 1, sh, prm))) break;
+        const int qb = i % C::NQ;
+        if (!(ok = warp_wait(&sh->q_full[qb], (i / C::NQ) & 1, sh, prm))) break;
         const uint32_t qa = q_base + qb * C::Q_BYTES;
         for (int n = 0; n < it.cnt; ++n) {
           if (entry_kb(it, n, NB) < 0) continue;
@@ -589,6 +626,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32 + grp * 16) << 16;
     const float sl2 = prm.scale_log2;
     const uint64_t scale2 = f2_pack(sl2, sl2);
+    if (kGroupOffset > 0 && grp == 1) {
+      // the second group starts later, so that the two groups' exponentials
+      // (bound by the exp unit they share) fall at different times
+      const uint64_t c0 = clock64();
+      while (clock64() - c0 < static_cast<uint64_t>(kGroupOffset)) {
+      }
+    }
     int u = 0;
     bool ok = true;
     for (int i = 0; ok; ++i) {
@@ -614,8 +658,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // s[chunk][0..1]: row rA, keys 8*chunk + 2*j4 + {0,1}; s[chunk][2..3]: row rA+8
         uint32_t sr[2][32];
-        tmem_ld_16x256b_x8(tS, sr[0]);
-        tmem_ld_16x256b_x8(tS + 64, sr[1]);
+        if constexpr (kWideLoad) {
+          tmem_ld_16x256b_x16(tS, reinterpret_cast<uint32_t(&)[64]>(sr));
+        } else {
+          tmem_ld_16x256b_x8(tS, sr[0]);
+          tmem_ld_16x256b_x8(tS + 64, sr[1]);
+        }
         tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < 2; ++q)
@@ -688,11 +736,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t* c4 = &sr[k >> 3][(k & 7) * 4];
           const uint64_t xA = f2_fma(f2_pack(__uint_as_float(c4[0]), __uint_as_float(c4[1])), scale2, negA);
           const uint64_t xB = f2_fma(f2_pack(__uint_as_float(c4[2]), __uint_as_float(c4[3])), scale2, negB);
-          float a0, a1, b0, b1;
-          f2_unpack(xA, a0, a1);
-          f2_unpack(xB, b0, b1);
-          const float pa0 = ex2_approx(a0), pa1 = ex2_approx(a1);
-          const float pb0 = ex2_approx(b0), pb1 = ex2_approx(b1);
+          float pa0, pa1, pb0, pb1;
+          if ((kPolyPairs >> (2 * k)) & 1u) {
+            f2_unpack(exp2_poly(xA), pa0, pa1);
+          } else {
+            float a0, a1;
+            f2_unpack(xA, a0, a1);
+            pa0 = ex2_approx(a0);
+            pa1 = ex2_approx(a1);
+          }
+          if ((kPolyPairs >> (2 * k + 1)) & 1u) {
+            f2_unpack(exp2_poly(xB), pb0, pb1);
+          } else {
+            float b0, b1;
+            f2_unpack(xB, b0, b1);
+            pb0 = ex2_approx(b0);
+            pb1 = ex2_approx(b1);
+          }
           if (k & 1) {
             accA1 = f2_add(accA1, f2_pack(pa0, pa1));
             accB1 = f2_add(accB1, f2_pack(pb0, pb1));

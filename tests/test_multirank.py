@@ -66,7 +66,7 @@ def test_reference_arm_two_ranks_prints_one_line_from_rank_zero():
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1
     d = json.loads(lines[0])
-    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["scaling"] == "weak"
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["scaling"] == "strong"  # heads sharded
     assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
 
 
