@@ -42,9 +42,11 @@ Modules:
                  and its reconstruction with a cached refinement
   intervals   -- interval (skip-list) encoding of the kept blocks, merging of
                  outlier rows to a width, the width for a merge percentage
+  fp8         -- E4M3 quantization of Q and K per token block (the FP8 path)
 
-Every function carries a "Pinned by" note naming the tests in
-``tests/test_oracle.py`` that tie it to something other than itself.
+Every function carries a "Pinned by" note naming the tests (in
+``tests/test_oracle.py`` unless stated) that tie it to something other than
+itself.
 """
 
-from . import hilbert, scoring, topp, attention, correction, refresh, reuse, intervals, tail  # noqa: F401
+from . import hilbert, scoring, topp, attention, correction, refresh, reuse, intervals, tail, fp8  # noqa: F401
