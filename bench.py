@@ -340,6 +340,40 @@ def tail_timings(q, k, v, mask, idx, cnt, blk, barrier):
     return ms
 
 
+def fp8_timings(q, k, v, idx, cnt, blk, flops, barrier, hbm_gbs):
+    """FP8 Q.K^T attention on a step's inputs: E4M3 quantization of Q and K
+    per token block (HBM-bound: 2 bytes read and 1 written per element), then
+    the block-sparse attention over the same kept lists with S = Q.K^T from
+    the codes; ms per call and kept TFLOP/s."""
+    from block_sparse_attention_logits_b200 import api
+    st = torch.zeros(1, dtype=torch.int32, device=q.device)
+    q8, qs = api.quantize_fp8(q, blk)
+    k8, ks = api.quantize_fp8(k, blk)
+    o, lse = api.sparse_attn_fwd_fp8(q8, qs, k8, ks, v, blk, idx, cnt, status=st)
+    calls = (("quantize_qk", lambda: (api.quantize_fp8(q, blk, q8, qs), api.quantize_fp8(k, blk, k8, ks))),
+             ("attention", lambda: api.sparse_attn_fwd_fp8(q8, qs, k8, ks, v, blk, idx, cnt, o=o, lse=lse,
+                                                           status=st)))
+    ms = {}
+    for name, fn in calls:
+        fn()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(5):
+            fn()
+        a1.record()
+        barrier()
+        ms[name] = a0.elapsed_time(a1) / 5
+    qk_bytes = 2 * q.numel() * 3
+    return {"quantize_qk_ms": round(ms["quantize_qk"], 4),
+            "quantize_GB/s": round(qk_bytes / (ms["quantize_qk"] * 1e-3) / 1e9, 1),
+            "quantize_frac_of_hbm": round(qk_bytes / (ms["quantize_qk"] * 1e-3) / 1e9 / hbm_gbs, 3),
+            "attention_ms": round(ms["attention"], 4),
+            "kept_tflops": round(flops / (ms["attention"] * 1e-3) / 1e12, 2),
+            "scaling": "E4M3 per (batch, head, 128-token block), scale = amax / 448; P and V bf16",
+            "status": int(st.item())}
+
+
 def run_ours(args, w, world, rank, local):
     from block_sparse_attention_logits_b200 import api, _lib
     from block_sparse_attention_logits_b200 import build as bsa_build
@@ -573,6 +607,16 @@ def run_ours(args, w, world, rank, local):
         except Exception as e:  # noqa: BLE001
             tail = {"error": f"{type(e).__name__}: {e}"}
 
+    # FP8 Q.K^T attention over the step's kept lists (D = 128, 128-token blocks)
+    fp8 = None
+    if not args.no_refresh and D == 128 and blk == 128:
+        try:
+            qs_, ks_, vs_ = (bufs["qh"], bufs["kh"], bufs["vh"]) if w.hilbert else (q, k, v)
+            fp8 = fp8_timings(qs_, ks_, vs_, bufs["idx"], bufs["cnt"], blk, flops, barrier,
+                              load_peaks()[0]["hbm_gbs"])
+        except Exception as e:  # noqa: BLE001
+            fp8 = {"error": f"{type(e).__name__}: {e}"}
+
     # the elementwise calls (refinement at a refresh, standalone correction):
     # HBM-bound, three [B,H,L,D] bf16 streams each
     elementwise = None
@@ -683,7 +727,7 @@ def run_ours(args, w, world, rank, local):
         "stages_ms": {"gather_score_and_select": round(float(np.mean(sel_ms)), 4), "attention": round(attn_avg_ms, 4),
                       "rest": round(ms_step - attn_avg_ms - float(np.mean(sel_ms)), 4)},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "refresh": refresh, "reuse": reuse,
-        "elementwise": elementwise, "sweep": sweep, "intervals": intervals, "tail": tail,
+        "elementwise": elementwise, "sweep": sweep, "intervals": intervals, "tail": tail, "fp8": fp8,
         "gpu_launches": LAUNCHES_PER_STEP * K if w.hilbert else (LAUNCHES_PER_STEP - 1) * K,
         "clocks": clk,
     }

@@ -16,7 +16,7 @@ EXPORTS = (
     "bsa_select_topp_mask", "bsa_select_topp_mask_restricted",
     "bsa_interval_runs", "bsa_interval_width_for_merge", "bsa_kept_to_intervals", "bsa_intervals_to_kept",
     "bsa_tail_workspace_bytes", "bsa_tail_stats", "bsa_coarse_tail", "bsa_tail_refinement", "bsa_tail_reconstruct",
-    "bsa_complement_lists",
+    "bsa_complement_lists", "bsa_quantize_fp8", "bsa_sparse_attn_fwd_fp8",
     "bsa_wait_selftest",
     "bsa_reorder_workspace_bytes", "bsa_reorder_tokens", "bsa_reorder_tokens_noalloc", "bsa_permute_tokens",
     "bsa_sparse_attn_fwd", "bsa_sparse_attn_fwd_scatter", "bsa_sparse_attn_refresh", "bsa_refresh_refinement", "bsa_apply_correction",
@@ -76,6 +76,8 @@ def load():
         "bsa_tail_refinement": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_tail_reconstruct": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_complement_lists": (_I, [Shape, _P, _P, _P, _P]),
+        "bsa_quantize_fp8": (_I, [Shape, _P, _P, _P, _P]),
+        "bsa_sparse_attn_fwd_fp8": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_reorder_workspace_bytes": (_SZ, [_I, _I, _I]),
         "bsa_reorder_tokens": (_I, [_I, _I, _I, _P, _P, _P, _SZ, _P]),
         "bsa_reorder_tokens_noalloc": (_I, [_I, _I, _I, _P, _P, _P]),

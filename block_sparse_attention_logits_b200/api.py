@@ -31,6 +31,8 @@ __all__ = [
     "tail_refinement",
     "tail_reconstruct",
     "complement_lists",
+    "quantize_fp8",
+    "sparse_attn_fwd_fp8",
     "reorder_workspace_bytes",
     "reorder_tokens",
     "permute_tokens",
@@ -351,6 +353,50 @@ def complement_lists(mask, L, blk, D=128):
     check("bsa_complement_lists", _lib.load().bsa_complement_lists(
         Shape(B, H, L, D, blk), _ptr(mask), _ptr(idx), _ptr(cnt), _stream()))
     return idx, cnt
+
+
+def quantize_fp8(x, blk, codes=None, scales=None):
+    """E4M3 codes (uint8 [B,H,L,D]) and per-block scales (float32 [B,H,NB]) of
+    a bf16 [B,H,L,D] tensor: scale = amax / 448 per (b, h, block)."""
+    B, H, L, D = x.shape
+    nb = n_blocks(L, blk)
+    _need(x, torch.bfloat16, (B, H, L, D), "x")
+    codes = codes if codes is not None else torch.empty((B, H, L, D), dtype=torch.uint8, device=x.device)
+    scales = scales if scales is not None else torch.empty((B, H, nb), dtype=torch.float32, device=x.device)
+    _need(codes, torch.uint8, (B, H, L, D), "codes")
+    _need(scales, torch.float32, (B, H, nb), "scales")
+    check("bsa_quantize_fp8", _lib.load().bsa_quantize_fp8(
+        Shape(B, H, L, D, blk), _ptr(x), _ptr(codes), _ptr(scales), _stream()))
+    return codes, scales
+
+
+def sparse_attn_fwd_fp8(q8, q_scale, k8, k_scale, v, blk, kept_idx=None, kept_cnt=None, R=None, alpha=None,
+                        o=None, lse=None, status=None):
+    """Block-sparse attention with S = Q.K^T from E4M3 codes (blk 128, D 128);
+    otherwise as sparse_attn_fwd.  Returns (o bf16, lse float32)."""
+    B, H, L, D = v.shape
+    nb = n_blocks(L, blk)
+    _need(v, torch.bfloat16, (B, H, L, D), "v")
+    for name, t in (("q8", q8), ("k8", k8)):
+        _need(t, torch.uint8, (B, H, L, D), name)
+    for name, t in (("q_scale", q_scale), ("k_scale", k_scale)):
+        _need(t, torch.float32, (B, H, nb), name)
+    if kept_idx is not None:
+        _need(kept_idx, torch.int32, (B, H, nb, nb), "kept_idx")
+        _need(kept_cnt, torch.int32, (B, H, nb), "kept_cnt")
+    if R is not None:
+        _need(R, torch.bfloat16, (B, H, L, D), "R")
+        _need(alpha, torch.float32, (H,), "alpha")
+    o = o if o is not None else torch.empty_like(v)
+    lse = lse if lse is not None else torch.empty((B, H, L), dtype=torch.float32, device=v.device)
+    _need(o, torch.bfloat16, (B, H, L, D), "o")
+    _need(lse, torch.float32, (B, H, L), "lse")
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
+    check("bsa_sparse_attn_fwd_fp8", _lib.load().bsa_sparse_attn_fwd_fp8(
+        Shape(B, H, L, D, blk), _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(v), _ptr(kept_idx),
+        _ptr(kept_cnt), _ptr(R), _ptr(alpha), _ptr(o), _ptr(lse), _ptr(status), _stream()))
+    return o, lse
 
 
 def reorder_workspace_bytes(T, Hh, W):

@@ -357,6 +357,47 @@ int bsa_sparse_attn_fwd_scatter(bsa_shape s, const bsa_bf16* q, const bsa_bf16* 
   return bsa::launch_sparse_attn(s, a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int bsa_quantize_fp8(bsa_shape s, const bsa_bf16* x, uint8_t* codes, float* scales, bsa_stream stream) {
+  if (!x || !codes || !scales) return BSA_EINVAL;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (int r = check_device()) return r;
+  return from_cuda(bsa::launch_quantize_fp8(s, reinterpret_cast<const __nv_bfloat16*>(x), codes, scales,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int bsa_sparse_attn_fwd_fp8(bsa_shape s, const uint8_t* q8, const float* q_scale, const uint8_t* k8,
+                            const float* k_scale, const bsa_bf16* v, const int32_t* kept_idx, const int32_t* kept_cnt,
+                            const bsa_bf16* R, const float* alpha, bsa_bf16* o, float* lse, int32_t* status,
+                            bsa_stream stream) {
+  if (!q8 || !q_scale || !k8 || !k_scale || !v || !o || !lse) return BSA_EINVAL;
+  if ((kept_idx == nullptr) != (kept_cnt == nullptr)) return BSA_EINVAL;
+  if ((R == nullptr) != (alpha == nullptr)) return BSA_EINVAL;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return BSA_EINVAL;
+  if ((kept_idx && !aligned16(kept_idx)) || (kept_cnt && !aligned16(kept_cnt)) || (R && !aligned16(R)))
+    return BSA_EINVAL;
+  if (!word_ok(q_scale) || !word_ok(k_scale) || !word_ok(status) || !word_ok(alpha)) return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (s.blk != 128 || s.D != 128) return BSA_ESHAPE;
+  if (int r = check_device()) return r;
+  bsa::AttnArgs a;
+  a.q = nullptr;
+  a.k = nullptr;
+  a.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  a.kept_idx = kept_idx;
+  a.kept_cnt = kept_cnt;
+  a.R = reinterpret_cast<const __nv_bfloat16*>(R);
+  a.alpha = alpha;
+  a.o = reinterpret_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.status = status;
+  a.q8 = q8;
+  a.k8 = k8;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  return bsa::launch_sparse_attn(s, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int bsa_sparse_attn_refresh(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
                             const int32_t* kept_idx, const int32_t* kept_cnt, bsa_bf16* o_dense, float* lse_dense,
                             bsa_bf16* o_sparse, float* lse_sparse, bsa_bf16* R, float* kept_mass, int32_t* status,

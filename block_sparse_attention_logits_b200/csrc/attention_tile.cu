@@ -92,8 +92,6 @@ constexpr uint32_t kPolyPairs = 0x0000C000u;
 constexpr int kQBuffers = 1;
 // S of a block read by one 128-column TMEM load per warp instead of two
 constexpr bool kWideLoad = false;
-// cycles by which the second softmax group starts after the first (0: none)
-constexpr int kGroupOffset = 500;
 constexpr int kQueue = 4;                       // item queue depth
 constexpr int kItemReaders = 32 * 3 + 256 + 128;  // threads of the roles that read the queue
 // registers per thread: launch 65536 / 512 = 128, then re-balanced per warpgroup
@@ -135,31 +133,44 @@ struct Params {
   float* mass;           //                kept attention share (nullable)
   const int32_t* out_rows;  // output row map (nullable = identity)
   int32_t* status;
+  const float* q_scale;  // FP8 Q.K^T: dequantization scale per (b, h, block) of Q and of K
+  const float* k_scale;
   int H, L, NB, NT, n_work;
   float scale_log2;
   int dense;
   int sched_slot;
 };
 
-template <int D>
+// kF8: Q and K are E4M3 (one byte per element), S = Q.K^T runs as a
+// kind::f8f6f4 MMA; V, P and O stay bf16.
+template <int D, bool kF8>
 struct Cfg {
-  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int QK_ELEM = kF8 ? 1 : 2;        // bytes per Q / K element
+  static constexpr int Q_BYTES = BM * D * QK_ELEM;
   static constexpr int NQ = kQBuffers;            // Q buffers across items
-  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int K_BYTES = BN * D * QK_ELEM;
+  static constexpr int V_BYTES = BN * D * 2;
   static constexpr int STATS_BYTES = 2 * 3 * BM * 4;  // [item parity][l, m, l_kept][row]
   static constexpr int MISC_BYTES = 512;
-  static constexpr int SLOTS = (227 * 1024 - 1024 - NQ * Q_BYTES - STATS_BYTES - MISC_BYTES) / KV_BYTES;
-  static constexpr int NSK = ((SLOTS + 1) / 2) > 4 ? 4 : (SLOTS + 1) / 2;
-  static constexpr int NSV = (SLOTS / 2) > 4 ? 4 : SLOTS / 2;
+  static constexpr int AVAIL = 227 * 1024 - 1024 - NQ * Q_BYTES - STATS_BYTES - MISC_BYTES;
+  static constexpr int SLOTS = AVAIL / V_BYTES;   // equal K and V slots (bf16)
+  static constexpr int NSK = kF8 ? 4 : (((SLOTS + 1) / 2) > 4 ? 4 : (SLOTS + 1) / 2);
+  static constexpr int NSV_FIT = kF8 ? (AVAIL - NSK * K_BYTES) / V_BYTES : SLOTS / 2;
+  static constexpr int NSV = NSV_FIT > 4 ? 4 : NSV_FIT;
   static_assert(NSK >= 2 && NSV >= 2, "shared memory too small for double-buffered K and V");
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = NQ * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
-  static constexpr int OFF_STATS = OFF_V + NSV * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + NSK * K_BYTES;
+  static constexpr int OFF_STATS = OFF_V + NSV * V_BYTES;
   static constexpr int OFF_MISC = OFF_STATS + STATS_BYTES;
   static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static constexpr int COL_S = 0;        // S[b] at b*BN
-  static constexpr int PANELS = D / 64;
+  // 128-byte rows of the swizzled tiles: Q/K panels of 64 bf16 or 128 E4M3
+  static constexpr int QK_PANEL_ELEMS = 128 / QK_ELEM;
+  static constexpr int QK_PANELS = D / QK_PANEL_ELEMS;
+  static constexpr int PANELS = D / 64;              // V panels
+  static constexpr int S_KSTEPS = D * QK_ELEM / 32;  // 32 bytes of K per MMA
 };
 
 struct Shared {
@@ -361,11 +372,11 @@ __device__ __forceinline__ bool kept_at(const Item& it, int j, int& kp, bool& ba
   return false;
 }
 
-template <int D, bool kFused>
+template <int D, bool kFused, bool kF8>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const Params prm) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kF8>;
   // TMEM (512 columns): NS buffers of S (128 columns each) then OB buffers of
   // the accumulator(s) of an item (D columns each; the fused refresh keeps two
   // per item, OK and OR).  D = 128: S0|S1|S2|O, fused S0|S1|OK|OR.
@@ -463,8 +474,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i >= C::NQ && !(ok = warp_wait(&sh->q_empty[qb], ((i - C::NQ) / C::NQ) & 1, sh, prm))) break;
         if (lane == 0) {
           mbar_arrive_expect_tx(&sh->q_full[qb], C::Q_BYTES);
-          for (int pnl = 0; pnl < C::PANELS; ++pnl)
-            tma_load_3d(q_smem + qb * C::Q_BYTES + pnl * BM * 128, &tmQ, &sh->q_full[qb], pnl * 64, it.qb * BM,
+          for (int pnl = 0; pnl < C::QK_PANELS; ++pnl)
+            tma_load_3d(q_smem + qb * C::Q_BYTES + pnl * BM * 128, &tmQ, &sh->q_full[qb], pnl * C::QK_PANEL_ELEMS,
+                        it.qb * BM,
                         it.bh);
         }
         __syncwarp();
@@ -477,9 +489,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int slot = u % NSK;
           if (u >= NSK && !(ok = warp_wait(&sh->empty_k[slot], ((u / NSK) - 1) & 1, sh, prm))) break;
           if (lane == 0) {
-            mbar_arrive_expect_tx(&sh->full_k[slot], C::KV_BYTES);
-            for (int pnl = 0; pnl < C::PANELS; ++pnl)
-              tma_load_3d(k_ring + slot * C::KV_BYTES + pnl * BN * 128, &tmK, &sh->full_k[slot], pnl * 64, kb * BN,
+            mbar_arrive_expect_tx(&sh->full_k[slot], C::K_BYTES);
+            for (int pnl = 0; pnl < C::QK_PANELS; ++pnl)
+              tma_load_3d(k_ring + slot * C::K_BYTES + pnl * BN * 128, &tmK, &sh->full_k[slot],
+                          pnl * C::QK_PANEL_ELEMS, kb * BN,
                           it.bh);
           }
           __syncwarp();
@@ -505,9 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int slot = u % NSV;
           if (u >= NSV && !(ok = warp_wait(&sh->empty_v[slot], ((u / NSV) - 1) & 1, sh, prm))) break;
           if (lane == 0) {
-            mbar_arrive_expect_tx(&sh->full_v[slot], C::KV_BYTES);
+            mbar_arrive_expect_tx(&sh->full_v[slot], C::V_BYTES);
             for (int pnl = 0; pnl < C::PANELS; ++pnl)
-              tma_load_3d(v_ring + slot * C::KV_BYTES + pnl * BN * 128, &tmV, &sh->full_v[slot], pnl * 64, kb * BN,
+              tma_load_3d(v_ring + slot * C::V_BYTES + pnl * BN * 128, &tmV, &sh->full_v[slot], pnl * 64, kb * BN,
                           it.bh);
           }
           __syncwarp();
@@ -519,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     } else if (warp == 2) {
       // ---------------------------------------------------------- S issuer
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t idS = kF8 ? idesc_e4m3_f32(BM, BN) : idesc_bf16_f32(BM, BN, false, false);
       const uint32_t q_base = smem_u32(q_smem);
       const uint32_t k_base = smem_u32(k_ring);
       int u = 0;
@@ -540,13 +553,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (u >= NS && !(ok = warp_wait(&sh->pv_done[b], ((u - NS) / NS) & 1, sh, prm))) break;
           tc_fence_after();
           if (lane == 0) {
-            const uint32_t ka = k_base + sk * C::KV_BYTES;
+            const uint32_t ka = k_base + sk * C::K_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
+            for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
               const uint32_t off_q = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
               const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-              mma_ss(tmem + C::COL_S + b * BN, sdesc_sw128(qa + off_q, 16, 1024), sdesc_sw128(ka + off_k, 16, 1024),
-                     idS, kk > 0 ? 1u : 0u);
+              if constexpr (kF8)
+                mma_ss_f8(tmem + C::COL_S + b * BN, sdesc_sw128(qa + off_q, 16, 1024),
+                          sdesc_sw128(ka + off_k, 16, 1024), idS, kk > 0 ? 1u : 0u);
+              else
+                mma_ss(tmem + C::COL_S + b * BN, sdesc_sw128(qa + off_q, 16, 1024),
+                       sdesc_sw128(ka + off_k, 16, 1024), idS, kk > 0 ? 1u : 0u);
             }
             tc_commit(&sh->s_full[b]);
             tc_commit(&sh->empty_k[sk]);
@@ -589,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const bool fresh = kept ? first : first_rest;
           if (lane == 0) {
-            const uint32_t va = v_base + sv * C::KV_BYTES;
+            const uint32_t va = v_base + sv * C::V_BYTES;
             const uint32_t dst = tmem + COL_O + (kFused ? (kept ? 0 : D) : ob * D);
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)
@@ -624,15 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int j4 = lane & 3;             // column slot within each chunk
     const int rA = quarter * 32 + grp * 16 + (lane >> 2);  // the thread's two rows: rA, rA + 8
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32 + grp * 16) << 16;
-    const float sl2 = prm.scale_log2;
-    const uint64_t scale2 = f2_pack(sl2, sl2);
-    if (kGroupOffset > 0 && grp == 1) {
-      // the second group starts later, so that the two groups' exponentials
-      // (bound by the exp unit they share) fall at different times
-      const uint64_t c0 = clock64();
-      while (clock64() - c0 < static_cast<uint64_t>(kGroupOffset)) {
-      }
-    }
+    const float sl2_base = prm.scale_log2;
     int u = 0;
     bool ok = true;
     for (int i = 0; ok; ++i) {
@@ -642,18 +651,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ob = i % OB;
       const int sb = i & 1;  // statistics buffer
       const uint32_t tO = tmem + lane_off + COL_O + ob * D;
+      // FP8: the logits of block pair (i, j) carry the scales of Q block i and K block j
+      const float sl2_item =
+          kF8 ? sl2_base * __ldg(prm.q_scale + static_cast<size_t>(it.bh) * prm.NB + it.qb) : sl2_base;
       float mA = -INFINITY, mB = -INFINITY;  // reference max of rows rA, rA+8 (log2 units)
       float lA = 0.f, lB = 0.f;              // this thread's share of the row sums
       float kA = 0.f, kB = 0.f;              // fused refresh: the same over the kept blocks
       int nt = 0;
       int kp = 0;
       bool bad = false;
+      // FP8: the K block scale of list entry n, loaded one block ahead
+      const float* ks_row = kF8 ? prm.k_scale + static_cast<size_t>(it.bh) * prm.NB : nullptr;
+      auto k_scale_at = [&](int n) {
+        const int kb = entry_kb(it, n, NB);
+        return kb >= 0 ? __ldg(ks_row + kb) : 1.f;
+      };
+      float ks_next = kF8 && it.cnt > 0 ? k_scale_at(0) : 1.f;
       for (int n = 0; n < it.cnt; ++n) {
         const int kb = entry_kb(it, n, NB);
+        float ks = 1.f;
+        if constexpr (kF8) {
+          ks = ks_next;
+          if (n + 1 < it.cnt) ks_next = k_scale_at(n + 1);
+        }
         if (kb < 0) continue;
         const bool kept = !kFused || kept_at(it, kb, kp, bad);
         const int b = u % NS;
         const uint32_t tS = tmem + lane_off + C::COL_S + b * BN;
+        const float sl2 = kF8 ? sl2_item * ks : sl2_item;
+        const uint64_t scale2 = f2_pack(sl2, sl2);
         if (!(ok = warp_wait(&sh->s_full[b], (u / NS) & 1, sh, prm))) break;
         tc_fence_after();
         // s[chunk][0..1]: row rA, keys 8*chunk + 2*j4 + {0,1}; s[chunk][2..3]: row rA+8
@@ -994,16 +1020,33 @@ bool make_map(CUtensorMap* m, const void* base, int D, int L, int BH, int box_ro
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool kFused>
+// [BH, L, D] E4M3 (raw bytes) as a 3-D tensor; box = 128 columns (128 bytes) x rows x 1.
+bool make_map8(CUtensorMap* m, const void* base, int D, int L, int BH, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L) * D};
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool kFused, bool kF8 = false>
 int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
-  using C = Cfg<D>;
-  if (smem_opt_in(reinterpret_cast<const void*>(sparse_attn_tile_kernel<D, kFused>), C::SMEM_BYTES) != cudaSuccess)
+  using C = Cfg<D, kF8>;
+  if (smem_opt_in(reinterpret_cast<const void*>(sparse_attn_tile_kernel<D, kFused, kF8>), C::SMEM_BYTES) !=
+      cudaSuccess)
     return BSA_ECUDA;
   const int BH = s.B * s.H;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.q, D, s.L, BH, BM) || !make_map(&mk, a.k, D, s.L, BH, BN) ||
-      !make_map(&mv, a.v, D, s.L, BH, BN))
+  if (kF8) {
+    if (!make_map8(&mq, a.q8, D, s.L, BH, BM) || !make_map8(&mk, a.k8, D, s.L, BH, BN)) return BSA_ECUDA;
+  } else if (!make_map(&mq, a.q, D, s.L, BH, BM) || !make_map(&mk, a.k, D, s.L, BH, BN)) {
     return BSA_ECUDA;
+  }
+  if (!make_map(&mv, a.v, D, s.L, BH, BN)) return BSA_ECUDA;
   Params prm;
   prm.kept_idx = a.kept_idx;
   prm.kept_cnt = a.kept_cnt;
@@ -1017,6 +1060,8 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   prm.mass = a.mass;
   prm.out_rows = a.out_rows;
   prm.status = a.status;
+  prm.q_scale = a.q_scale;
+  prm.k_scale = a.k_scale;
   prm.H = s.H;
   prm.L = s.L;
   prm.NB = n_blocks(s.L, s.blk);
@@ -1028,7 +1073,7 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   prm.sched_slot = static_cast<int>(launches.fetch_add(1u) % kSchedSlots);
   const int sms = sm_count();
   const int grid = prm.n_work < sms ? prm.n_work : sms;
-  sparse_attn_tile_kernel<D, kFused><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, prm);
+  sparse_attn_tile_kernel<D, kFused, kF8><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ECUDA;
 }
 
@@ -1036,6 +1081,10 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
 
 int launch_sparse_attn_tile(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   if (s.blk != 128) return BSA_ESHAPE;
+  if (a.q8) {
+    if (s.D == 128 && !a.o2) return tile_attn::run<128, false, true>(s, a, st);
+    return BSA_ESHAPE;
+  }
   if (a.o2) {
     if (s.D == 128) return tile_attn::run<128, true>(s, a, st);
     if (s.D == 64) return tile_attn::run<64, true>(s, a, st);

@@ -67,6 +67,9 @@ int launch_tail_merge(const bsa_shape& s, const float* l_S, const __nv_bfloat16*
                       const __nv_bfloat16* obar, const float* d_l, const __nv_bfloat16* d_o, __nv_bfloat16* o,
                       float* lse, cudaStream_t st);
 int launch_complement(const bsa_shape& s, const uint8_t* mask, int32_t* idx, int32_t* cnt, cudaStream_t st);
+// E4M3 codes and per-block scales of a bf16 [B,H,L,D] tensor (blocks of s.blk tokens)
+cudaError_t launch_quantize_fp8(const bsa_shape& s, const __nv_bfloat16* x, uint8_t* codes, float* scales,
+                                cudaStream_t st);
 size_t hilbert_workspace_bytes(int T, int Hh, int W);
 cudaError_t launch_hilbert(int T, int Hh, int W, int32_t* perm, int32_t* inv, void* ws, cudaStream_t st);
 cudaError_t launch_permute(const bsa_shape& s, const __nv_bfloat16* x, const int32_t* perm, __nv_bfloat16* y,
@@ -96,6 +99,13 @@ struct AttnArgs {
   // blk = 128, not the fused refresh: output row r of (b, h) goes to row
   // out_rows[r] of o and lse (nullable = identity)
   const int32_t* out_rows = nullptr;
+  // FP8 Q.K^T (blk = 128, D = 128): E4M3 codes of Q and K ([B,H,L,D] bytes) and
+  // their dequantization scales per (b, h, 128-token block); non-null q8
+  // selects it (q and k are then unused)
+  const uint8_t* q8 = nullptr;
+  const uint8_t* k8 = nullptr;
+  const float* q_scale = nullptr;
+  const float* k_scale = nullptr;
 };
 // Returns BSA_OK / BSA_ECUDA (tensor-map encoding or launch failure).
 // blk = 128: persistent one-tile-per-step kernel (attention_tile.cu);

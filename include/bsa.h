@@ -418,6 +418,40 @@ BSA_API int bsa_sparse_attn_fwd_scatter(bsa_shape s, const bsa_bf16* q, const bs
                                 int32_t* status, bsa_stream stream);
 
 /*
+ * FP8 Q.K^T.  Defines: the sparse attention of a distilled pipeline run in
+ * FP8 with fused kernels (abstract on the page titled RECAP).  The page gives
+ * no format or scaling rule; here Q and K are quantized to OCP E4M3 (max 448,
+ * round to nearest even, saturating) with one scale per (b, h, token block),
+ * the logits are (s_q * s_k) * (q8 . k8) accumulated in fp32 by the tensor
+ * cores, and the softmax, P.V (bf16 V) and the epilogue are those of
+ * bsa_sparse_attn_fwd.  The result is the block-sparse attention of the
+ * dequantized Q and K.
+ */
+
+/*
+ * bsa_quantize_fp8 -- E4M3 codes and per-block scales of a bf16 tensor.
+ *   per (b, h, block j of s.blk tokens): amax = max |x|,
+ *   scale[b,h,j] = amax / 448 (1 for an all-zero block),
+ *   codes = E4M3_rn_satfinite(x * (448 / amax))  (float32 reciprocal and product)
+ * x: bf16 [B,H,L,D]; codes: uint8 [B,H,L,D]; scales: float32 [B,H,NB].
+ * Errors: BSA_EINVAL on null or misaligned pointers; BSA_ESHAPE; BSA_ENODEV;
+ * BSA_ECUDA.
+ */
+BSA_API int bsa_quantize_fp8(bsa_shape s, const bsa_bf16* x, uint8_t* codes, float* scales, bsa_stream stream);
+
+/*
+ * bsa_sparse_attn_fwd_fp8 -- bsa_sparse_attn_fwd with S = Q.K^T from E4M3
+ * codes (kind::f8f6f4 tensor-core MMAs).  q8/q_scale and k8/k_scale as
+ * bsa_quantize_fp8 writes them (blocks of 128 tokens); v, kept lists, R/alpha,
+ * o, lse and status as bsa_sparse_attn_fwd.  s.blk and s.D must be 128.
+ * Errors: as bsa_sparse_attn_fwd; BSA_ESHAPE for another blk or D.
+ */
+BSA_API int bsa_sparse_attn_fwd_fp8(bsa_shape s, const uint8_t* q8, const float* q_scale, const uint8_t* k8,
+                                    const float* k_scale, const bsa_bf16* v, const int32_t* kept_idx,
+                                    const int32_t* kept_cnt, const bsa_bf16* R, const float* alpha, bsa_bf16* o,
+                                    float* lse, int32_t* status, bsa_stream stream);
+
+/*
  * bsa_refresh_refinement -- renew the cached refinement at a dense refresh.
  * Defines: the refinement cached at a dense refresh and renewed only there
  * (RECAP, sections 1, 3.4 and 4.3).
