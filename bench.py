@@ -43,7 +43,10 @@ from block_sparse_attention_logits_b200.synthetic import make_qkv, random_bf16  
 
 METRIC = "block-sparse attn ms/call & TFLOP/s on kept blocks vs bf16 TC peak at 90% sparsity"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 5  # pooling with the Q/K gather, block softmax, selection, V gather, attention (O in grid order)
+# launches of this library per step: pooling (with the Q/K gather into curve
+# order), block softmax, selection, attention (O in grid order); the
+# reordered-copies form adds the V gather
+LAUNCHES_PER_STEP = 4
 E2E_MAX_CHUNKS = 8     # head chunks of the pipelined end-to-end step
 
 
@@ -63,6 +66,9 @@ def parse_args():
     ap.add_argument("--no-refresh", action="store_true",
                     help="skip the dense-refresh, mask-reuse, elementwise and sweep timings")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--gather", action="store_true",
+                    help="Hilbert workloads: the attention gathers its tiles from the grid-order tensors "
+                         "(no reordered copies; 4-row TMA gathers, slower) instead of reading reordered copies")
     ap.add_argument("--shard", choices=["heads", "replicas"], default="heads",
                     help="N > 1: split the workload's heads over the ranks (strong scaling, the default) or run "
                          "one full replica per rank (weak scaling)")
@@ -393,20 +399,23 @@ def run_ours(args, w, world, rank, local):
     host = {n: torch.empty((B, H, L, D), dtype=torch.bfloat16, pin_memory=pin) for n in ("q", "k", "v")}
     make_qkv(B, H, w.grid, D, w.fp, out=host, h0=h_lo)
     q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
-    R_h = random_bf16((B, H, L, D), 99 + h_lo, scale=0.05).to(dev)  # cached refinement (curve order)
+    # cached refinement: in grid order when the attention gathers its tiles,
+    # in curve order when it reads reordered copies
+    R_h = random_bf16((B, H, L, D), 99 + h_lo, scale=0.05).to(dev)
     alpha = torch.tensor(w.alpha()[h_lo:h_hi], dtype=torch.float32, device=dev)
     strong = args.shard == "heads" and world > 1
 
     perm = api.reorder_tokens(*w.grid, device=dev)[0] if w.hilbert else None
+    gather = w.hilbert and args.gather
     nb = api.n_blocks(L, blk)
-    bufs = alloc_buffers(B, H, L, D, blk, dev)
+    bufs = alloc_buffers(B, H, L, D, blk, dev, copies=not gather)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def path(b, qi, ki, vi, Ri, ai, events=None):
         """One pass of the hot path on buffers `b` (the full set or one head
-        chunk): Hilbert gathers, scoring, selection, sparse attention with the
+        chunk): scoring in Hilbert order, selection, sparse attention with the
         fused correction, output in grid order."""
-        return run_step(b, qi, ki, vi, blk, p, perm, Ri, ai, status, events)
+        return run_step(b, qi, ki, vi, blk, p, perm, Ri, ai, status, events, gather=gather)
 
     def step(qi, ki, vi, events=None):
         return path(bufs, qi, ki, vi, R_h, alpha, events)
@@ -468,7 +477,7 @@ def run_ours(args, w, world, rank, local):
             # token-row buffers are head slices (16-byte aligned offsets); the
             # per-block score and list buffers get their own allocations (an
             # [NB, NB] slice of an odd NB is not 16-byte aligned)
-            chunk_bufs.append({n: (t[:, hs] if n in ("qh", "kh", "vh", "oh", "o", "lse") else
+            chunk_bufs.append({n: (None if t is None else t[:, hs] if n in ("qh", "kh", "vh", "oh", "o", "lse") else
                                    torch.empty_like(t[:, hs])) for n, t in bufs.items()})
 
         def chunk_step(c, qi, ki, vi):
@@ -517,6 +526,11 @@ def run_ours(args, w, world, rank, local):
                "ms_per_step": round(e_ms / Ke, 3), "steps": Ke,
                "pipeline": f"{n_chunks} head chunks on 3 streams (copy-in, compute, copy-out)",
                "h2d_bytes_per_step": 3 * B * H * L * D * 2, "d2h_bytes_per_step": B * H * L * D * 2 + B * H * L * 4}
+
+    # the calls below run on the curve-order tensors: with gathered tiles the
+    # step made no copies, so make them here, outside every timed region
+    if gather and not args.no_refresh:
+        bufs["qh"], bufs["kh"], bufs["vh"] = (api.permute_tokens(x, perm) for x in (q, k, v))
 
     # dense refresh on the same inputs and kept lists: the single-pass call
     # against the two-pass path (dense call, sparse call, refinement)
@@ -654,6 +668,7 @@ def run_ours(args, w, world, rank, local):
             sb = dict(o_dense=torch.empty_like(q), o_sparse=torch.empty_like(q), R=Rs,
                       lse_dense=torch.empty((B, H, L), dtype=torch.float32, device=dev),
                       lse_sparse=torch.empty((B, H, L), dtype=torch.float32, device=dev))
+            Rg = torch.zeros_like(q)  # the refinement in grid order, for the gathering attention
             steps_ms, kinds = [], []
             for st_ in range(10):
                 if st_ > 0:
@@ -663,21 +678,33 @@ def run_ours(args, w, world, rank, local):
                 a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a0.record()
                 b_ = bufs
+                refresh_step = st_ % 5 == 0
+                # the refresh runs on reordered copies; sparse steps gather their tiles
+                copies = refresh_step or not gather
                 if st_ % 3 == 0:
-                    api.score_blocks_gather(qd_, kd_, perm, blk, b_["qh"], b_["kh"], b_["qp"], b_["kp"], b_["probs"])
+                    api.score_blocks_gather(qd_, kd_, perm, blk, b_["qh"] if copies else None,
+                                            b_["kh"] if copies else None, b_["qp"], b_["kp"], b_["probs"],
+                                            copies=copies)
                     api.select_topp_mask(b_["probs"], p, L, blk, D, b_["mask"], b_["idx"], b_["cnt"])
-                else:
+                elif copies:
                     api.permute_tokens(qd_, perm, out=b_["qh"])
                     api.permute_tokens(kd_, perm, out=b_["kh"])
-                api.permute_tokens(v, perm, out=b_["vh"])
-                if st_ % 5 == 0:
+                if copies:
+                    api.permute_tokens(v, perm, out=b_["vh"])
+                if refresh_step:
                     api.sparse_attn_refresh(b_["qh"], b_["kh"], b_["vh"], blk, b_["idx"], b_["cnt"], want_mass=False,
                                             out=sb, status=status)
                     api.permute_tokens(sb["o_dense"], perm, inverse=True, out=b_["o"])
+                    if gather:
+                        api.permute_tokens(Rs, perm, inverse=True, out=Rg)
                     kinds.append("refresh")
                 else:
-                    api.sparse_attn_fwd(b_["qh"], b_["kh"], b_["vh"], blk, b_["idx"], b_["cnt"], Rs, alpha, b_["o"],
-                                        b_["lse"], status=status, out_rows=perm)
+                    if gather:
+                        api.sparse_attn_fwd(qd_, kd_, v, blk, b_["idx"], b_["cnt"], Rg, alpha, b_["o"], b_["lse"],
+                                            status=status, in_rows=perm)
+                    else:
+                        api.sparse_attn_fwd(b_["qh"], b_["kh"], b_["vh"], blk, b_["idx"], b_["cnt"], Rs, alpha,
+                                            b_["o"], b_["lse"], status=status, out_rows=perm)
                     kinds.append("sparse+mask" if st_ % 3 == 0 else "sparse, mask reused")
                 a1.record()
                 barrier()
@@ -714,7 +741,10 @@ def run_ours(args, w, world, rank, local):
         "scaling": "strong" if strong else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": B, "H": w.H, "L": L, "D": D, "blk": blk, "grid": list(w.grid),
-                   "hilbert": w.hilbert, "top_p": p, "block_sparsity": round(sparsity, 4),
+                   "hilbert": w.hilbert,
+                   "reorder": ("attention tiles gathered from the grid-order tensors" if gather else
+                               "reordered copies of Q, K, V" if w.hilbert else "none"),
+                   "top_p": p, "block_sparsity": round(sparsity, 4),
                    "fused_correction": True, "kept_tflop_per_step": round(job_flops / 1e12, 4),
                    "l2": f"inputs larger than L2 (Q/K/V {3 * B * H * L * D * 2 / 1e9:.2f} GB per step per GPU), "
                          "no flush",
@@ -728,7 +758,7 @@ def run_ours(args, w, world, rank, local):
                       "rest": round(ms_step - attn_avg_ms - float(np.mean(sel_ms)), 4)},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "refresh": refresh, "reuse": reuse,
         "elementwise": elementwise, "sweep": sweep, "intervals": intervals, "tail": tail, "fp8": fp8,
-        "gpu_launches": LAUNCHES_PER_STEP * K if w.hilbert else (LAUNCHES_PER_STEP - 1) * K,
+        "gpu_launches": (LAUNCHES_PER_STEP + (1 if w.hilbert and not gather else 0)) * K,
         "clocks": clk,
     }
     if world > 1:

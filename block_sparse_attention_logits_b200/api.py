@@ -107,22 +107,29 @@ def score_blocks(q, k, blk, q_pool=None, k_pool=None, probs=None, candidates=Non
     return q_pool, k_pool, probs
 
 
-def score_blocks_gather(q, k, perm, blk, q_out=None, k_out=None, q_pool=None, k_pool=None, probs=None):
+def score_blocks_gather(q, k, perm, blk, q_out=None, k_out=None, q_pool=None, k_pool=None, probs=None,
+                        copies=True):
     """permute_tokens(q), permute_tokens(k) and score_blocks of the results in
-    one pass.  Returns (q_out, k_out, q_pool, k_pool, probs)."""
+    one pass.  Returns (q_out, k_out, q_pool, k_pool, probs); with
+    copies=False the reordered q and k are not written (q_out = k_out = None),
+    for sparse_attn_fwd(..., in_rows=perm)."""
     B, H, L, D = q.shape
     nb = n_blocks(L, blk)
     _need(q, torch.bfloat16, (B, H, L, D), "q")
     _need(k, torch.bfloat16, (B, H, L, D), "k")
     _need(perm, torch.int32, (L,), "perm")
     dev = q.device
-    q_out = q_out if q_out is not None else torch.empty_like(q)
-    k_out = k_out if k_out is not None else torch.empty_like(k)
+    if copies:
+        q_out = q_out if q_out is not None else torch.empty_like(q)
+        k_out = k_out if k_out is not None else torch.empty_like(k)
+    else:
+        q_out = k_out = None
     q_pool = q_pool if q_pool is not None else torch.empty((B, H, nb, D), dtype=torch.float32, device=dev)
     k_pool = k_pool if k_pool is not None else torch.empty((B, H, nb, D), dtype=torch.float32, device=dev)
     probs = probs if probs is not None else torch.empty((B, H, nb, nb), dtype=torch.float32, device=dev)
-    for name, t in (("q_out", q_out), ("k_out", k_out)):
-        _need(t, torch.bfloat16, (B, H, L, D), name)
+    if copies:
+        for name, t in (("q_out", q_out), ("k_out", k_out)):
+            _need(t, torch.bfloat16, (B, H, L, D), name)
     _need(q_pool, torch.float32, (B, H, nb, D), "q_pool")
     _need(k_pool, torch.float32, (B, H, nb, D), "k_pool")
     _need(probs, torch.float32, (B, H, nb, nb), "probs")
@@ -433,13 +440,16 @@ def permute_tokens(x, perm, inverse=False, out=None):
 
 
 def sparse_attn_fwd(q, k, v, blk, kept_idx=None, kept_cnt=None, R=None, alpha=None,
-                    o=None, lse=None, status=None, out_rows=None):
+                    o=None, lse=None, status=None, out_rows=None, in_rows=None):
     """Block-sparse attention over the kept blocks (dense when kept_* are None).
 
     Returns (o bf16 [B,H,L,D], lse float32 [B,H,L]).  With R / alpha the
     epilogue adds alpha_h * R.  `status` (int32 [1] on the device, zeroed by
     the caller) receives BSA_DEV_* bits.  With `out_rows` (int32 [L], a
     permutation; blk 128) output row r goes to row out_rows[r] of o and lse.
+    With `in_rows` (int32 [L], a permutation; blk = D = 128) the attention
+    runs over the tokens in that order with q, k, v, R, o and lse all in the
+    caller's order: token t is row in_rows[t] (bsa_sparse_attn_fwd_gather).
     """
     B, H, L, D = q.shape
     nb = n_blocks(L, blk)
@@ -457,7 +467,14 @@ def sparse_attn_fwd(q, k, v, blk, kept_idx=None, kept_cnt=None, R=None, alpha=No
     _need(lse, torch.float32, (B, H, L), "lse")
     if status is not None:
         _need(status, torch.int32, (1,), "status")
-    if out_rows is None:
+    if in_rows is not None:
+        if out_rows is not None:
+            raise ValueError("in_rows writes the output through the same rows: pass no out_rows")
+        _need(in_rows, torch.int32, (L,), "in_rows")
+        check("bsa_sparse_attn_fwd_gather", _lib.load().bsa_sparse_attn_fwd_gather(
+            Shape(B, H, L, D, blk), _ptr(q), _ptr(k), _ptr(v), _ptr(in_rows), _ptr(kept_idx), _ptr(kept_cnt),
+            _ptr(R), _ptr(alpha), _ptr(o), _ptr(lse), _ptr(status), _stream()))
+    elif out_rows is None:
         check("bsa_sparse_attn_fwd", _lib.load().bsa_sparse_attn_fwd(
             Shape(B, H, L, D, blk), _ptr(q), _ptr(k), _ptr(v), _ptr(kept_idx), _ptr(kept_cnt),
             _ptr(R), _ptr(alpha), _ptr(o), _ptr(lse), _ptr(status), _stream()))

@@ -96,11 +96,12 @@ int bsa_score_blocks_restricted(bsa_shape s, const bsa_bf16* q, const bsa_bf16* 
 
 int bsa_score_blocks_gather(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const int32_t* perm, bsa_bf16* q_out,
                             bsa_bf16* k_out, float* q_pool, float* k_pool, float* probs, bsa_stream stream) {
-  if (!q || !k || !perm || !q_out || !k_out || !q_pool || !k_pool || !probs) return BSA_EINVAL;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(perm) || !aligned16(q_out) || !aligned16(k_out) ||
-      !aligned16(q_pool) || !aligned16(k_pool) || !aligned16(probs))
+  if (!q || !k || !perm || !q_pool || !k_pool || !probs) return BSA_EINVAL;
+  if ((q_out == nullptr) != (k_out == nullptr)) return BSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(perm) || (q_out && !aligned16(q_out)) ||
+      (k_out && !aligned16(k_out)) || !aligned16(q_pool) || !aligned16(k_pool) || !aligned16(probs))
     return BSA_EINVAL;
-  if (q_out == q || q_out == k || k_out == q || k_out == k || q_out == k_out) return BSA_EINVAL;
+  if (q_out && (q_out == q || q_out == k || k_out == q || k_out == k || q_out == k_out)) return BSA_EINVAL;
   if (int r = check_block_shape(s)) return r;
   if (int r = check_device()) return r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -354,6 +355,38 @@ int bsa_sparse_attn_fwd_scatter(bsa_shape s, const bsa_bf16* q, const bsa_bf16* 
   a.lse = lse;
   a.status = status;
   a.out_rows = out_rows;
+  return bsa::launch_sparse_attn(s, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bsa_sparse_attn_fwd_gather(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
+                               const int32_t* rows, const int32_t* kept_idx, const int32_t* kept_cnt,
+                               const bsa_bf16* R, const float* alpha, bsa_bf16* o, float* lse, int32_t* status,
+                               bsa_stream stream) {
+  if (!q || !k || !v || !rows || !o || !lse) return BSA_EINVAL;
+  if ((kept_idx == nullptr) != (kept_cnt == nullptr)) return BSA_EINVAL;
+  if ((R == nullptr) != (alpha == nullptr)) return BSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(rows))
+    return BSA_EINVAL;
+  if ((kept_idx && !aligned16(kept_idx)) || (kept_cnt && !aligned16(kept_cnt)) || (R && !aligned16(R)))
+    return BSA_EINVAL;
+  if (!word_ok(status) || !word_ok(alpha)) return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (s.blk != 128 || s.D != 128) return BSA_ESHAPE;
+  if (static_cast<long long>(s.B) * s.H * s.L >= (1ll << 31)) return BSA_ESHAPE;
+  if (int r = check_device()) return r;
+  bsa::AttnArgs a;
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  a.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  a.kept_idx = kept_idx;
+  a.kept_cnt = kept_cnt;
+  a.R = reinterpret_cast<const __nv_bfloat16*>(R);
+  a.alpha = alpha;
+  a.o = reinterpret_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.status = status;
+  a.in_rows = rows;
+  a.out_rows = rows;
   return bsa::launch_sparse_attn(s, a, reinterpret_cast<cudaStream_t>(stream));
 }
 

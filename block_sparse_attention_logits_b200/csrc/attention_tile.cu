@@ -135,7 +135,9 @@ struct Params {
   int32_t* status;
   const float* q_scale;  // FP8 Q.K^T: dequantization scale per (b, h, block) of Q and of K
   const float* k_scale;
+  const int32_t* in_rows;  // row gathers: token t is row in_rows[t] of q, k, v
   int H, L, NB, NT, n_work;
+  int n_rows;              // B * H * L: the first row past q, k, v (reads zeros)
   float scale_log2;
   int dense;
   int sched_slot;
@@ -372,11 +374,41 @@ __device__ __forceinline__ bool kept_at(const Item& it, int j, int& kp, bool& ba
   return false;
 }
 
-template <int D, bool kFused, bool kF8>
+// Row gathers: the 128 tokens t0..t0+127 of the attention's order, rows
+// in_rows[t] of (b, h) = it.bh, as two 64-column panels of a 128-row tile at
+// dst (the layout a tiled load gives).  Lane l fetches tokens 4l..4l+3 with one
+// 4-row gather per panel; tokens past L and rows outside [0, L) read zeros
+// (the latter also flagged).  The caller has set the barrier's byte count.
+__device__ __forceinline__ void gather_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int bh, int t0,
+                                            int lane, const Params& prm) {
+  const int t = t0 + 4 * lane;
+  int g[4];
+  if (t + 4 <= prm.L) {
+    const int4 v = __ldg(reinterpret_cast<const int4*>(prm.in_rows + t));
+    g[0] = v.x, g[1] = v.y, g[2] = v.z, g[3] = v.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) g[e] = t + e < prm.L ? __ldg(prm.in_rows + t + e) : -1;
+  }
+  bool bad = false;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const bool in = static_cast<unsigned>(g[e]) < static_cast<unsigned>(prm.L);
+    bad |= !in && t + e < prm.L;
+    g[e] = in ? bh * prm.L + g[e] : prm.n_rows;
+  }
+  if (bad) flag_status(prm, BSA_DEV_BAD_INDEX);
+#pragma unroll
+  for (int pnl = 0; pnl < 2; ++pnl)
+    tma_gather4(dst + pnl * (BM * 128) + lane * 512, map, bar, pnl * 64, g[0], g[1], g[2], g[3]);
+}
+
+template <int D, bool kFused, bool kF8, bool kGather>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const Params prm) {
   using C = Cfg<D, kF8>;
+  static_assert(!kGather || (D == 128 && !kFused && !kF8), "row gathers: bf16, D = 128, not the fused refresh");
   // TMEM (512 columns): NS buffers of S (128 columns each) then OB buffers of
   // the accumulator(s) of an item (D columns each; the fused refresh keeps two
   // per item, OK and OR).  D = 128: S0|S1|S2|O, fused S0|S1|OK|OR.
@@ -472,7 +504,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it.bad_cnt && lane == 0) flag_status(prm, BSA_DEV_BAD_INDEX);
         const int qb = i % C::NQ;
         if (i >= C::NQ && !(ok = warp_wait(&sh->q_empty[qb], ((i - C::NQ) / C::NQ) & 1, sh, prm))) break;
-        if (lane == 0) {
+        if constexpr (kGather) {
+          if (lane == 0) mbar_arrive_expect_tx(&sh->q_full[qb], C::Q_BYTES);
+          __syncwarp();
+          gather_tile(q_smem + qb * C::Q_BYTES, &tmQ, &sh->q_full[qb], it.bh, it.qb * BM, lane, prm);
+        } else if (lane == 0) {
           mbar_arrive_expect_tx(&sh->q_full[qb], C::Q_BYTES);
           for (int pnl = 0; pnl < C::QK_PANELS; ++pnl)
             tma_load_3d(q_smem + qb * C::Q_BYTES + pnl * BM * 128, &tmQ, &sh->q_full[qb], pnl * C::QK_PANEL_ELEMS,
@@ -488,7 +524,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int slot = u % NSK;
           if (u >= NSK && !(ok = warp_wait(&sh->empty_k[slot], ((u / NSK) - 1) & 1, sh, prm))) break;
-          if (lane == 0) {
+          if constexpr (kGather) {
+            if (lane == 0) mbar_arrive_expect_tx(&sh->full_k[slot], C::K_BYTES);
+            __syncwarp();
+            gather_tile(k_ring + slot * C::K_BYTES, &tmK, &sh->full_k[slot], it.bh, kb * BN, lane, prm);
+          } else if (lane == 0) {
             mbar_arrive_expect_tx(&sh->full_k[slot], C::K_BYTES);
             for (int pnl = 0; pnl < C::QK_PANELS; ++pnl)
               tma_load_3d(k_ring + slot * C::K_BYTES + pnl * BN * 128, &tmK, &sh->full_k[slot],
@@ -517,7 +557,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kb < 0) continue;
           const int slot = u % NSV;
           if (u >= NSV && !(ok = warp_wait(&sh->empty_v[slot], ((u / NSV) - 1) & 1, sh, prm))) break;
-          if (lane == 0) {
+          if constexpr (kGather) {
+            if (lane == 0) mbar_arrive_expect_tx(&sh->full_v[slot], C::V_BYTES);
+            __syncwarp();
+            gather_tile(v_ring + slot * C::V_BYTES, &tmV, &sh->full_v[slot], it.bh, kb * BN, lane, prm);
+          } else if (lane == 0) {
             mbar_arrive_expect_tx(&sh->full_v[slot], C::V_BYTES);
             for (int pnl = 0; pnl < C::PANELS; ++pnl)
               tma_load_3d(v_ring + slot * C::V_BYTES + pnl * BN * 128, &tmV, &sh->full_v[slot], pnl * 64, kb * BN,
@@ -944,7 +988,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = l > 0.f ? __uint_as_float(regs[e]) * inv_l : 0.f;
             if (prm.R) {
-              const uint4* rp = reinterpret_cast<const uint4*>(prm.R + row_elem + cc * 32);
+              // R follows q, k, v; with row gathers, the order of o
+              const uint4* rp = reinterpret_cast<const uint4*>(prm.R + (kGather ? out_elem : row_elem) + cc * 32);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const uint4 rv = __ldg(rp + q);
@@ -1020,6 +1065,20 @@ bool make_map(CUtensorMap* m, const void* base, int D, int L, int BH, int box_ro
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [BH * L, D] bf16 as a 2-D tensor whose box is one row of 64 columns, for
+// 4-row gathers.
+bool make_map_rows(CUtensorMap* m, const void* base, int D, long long rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [BH, L, D] E4M3 (raw bytes) as a 3-D tensor; box = 128 columns (128 bytes) x rows x 1.
 bool make_map8(CUtensorMap* m, const void* base, int D, int L, int BH, int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
@@ -1033,20 +1092,26 @@ bool make_map8(CUtensorMap* m, const void* base, int D, int L, int BH, int box_r
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool kFused, bool kF8 = false>
+template <int D, bool kFused, bool kF8 = false, bool kGather = false>
 int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   using C = Cfg<D, kF8>;
-  if (smem_opt_in(reinterpret_cast<const void*>(sparse_attn_tile_kernel<D, kFused, kF8>), C::SMEM_BYTES) !=
+  if (smem_opt_in(reinterpret_cast<const void*>(sparse_attn_tile_kernel<D, kFused, kF8, kGather>), C::SMEM_BYTES) !=
       cudaSuccess)
     return BSA_ECUDA;
   const int BH = s.B * s.H;
+  const long long n_rows = static_cast<long long>(BH) * s.L;
+  if (kGather && n_rows >= (1ll << 31)) return BSA_ESHAPE;  // row coordinates are int32
   CUtensorMap mq, mk, mv;
-  if (kF8) {
+  if (kGather) {
+    if (!make_map_rows(&mq, a.q, D, n_rows) || !make_map_rows(&mk, a.k, D, n_rows) ||
+        !make_map_rows(&mv, a.v, D, n_rows))
+      return BSA_ECUDA;
+  } else if (kF8) {
     if (!make_map8(&mq, a.q8, D, s.L, BH, BM) || !make_map8(&mk, a.k8, D, s.L, BH, BN)) return BSA_ECUDA;
   } else if (!make_map(&mq, a.q, D, s.L, BH, BM) || !make_map(&mk, a.k, D, s.L, BH, BN)) {
     return BSA_ECUDA;
   }
-  if (!make_map(&mv, a.v, D, s.L, BH, BN)) return BSA_ECUDA;
+  if (!kGather && !make_map(&mv, a.v, D, s.L, BH, BN)) return BSA_ECUDA;
   Params prm;
   prm.kept_idx = a.kept_idx;
   prm.kept_cnt = a.kept_cnt;
@@ -1062,6 +1127,8 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   prm.status = a.status;
   prm.q_scale = a.q_scale;
   prm.k_scale = a.k_scale;
+  prm.in_rows = a.in_rows;
+  prm.n_rows = static_cast<int>(n_rows < (1ll << 31) ? n_rows : 0);
   prm.H = s.H;
   prm.L = s.L;
   prm.NB = n_blocks(s.L, s.blk);
@@ -1073,7 +1140,7 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   prm.sched_slot = static_cast<int>(launches.fetch_add(1u) % kSchedSlots);
   const int sms = sm_count();
   const int grid = prm.n_work < sms ? prm.n_work : sms;
-  sparse_attn_tile_kernel<D, kFused, kF8><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, prm);
+  sparse_attn_tile_kernel<D, kFused, kF8, kGather><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ECUDA;
 }
 
@@ -1081,6 +1148,10 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
 
 int launch_sparse_attn_tile(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   if (s.blk != 128) return BSA_ESHAPE;
+  if (a.in_rows) {
+    if (s.D == 128 && !a.o2 && !a.q8) return tile_attn::run<128, false, false, true>(s, a, st);
+    return BSA_ESHAPE;
+  }
   if (a.q8) {
     if (s.D == 128 && !a.o2) return tile_attn::run<128, false, true>(s, a, st);
     return BSA_ESHAPE;

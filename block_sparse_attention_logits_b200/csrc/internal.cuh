@@ -99,6 +99,10 @@ struct AttnArgs {
   // blk = 128, not the fused refresh: output row r of (b, h) goes to row
   // out_rows[r] of o and lse (nullable = identity)
   const int32_t* out_rows = nullptr;
+  // blk = 128, bf16, not the fused refresh: token t of the attention's order
+  // is row in_rows[t] of q, k and v (loaded by row gathers), and R is read in
+  // the order of o (nullable = q, k, v already in the attention's order)
+  const int32_t* in_rows = nullptr;
   // FP8 Q.K^T (blk = 128, D = 128): E4M3 codes of Q and K ([B,H,L,D] bytes) and
   // their dequantization scales per (b, h, 128-token block); non-null q8
   // selects it (q and k are then unused)

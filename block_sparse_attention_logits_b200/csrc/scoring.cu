@@ -9,7 +9,8 @@
 //   softmax: one CTA per (64 query blocks, head); pooled means staged
 //            transposed in shared memory, a 4x4 register tile of logits per
 //            thread, raw logits written to `probs`, then each warp
-//            normalises its rows in place.
+//            normalises its rows in place: a row of up to 1024 blocks is read
+//            once into registers (every load in flight), P written once.
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
@@ -27,7 +28,8 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& v) {
 }
 
 // With `perm` (gathering form) token t of the block is row perm[t] of the
-// input, and the gathered rows are also written to q_out / k_out in order.
+// input, and the gathered rows are also written to q_out / k_out in order
+// (when given).
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k, float* __restrict__ qp,
@@ -48,12 +50,19 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (perm) {
     const uint4* src = reinterpret_cast<const uint4*>(x + bh * L * D) + c;
-    uint4* dst = reinterpret_cast<uint4*>((blockIdx.z ? k_out : q_out) + (bh * L + t0) * D) + c;
+    __nv_bfloat16* copy = blockIdx.z ? k_out : q_out;
+    if (copy) {
+      uint4* dst = reinterpret_cast<uint4*>(copy + (bh * L + t0) * D) + c;
 #pragma unroll 4
-    for (int row = r; row < n; row += RPI) {
-      const uint4 v = __ldg(src + static_cast<size_t>(__ldg(perm + t0 + row)) * TPR);
-      dst[static_cast<size_t>(row) * TPR] = v;
-      add_bf16x8(acc, v);
+      for (int row = r; row < n; row += RPI) {
+        const uint4 v = __ldg(src + static_cast<size_t>(__ldg(perm + t0 + row)) * TPR);
+        dst[static_cast<size_t>(row) * TPR] = v;
+        add_bf16x8(acc, v);
+      }
+    } else {
+#pragma unroll 4
+      for (int row = r; row < n; row += RPI)
+        add_bf16x8(acc, __ldg(src + static_cast<size_t>(__ldg(perm + t0 + row)) * TPR));
     }
   } else {
     const uint4* base = reinterpret_cast<const uint4*>(x + (bh * L + t0) * D) + c;
@@ -79,8 +88,8 @@ constexpr int kPad = 68;    // row pitch (floats) of the transposed tiles: 16-by
 // thread a 4x4 register tile (two 16-byte shared loads per 16 FMAs); raw
 // scaled logits go to `probs`, then each warp normalises 8 of the strip's rows
 // in place (max, exp and sum, divide).
-template <int D>
-__global__ void __launch_bounds__(256) block_softmax_kernel(const float* __restrict__ qp,
+template <int D, int PER>
+__global__ void __launch_bounds__(256, 3) block_softmax_kernel(const float* __restrict__ qp,
                                                             const float* __restrict__ kp, float* __restrict__ probs,
                                                             const uint8_t* __restrict__ cand, int NB, float scale) {
   extern __shared__ __align__(16) float sm[];
@@ -134,6 +143,41 @@ __global__ void __launch_bounds__(256) block_softmax_kernel(const float* __restr
   __syncthreads();
   // row softmax: warp w normalises rows w, w+8, ...
   const int w = tid >> 5, lane = tid & 31;
+  if constexpr (PER > 0) {
+    // the row in registers: one read and one write per element
+    for (int rr = w; rr < kTile; rr += 8) {
+      const int i = i0 + rr;
+      if (i >= NB) break;
+      float* row = probs + (bh * NB + i) * NB;
+      const uint8_t* crow = cand ? cand + (bh * NB + i) * NB : nullptr;
+      float x[PER];
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const int j = lane + 32 * e;
+        x[e] = (j < NB && (!crow || crow[j])) ? row[j] : -INFINITY;
+      }
+      float m = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) m = fmaxf(m, x[e]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float sum = 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        x[e] = x[e] == -INFINITY ? 0.f : expf(x[e] - m);
+        sum += x[e];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      // a row without candidates (sum 0) stays all zeros
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const int j = lane + 32 * e;
+        if (j < NB) row[j] = sum > 0.f ? x[e] / sum : 0.f;
+      }
+    }
+    return;
+  }
   for (int rr = w; rr < kTile; rr += 8) {
     const int i = i0 + rr;
     if (i >= NB) break;
@@ -210,21 +254,37 @@ cudaError_t launch_pool(const bsa_shape& s, const __nv_bfloat16* q, const __nv_b
   return cudaGetLastError();
 }
 
+namespace {
+
+// PER: values of a row per lane in the register row pass (0: rows longer
+// than 1024 blocks, three passes over the row in `probs`)
+template <int D, int PER>
+cudaError_t launch_softmax(dim3 grid, const float* qp, const float* kp, float* probs, const uint8_t* cand, int NB,
+                           float scale, cudaStream_t st) {
+  // 69.6 KB of transposed tiles at D = 128: above the default 48 KB
+  constexpr size_t smem = 2 * D * kPad * 4;
+  if (cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(block_softmax_kernel<D, PER>), smem)) return e;
+  block_softmax_kernel<D, PER><<<grid, 256, smem, st>>>(qp, kp, probs, cand, NB, scale);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_block_softmax(const bsa_shape& s, const float* qp, const float* kp, float* probs,
                                  const uint8_t* cand, cudaStream_t st) {
   const int NB = n_blocks(s.L, s.blk);
   dim3 grid((NB + kTile - 1) / kTile, s.B * s.H);
   const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(s.D)));
-  // 69.6 KB of transposed tiles at D = 128: above the default 48 KB
-  if (cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(block_softmax_kernel<128>), 2 * 128 * kPad * 4))
-    return e;
-  if (cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(block_softmax_kernel<64>), 2 * 64 * kPad * 4))
-    return e;
-  if (s.D == 128)
-    block_softmax_kernel<128><<<grid, 256, 2 * 128 * kPad * 4, st>>>(qp, kp, probs, cand, NB, scale);
-  else
-    block_softmax_kernel<64><<<grid, 256, 2 * 64 * kPad * 4, st>>>(qp, kp, probs, cand, NB, scale);
-  return cudaGetLastError();
+  if (s.D == 128) {
+    if (NB <= 256) return launch_softmax<128, 8>(grid, qp, kp, probs, cand, NB, scale, st);
+    if (NB <= 640) return launch_softmax<128, 20>(grid, qp, kp, probs, cand, NB, scale, st);
+    if (NB <= 1024) return launch_softmax<128, 32>(grid, qp, kp, probs, cand, NB, scale, st);
+    return launch_softmax<128, 0>(grid, qp, kp, probs, cand, NB, scale, st);
+  }
+  if (NB <= 256) return launch_softmax<64, 8>(grid, qp, kp, probs, cand, NB, scale, st);
+  if (NB <= 640) return launch_softmax<64, 20>(grid, qp, kp, probs, cand, NB, scale, st);
+  if (NB <= 1024) return launch_softmax<64, 32>(grid, qp, kp, probs, cand, NB, scale, st);
+  return launch_softmax<64, 0>(grid, qp, kp, probs, cand, NB, scale, st);
 }
 
 cudaError_t launch_drift(const bsa_shape& s, const float* qp_ref, const float* kp_ref, const float* qp,

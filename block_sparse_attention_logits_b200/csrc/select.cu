@@ -45,10 +45,17 @@ __device__ __forceinline__ uint64_t fixed_mass(uint32_t key) {
   return (-sh >= 24) ? 0ull : (m >> (-sh));
 }
 
+// Exact warp sum of per-lane masses below 2^53 (a row's total is at most
+// 2^52): three 21-bit limbs, each summed by one redux over 32 lanes (limb sums
+// stay below 2^26), then recombined.
 __device__ __forceinline__ uint64_t warp_sum(uint64_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+  const uint32_t l0 = static_cast<uint32_t>(v) & 0x1FFFFFu;
+  const uint32_t l1 = static_cast<uint32_t>(v >> 21) & 0x1FFFFFu;
+  const uint32_t l2 = static_cast<uint32_t>(v >> 42);
+  const uint64_t s0 = __reduce_add_sync(0xffffffffu, l0);
+  const uint64_t s1 = __reduce_add_sync(0xffffffffu, l1);
+  const uint64_t s2 = __reduce_add_sync(0xffffffffu, l2);
+  return s0 + (s1 << 21) + (s2 << 42);
 }
 
 __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ probs, const __grid_constant__ TopP tp,
@@ -252,10 +259,10 @@ __global__ void __launch_bounds__(256) select_reg_kernel(const float* __restrict
 #pragma unroll 1
     for (int b = 30; b >= 0; --b) {
       const uint32_t c = tau | (1u << b);
-      uint64_t g = 0;
+      uint64_t g[4] = {0ull, 0ull, 0ull, 0ull};  // independent partial sums
 #pragma unroll
-      for (int r = 0; r < R; ++r) g += key[r] >= c ? u[r] : 0ull;
-      if (warp_sum(g) >= T) tau = c;
+      for (int r = 0; r < R; ++r) g[r & 3] += key[r] >= c ? u[r] : 0ull;
+      if (warp_sum((g[0] + g[1]) + (g[2] + g[3])) >= T) tau = c;
     }
     uint64_t above = 0;
 #pragma unroll

@@ -5,7 +5,14 @@ and GSRS abstracts: cumulative top-p selection per query block; CalibAtt
 Fig. 5(b): attention over the kept blocks only; RECAP section 1: the cached
 refinement scaled per head):
 
-  with a latent grid (Hilbert order):
+  with a latent grid (Hilbert order), gather=True:
+    score_blocks_gather  block means of Q, K in curve order, read through perm
+                         (no reordered copies)
+    select_topp_mask     kept lists from the GPU's own block scores
+    sparse_attn_fwd      (in_rows = perm) attention whose Q, K and V tiles are
+                         gathered rows of the grid-order tensors, with the fused
+                         O + alpha*R epilogue writing O and LSE in grid order
+  with a latent grid, gather=False:
     score_blocks_gather  Q, K gathered into curve order inside the pooling pass
     permute_tokens       V gathered into curve order
     select_topp_mask     kept lists from the GPU's own block scores
@@ -24,13 +31,15 @@ import torch
 from . import api
 
 
-def alloc_buffers(B, H, L, D, blk, device):
-    """Device buffers of one pass: curve-order copies, scores, lists, outputs."""
+def alloc_buffers(B, H, L, D, blk, device, copies=True):
+    """Device buffers of one pass: curve-order copies (unless copies=False),
+    scores, lists, outputs."""
     nb = api.n_blocks(L, blk)
     dev = torch.device(device)
     bf = dict(dtype=torch.bfloat16, device=dev)
+    cp = (lambda: torch.empty((B, H, L, D), **bf)) if copies else (lambda: None)
     return dict(
-        qh=torch.empty((B, H, L, D), **bf), kh=torch.empty((B, H, L, D), **bf), vh=torch.empty((B, H, L, D), **bf),
+        qh=cp(), kh=cp(), vh=cp(),
         qp=torch.empty((B, H, nb, D), dtype=torch.float32, device=dev),
         kp=torch.empty((B, H, nb, D), dtype=torch.float32, device=dev),
         probs=torch.empty((B, H, nb, nb), dtype=torch.float32, device=dev),
@@ -43,20 +52,32 @@ def alloc_buffers(B, H, L, D, blk, device):
     )
 
 
-def run_step(b, q, k, v, blk, p, perm=None, R=None, alpha=None, status=None, events=None):
+def run_step(b, q, k, v, blk, p, perm=None, R=None, alpha=None, status=None, events=None, gather=False):
     """One pass on buffers `b` (from alloc_buffers, or slices of them).
 
     q, k, v: bf16 [B,H,L,D] in grid order.  perm: the Hilbert order (int32
     [L], from api.reorder_tokens) or None for no reorder.  p: top-p, one float
-    or one per head.  R (bf16 [B,H,L,D], in the order the attention reads:
-    curve order when perm is given) and alpha (float32 [H]) enable the fused
-    correction.  events: optional three CUDA events recorded before scoring,
-    after selection and after attention.
+    or one per head.  R (bf16 [B,H,L,D]) and alpha (float32 [H]) enable the
+    fused correction; R is in curve order when perm is given without gather,
+    in grid order otherwise.  gather (with perm): the attention gathers its
+    tiles from the grid-order tensors, no reordered copies are made.
+    events: optional three CUDA events recorded before scoring, after
+    selection and after attention.
     Returns (o, lse) in grid order.
     """
     B, H, L, D = q.shape
     if events:
         events[0].record()
+    if perm is not None and gather:
+        api.score_blocks_gather(q, k, perm, blk, None, None, b["qp"], b["kp"], b["probs"], copies=False)
+        api.select_topp_mask(b["probs"], p, L, blk, D, b["mask"], b["idx"], b["cnt"])
+        if events:
+            events[1].record()
+        api.sparse_attn_fwd(q, k, v, blk, b["idx"], b["cnt"], R, alpha, b["o"], b["lse"], status=status,
+                            in_rows=perm)
+        if events:
+            events[2].record()
+        return b["o"], b["lse"]
     if perm is not None:
         api.score_blocks_gather(q, k, perm, blk, b["qh"], b["kh"], b["qp"], b["kp"], b["probs"])
         api.permute_tokens(v, perm, out=b["vh"])

@@ -173,8 +173,9 @@ BSA_API int bsa_permute_tokens(bsa_shape s, const bsa_bf16* x, const int32_t* pe
  * bsa_score_blocks(q_out, k_out), in one pass that reads q and k once.
  * perm: device int32 [L], a permutation of [0, L) (e.g. from
  * bsa_reorder_tokens; not checked on the device).  q_out, k_out: bf16
- * [B,H,L,D], not overlapping q, k or each other.  Outputs and errors as
- * bsa_score_blocks and bsa_permute_tokens.
+ * [B,H,L,D], not overlapping q, k or each other; or both NULL to score the
+ * reordered tokens without writing them (for bsa_sparse_attn_fwd_gather).
+ * Outputs and errors as bsa_score_blocks and bsa_permute_tokens.
  */
 BSA_API int bsa_score_blocks_gather(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const int32_t* perm,
                             bsa_bf16* q_out, bsa_bf16* k_out, float* q_pool, float* k_pool, float* probs,
@@ -416,6 +417,28 @@ BSA_API int bsa_sparse_attn_fwd_scatter(bsa_shape s, const bsa_bf16* q, const bs
                                 const int32_t* kept_idx, const int32_t* kept_cnt, const bsa_bf16* R,
                                 const float* alpha, const int32_t* out_rows, bsa_bf16* o, float* lse,
                                 int32_t* status, bsa_stream stream);
+
+/*
+ * bsa_sparse_attn_fwd_gather -- the block-sparse attention of tokens taken in
+ * the order `rows` gives, with every tensor in the caller's (grid) order: the
+ * Hilbert reorder of the DFSAttn abstract without reordered copies of q, k, v.
+ * Token t of the attention's order is row rows[t] of every (b, h) of q, k and
+ * v (the `perm` of bsa_reorder_tokens); query and key blocks are the 128
+ * consecutive tokens of that order, and kept_idx/kept_cnt index those blocks
+ * (as bsa_select_topp_mask gives them after bsa_score_blocks_gather).  The
+ * output of token t goes to row rows[t] of o and lse, and R (with alpha) is
+ * read at that row too: o = bsa_permute_tokens(inverse) of what
+ * bsa_sparse_attn_fwd gives on the reordered q, k, v and reordered R.
+ * The kernel loads its Q, K and V tiles with 4-row TMA gathers.
+ * rows: device int32 [L], 16-byte aligned, a permutation of [0, L); a row
+ * outside [0, L) reads zeros, its output is skipped, and BSA_DEV_BAD_INDEX is
+ * set.  Other arguments and errors as bsa_sparse_attn_fwd; s.blk and s.D must
+ * be 128 and B*H*L below 2^31 (BSA_ESHAPE otherwise).
+ */
+BSA_API int bsa_sparse_attn_fwd_gather(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
+                                       const int32_t* rows, const int32_t* kept_idx, const int32_t* kept_cnt,
+                                       const bsa_bf16* R, const float* alpha, bsa_bf16* o, float* lse,
+                                       int32_t* status, bsa_stream stream);
 
 /*
  * FP8 Q.K^T.  Defines: the sparse attention of a distilled pipeline run in

@@ -156,6 +156,25 @@ def test_scatter_validation(lib):
                                            ctypes.c_void_p(FAKE.value + 4), FAKE, FAKE, NULL, NULL) == _lib.BSA_EINVAL
 
 
+def test_gather_attention_validation(lib):
+    qkv = [FAKE, ctypes.c_void_p(2 << 20), ctypes.c_void_p(3 << 20)]
+    ok = (NULL, NULL, NULL, NULL)  # kept_idx, kept_cnt, R, alpha
+    out = (ctypes.c_void_p(4 << 20), ctypes.c_void_p(5 << 20), NULL, NULL)  # o, lse, status, stream
+    rows = ctypes.c_void_p(6 << 20)
+    # rows required and 16-byte aligned; 128-token blocks and D = 128 only
+    assert lib.bsa_sparse_attn_fwd_gather(Shape(1, 2, 1000, 128, 128), *qkv, NULL, *ok, *out) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd_gather(Shape(1, 2, 1000, 128, 128), *qkv, ctypes.c_void_p(rows.value + 4), *ok,
+                                          *out) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd_gather(Shape(1, 2, 1000, 128, 64), *qkv, rows, *ok, *out) == _lib.BSA_ESHAPE
+    assert lib.bsa_sparse_attn_fwd_gather(Shape(1, 2, 1000, 64, 128), *qkv, rows, *ok, *out) == _lib.BSA_ESHAPE
+    # row coordinates are int32: B*H*L must stay below 2^31
+    assert lib.bsa_sparse_attn_fwd_gather(Shape(64, 64, 1 << 19, 128, 128), *qkv, rows, *ok,
+                                          *out) == _lib.BSA_ESHAPE
+    # kept_idx without kept_cnt
+    assert lib.bsa_sparse_attn_fwd_gather(Shape(1, 2, 1000, 128, 128), *qkv, rows, FAKE, NULL, NULL, NULL,
+                                          *out) == _lib.BSA_EINVAL
+
+
 def test_gather_scoring_validation(lib):
     s = Shape(1, 2, 1000, 128, 128)
     other = ctypes.c_void_p(2 << 20)
@@ -165,6 +184,9 @@ def test_gather_scoring_validation(lib):
                                        NULL) == _lib.BSA_EINVAL
     assert lib.bsa_score_blocks_gather(s, FAKE, other, FAKE, FAKE, third, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
     assert lib.bsa_score_blocks_gather(s, FAKE, other, FAKE, third, third, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+    # no copies: both outputs NULL, never one
+    assert lib.bsa_score_blocks_gather(s, FAKE, other, FAKE, third, NULL, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_score_blocks_gather(s, FAKE, other, FAKE, NULL, third, FAKE, FAKE, FAKE, NULL) == _lib.BSA_EINVAL
 
 
 def test_elementwise_validation(lib):

@@ -44,9 +44,18 @@ def _select_exact(P_np, p, L, blk, D):
 
 # ------------------------------------------------------------------ scoring
 
-@pytest.mark.parametrize("case", ["tiny", "480p_2heads", "ragged"])
+@pytest.mark.parametrize("case", ["tiny", "480p_2heads", "ragged", "rows_1200", "rows_4000"])
 def test_score_blocks_matches_oracle(case):
-    if case == "tiny":
+    """rows_*: one head with 1200 and 4000 key blocks per row (the largest
+    rows the exact selection takes are 4096 blocks), beyond the rows the block
+    softmax normalises in registers (1024)."""
+    if case.startswith("rows_"):
+        nb = int(case[5:])
+        L = nb * 128 - 37
+        q = random_bf16((1, 1, L, 128), 7)
+        k = random_bf16((1, 1, L, 128), 8)
+        blk = 128
+    elif case == "tiny":
         w = configs.TINY
         q, k, _ = _qkv(w.B, w.H, w.grid, w.D, w.fp)
         blk = w.blk

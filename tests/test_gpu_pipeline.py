@@ -1,7 +1,8 @@
 """GPU parity of the exact call sequence the benchmark times, against the
 oracle's own chain.
 
-The GPU side is `step.run_step`, the function bench.py times: Hilbert order,
+The GPU side is `step.run_step`, the function bench.py times, in both of its
+forms (reordered copies, or tiles gathered by the attention): Hilbert order,
 pooling that gathers Q and K into curve order, the V gather, top-p selection
 on the GPU's own block scores, and sparse attention with the fused
 O + alpha*R epilogue writing O and LSE back to grid order.  The oracle side
@@ -67,12 +68,13 @@ def _valid_topp(P_row, p, kept):
     return not dropped.size or max((row[j], -j) for j in dropped) < (row[worst], -worst)
 
 
-def _run_bench_step(w, q, k, v, R, alpha, p):
+def _run_bench_step(w, q, k, v, R, alpha, p, gather):
     """The benchmark's step on the device; returns host copies of what it wrote."""
     perm = api.reorder_tokens(*w.grid, device=DEV)[0] if w.hilbert else None
-    bufs = alloc_buffers(w.B, w.H, w.L, w.D, w.blk, DEV)
+    bufs = alloc_buffers(w.B, w.H, w.L, w.D, w.blk, DEV, copies=not gather)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    o, lse = run_step(bufs, q.to(DEV), k.to(DEV), v.to(DEV), w.blk, p, perm, R.to(DEV), alpha.to(DEV), status)
+    o, lse = run_step(bufs, q.to(DEV), k.to(DEV), v.to(DEV), w.blk, p, perm, R.to(DEV), alpha.to(DEV), status,
+                      gather=gather)
     torch.cuda.synchronize()
     assert status.item() == 0, f"status {status.item()}"
     out = {n: to_np(bufs[n]) for n in ("probs", "mask", "idx", "cnt")}
@@ -81,14 +83,15 @@ def _run_bench_step(w, q, k, v, R, alpha, p):
     return out
 
 
-def _check(w, p, units_of=None):
+def _check(w, p, units_of=None, gather=False):
     """Run both chains and compare.  units_of(H, NB, differ) -> query blocks
-    to compare (None: every block)."""
+    to compare (None: every block).  gather: the step's gathering form (R in
+    grid order) instead of the reordered copies (R in curve order)."""
     t = make_qkv(w.B, w.H, w.grid, w.D, w.fp)
     q, k, v = t["q"], t["k"], t["v"]
-    R = random_bf16(q.shape, 77, scale=0.05)  # refinement, in the order the attention reads
+    R = random_bf16(q.shape, 77, scale=0.05)  # refinement
     alpha = torch.tensor(w.alpha(), dtype=torch.float32)
-    g = _run_bench_step(w, q, k, v, R, alpha, p)
+    g = _run_bench_step(w, q, k, v, R, alpha, p, gather)
 
     # oracle chain from the same seeded inputs
     qn, kn, vn = (x.float().numpy() for x in (q, k, v))
@@ -123,7 +126,10 @@ def _check(w, p, units_of=None):
 
     units = None if units_of is None else units_of(w.H, w.NB, differ)
     O, LSE = oatt.masked_attention(qn, kn, vn, idx_use, cnt_use, w.blk, units=units)
-    O = ocor.apply_correction(O, R.float().numpy(), alpha.numpy())
+    Rn = R.float().numpy()
+    if w.hilbert and gather:  # R in grid order: the row each query token reads
+        Rn = ohil.permute_rows(Rn, perm_o)
+    O = ocor.apply_correction(O, Rn, alpha.numpy())
     if w.hilbert:  # back to grid order, as the epilogue writes it
         O = ohil.permute_rows(O, perm_o, inverse=True)
         LSE = ohil.permute_rows(LSE[..., None], perm_o, inverse=True)[..., 0]
@@ -131,15 +137,16 @@ def _check(w, p, units_of=None):
     return len(differ), emax, emean, lrel
 
 
-@pytest.mark.parametrize("hilbert", [False, True], ids=["grid-order", "hilbert"])
-def test_bench_step_every_element_480p_2heads(hilbert):
+@pytest.mark.parametrize("mode", ["grid-order", "hilbert-copies", "hilbert-gather"])
+def test_bench_step_every_element_480p_2heads(mode):
     """Every element of O and LSE, 512 work items (>= 3 per CTA)."""
-    w = dataclasses.replace(configs.WAN13B_480P, H=2, hilbert=hilbert)
+    w = dataclasses.replace(configs.WAN13B_480P, H=2, hilbert=mode != "grid-order")
     assert w.B * w.H * w.NB >= 3 * 148
-    _check(w, 0.9)
+    _check(w, 0.9, gather=mode == "hilbert-gather")
 
 
-def test_bench_step_720p_sampled():
+@pytest.mark.parametrize("gather", [False, True], ids=["copies", "gather"])
+def test_bench_step_720p_sampled(gather):
     """The benchmark's workload and calls, 4 heads: sampled query blocks
     (first and last of every head, 10 more per head) plus every row whose
     selection differs."""
@@ -154,4 +161,4 @@ def test_bench_step_720p_sampled():
         u |= {tuple(int(x) for x in d) for d in differ}
         return sorted(u)
 
-    _check(w, w.p[0], units_of)
+    _check(w, w.p[0], units_of, gather=gather)
