@@ -411,14 +411,16 @@ def run_ours(args, w, world, rank, local):
     bufs = alloc_buffers(B, H, L, D, blk, dev, copies=not gather)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def path(b, qi, ki, vi, Ri, ai, events=None):
+    side = torch.cuda.Stream(dev)  # the V gather beside block softmax and selection
+
+    def path(b, qi, ki, vi, Ri, ai, events=None, side_stream=None):
         """One pass of the hot path on buffers `b` (the full set or one head
         chunk): scoring in Hilbert order, selection, sparse attention with the
         fused correction, output in grid order."""
-        return run_step(b, qi, ki, vi, blk, p, perm, Ri, ai, status, events, gather=gather)
+        return run_step(b, qi, ki, vi, blk, p, perm, Ri, ai, status, events, gather=gather, side=side_stream)
 
     def step(qi, ki, vi, events=None):
-        return path(bufs, qi, ki, vi, R_h, alpha, events)
+        return path(bufs, qi, ki, vi, R_h, alpha, events, side)
 
     def barrier():
         if world > 1:

@@ -14,7 +14,8 @@ refinement scaled per head):
                          O + alpha*R epilogue writing O and LSE in grid order
   with a latent grid, gather=False:
     score_blocks_gather  Q, K gathered into curve order inside the pooling pass
-    permute_tokens       V gathered into curve order
+    permute_tokens       V gathered into curve order (on a side stream, beside
+                         the block softmax and the selection, when given one)
     select_topp_mask     kept lists from the GPU's own block scores
     sparse_attn_fwd      attention with the fused O + alpha*R epilogue, writing
                          O and LSE straight back to grid order (row map = perm)
@@ -52,7 +53,8 @@ def alloc_buffers(B, H, L, D, blk, device, copies=True):
     )
 
 
-def run_step(b, q, k, v, blk, p, perm=None, R=None, alpha=None, status=None, events=None, gather=False):
+def run_step(b, q, k, v, blk, p, perm=None, R=None, alpha=None, status=None, events=None, gather=False,
+             side=None):
     """One pass on buffers `b` (from alloc_buffers, or slices of them).
 
     q, k, v: bf16 [B,H,L,D] in grid order.  perm: the Hilbert order (int32
@@ -62,7 +64,10 @@ def run_step(b, q, k, v, blk, p, perm=None, R=None, alpha=None, status=None, eve
     in grid order otherwise.  gather (with perm): the attention gathers its
     tiles from the grid-order tensors, no reordered copies are made.
     events: optional three CUDA events recorded before scoring, after
-    selection and after attention.
+    selection and after attention.  side: optional second CUDA stream for
+    the V gather of the reordered-copies form: it starts when pooling is
+    done (both are HBM-bound) and runs beside block softmax and selection
+    (latency-bound); the attention waits for it.
     Returns (o, lse) in grid order.
     """
     B, H, L, D = q.shape
@@ -78,14 +83,26 @@ def run_step(b, q, k, v, blk, p, perm=None, R=None, alpha=None, status=None, eve
         if events:
             events[2].record()
         return b["o"], b["lse"]
+    v_done = None
     if perm is not None:
         api.score_blocks_gather(q, k, perm, blk, b["qh"], b["kh"], b["qp"], b["kp"], b["probs"])
-        api.permute_tokens(v, perm, out=b["vh"])
+        if side is not None:
+            pooled = torch.cuda.Event()
+            pooled.record()
+            side.wait_event(pooled)
+            with torch.cuda.stream(side):
+                api.permute_tokens(v, perm, out=b["vh"])
+                v_done = torch.cuda.Event()
+                v_done.record()
+        else:
+            api.permute_tokens(v, perm, out=b["vh"])
         qs, ks, vs = b["qh"], b["kh"], b["vh"]
     else:
         qs, ks, vs = q, k, v
         api.score_blocks(qs, ks, blk, b["qp"], b["kp"], b["probs"])
     api.select_topp_mask(b["probs"], p, L, blk, D, b["mask"], b["idx"], b["cnt"])
+    if v_done is not None:
+        torch.cuda.current_stream().wait_event(v_done)
     if events:
         events[1].record()
     o = b["o"] if perm is not None else b["oh"]

@@ -73,8 +73,9 @@ def _run_bench_step(w, q, k, v, R, alpha, p, gather):
     perm = api.reorder_tokens(*w.grid, device=DEV)[0] if w.hilbert else None
     bufs = alloc_buffers(w.B, w.H, w.L, w.D, w.blk, DEV, copies=not gather)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    side = torch.cuda.Stream()  # the V gather beside softmax and selection, as the benchmark runs it
     o, lse = run_step(bufs, q.to(DEV), k.to(DEV), v.to(DEV), w.blk, p, perm, R.to(DEV), alpha.to(DEV), status,
-                      gather=gather)
+                      gather=gather, side=side)
     torch.cuda.synchronize()
     assert status.item() == 0, f"status {status.item()}"
     out = {n: to_np(bufs[n]) for n in ("probs", "mask", "idx", "cnt")}
