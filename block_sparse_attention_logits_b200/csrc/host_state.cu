@@ -8,36 +8,30 @@
 // arrays) is rebuilt, so attributes are lost and addresses may move.  Entries
 // are therefore keyed by device ordinal and remember the context they were
 // made in; a call under another context (a second device, or the same device
-// after a reset) redoes the set-up.  Every table is guarded by one mutex, so
-// host threads may launch concurrently.
+// after a reset) redoes the set-up.  The rules live in device_cache.h (plain
+// C++, tested on the host with fake device calls); this file binds them to
+// the CUDA runtime.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <mutex>
-
+#include "device_cache.h"
 #include "internal.cuh"
 
 namespace bsa {
 namespace {
 
-constexpr int kMaxDevices = 64;
-constexpr int kMaxFuncs = 64;
-
 typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
-
-std::mutex g_mu;
 
 CtxGetCurrentFn ctx_get_current() {
   static CtxGetCurrentFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<CtxGetCurrentFn>(p);
-  }
+  });
   return fn;
 }
 
@@ -50,75 +44,36 @@ void* current_ctx() {
   return nullptr;
 }
 
-struct OptIn {
-  const void* func;
-  void* ctx;
-  size_t bytes;
-};
-OptIn g_optin[kMaxDevices][kMaxFuncs];
-int g_sms[kMaxDevices];
-void* g_sym_ctx[kMaxDevices][4];
-void* g_sym_addr[kMaxDevices][4];
-const void* g_sym_key[4];
+int get_device(int* dev) { return static_cast<int>(cudaGetDevice(dev)); }
+int set_smem(const void* func, size_t bytes) {
+  return static_cast<int>(
+      cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)));
+}
+int device_sms(int dev, int* n) {
+  return static_cast<int>(cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev));
+}
+int lookup_symbol(const void* sym, void** addr) { return static_cast<int>(cudaGetSymbolAddress(addr, sym)); }
+
+const DeviceOps kOps = {get_device, current_ctx, set_smem, device_sms, lookup_symbol,
+                        static_cast<int>(cudaErrorInvalidDevice), static_cast<int>(cudaErrorUnknown)};
+DeviceCache<64, 64, 4> g_cache;
 
 }  // namespace
 
 cudaError_t smem_opt_in(const void* func, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_mu);
-  void* ctx = current_ctx();
-  OptIn* slot = nullptr;
-  for (OptIn& o : g_optin[dev]) {
-    if (o.func == func) {
-      slot = &o;
-      break;
-    }
-    if (!slot && o.func == nullptr) slot = &o;  // first free entry, used if func is new
-  }
-  if (!slot) return cudaErrorUnknown;  // more kernels than the table holds (not reached: < 20 kernels)
-  if (slot->func == func && ctx != nullptr && slot->ctx == ctx && slot->bytes >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
-  if (e != cudaSuccess) return e;
-  slot->func = func;
-  slot->ctx = current_ctx();  // the attribute call made the primary context current if it was not
-  slot->bytes = slot->ctx == ctx ? (bytes > slot->bytes ? bytes : slot->bytes) : bytes;
-  return cudaSuccess;
+  return static_cast<cudaError_t>(g_cache.smem_opt_in(kOps, func, bytes));
 }
 
 int sm_count() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_sms[dev] <= 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-    g_sms[dev] = n;
-  }
-  return g_sms[dev];
+  int n = 0;
+  return g_cache.sm_count(kOps, &n) == 0 ? n : 148;
 }
 
 int symbol_address(const void* symbol, void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ENODEV;
-  std::lock_guard<std::mutex> lock(g_mu);
-  int k = 0;
-  for (; k < 4; ++k)
-    if (g_sym_key[k] == symbol || g_sym_key[k] == nullptr) break;
-  if (k == 4) return BSA_ECUDA;
-  g_sym_key[k] = symbol;
-  void* ctx = current_ctx();
-  if (g_sym_addr[dev][k] == nullptr || ctx == nullptr || g_sym_ctx[dev][k] != ctx) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess || p == nullptr) return BSA_ECUDA;
-    g_sym_addr[dev][k] = p;
-    g_sym_ctx[dev][k] = current_ctx();
-  }
-  *out = g_sym_addr[dev][k];
-  return BSA_OK;
+  const int e = g_cache.symbol_address(kOps, symbol, out);
+  if (e == static_cast<int>(cudaErrorInvalidDevice)) return BSA_ENODEV;
+  return e == 0 ? BSA_OK : BSA_ECUDA;
 }
 
 }  // namespace bsa
