@@ -29,9 +29,9 @@
 // meanwhile.  All MMAs are M=128, N=128 (or N=D), K=16: full-rate shapes.
 //
 // Warp roles (16 warps):
-//   warp 0       item queue; TMA: Q of every item (double buffered), K ring
+//   warp 0       item queue; TMA: Q of every item (kQBuffers buffers), K ring
 //   warp 1       TMA: V ring; TMEM allocation
-//   warp 2       S issuer:  S_n = Q K_n^T into S[n%2]
+//   warp 2       S issuer:  S_n = Q K_n^T into S[n%3] (S[n%2] when fused)
 //   warp 3       PV issuer: O[item%2] += P_n V_n, P read from TMEM
 //   warps 4-7    softmax of rows 32q+0..15 of every TMEM quarter q
 //   warps 8-11   softmax of rows 32q+16..31
@@ -90,8 +90,6 @@ constexpr float kRescaleThreshold = 8.0f;       // log2 units
 constexpr uint32_t kPolyPairs = 0x0000C000u;
 // Q tiles in shared memory across items: one leaves room for a third K slot
 constexpr int kQBuffers = 1;
-// S of a block read by one 128-column TMEM load per warp instead of two
-constexpr bool kWideLoad = false;
 constexpr int kQueue = 4;                       // item queue depth
 constexpr int kItemReaders = 32 * 3 + 256 + 128;  // threads of the roles that read the queue
 // registers per thread: launch 65536 / 512 = 128, then re-balanced per warpgroup
@@ -728,12 +726,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // s[chunk][0..1]: row rA, keys 8*chunk + 2*j4 + {0,1}; s[chunk][2..3]: row rA+8
         uint32_t sr[2][32];
-        if constexpr (kWideLoad) {
-          tmem_ld_16x256b_x16(tS, reinterpret_cast<uint32_t(&)[64]>(sr));
-        } else {
-          tmem_ld_16x256b_x8(tS, sr[0]);
-          tmem_ld_16x256b_x8(tS + 64, sr[1]);
-        }
+        tmem_ld_16x256b_x8(tS, sr[0]);
+        tmem_ld_16x256b_x8(tS + 64, sr[1]);
         tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < 2; ++q)

@@ -201,18 +201,6 @@ __device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)
       : BSA_R8(0), BSA_R8(8), BSA_R8(16), BSA_R8(24)
       : "r"(taddr));
 }
-// 16 chunks of 8 columns = 128 columns, 64 registers (r[0..31] the first 64
-// columns, r[32..63] the next 64, each in the x8 register order)
-__device__ __forceinline__ void tmem_ld_16x256b_x16(uint32_t taddr, uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
-      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
-      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
-      : BSA_R8(0), BSA_R8(8), BSA_R8(16), BSA_R8(24), BSA_R8(32), BSA_R8(40), BSA_R8(48), BSA_R8(56)
-      : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], "

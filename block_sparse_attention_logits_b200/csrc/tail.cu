@@ -78,62 +78,113 @@ __device__ __forceinline__ bool warp_wait_for(uint64_t* bar, uint32_t parity, in
 }
 
 // --------------------------------------------------------------- moments
-// grid (NB, B*H), D threads.  Writes (all per head bh, block j):
+// grid (NB, B*H), 256 threads.  Writes (all per head bh, block j):
 //   kbar, s2, vbar       float32 [bh][j][d]
 //   tabK = bf16(kbar), tabS = bf16(s2 / (2 sqrt(D))), tabV = bf16(vbar)   [bh][j][d]
 //   kcT, vcT             bf16 [bh][d][t] (row length Lp): the block-centred values
+// The block's keys, then its values, are read once from HBM with 16-byte
+// loads into shared memory; each (dimension, token part) thread sums its part
+// and the parts are combined; the centred values go out transposed, 8 tokens
+// (16 bytes) per store.  HBM-bound: K and V read once, kcT and vcT written.
+constexpr int kMomThreads = 256;
+
 template <int D>
-__global__ void __launch_bounds__(D) tail_moments_kernel(const __nv_bfloat16* __restrict__ k,
-                                                         const __nv_bfloat16* __restrict__ v, int L, int blk,
-                                                         int NB, int Lp, float* __restrict__ kbar,
-                                                         float* __restrict__ s2, float* __restrict__ vbar,
-                                                         __nv_bfloat16* __restrict__ tabK,
-                                                         __nv_bfloat16* __restrict__ tabS,
-                                                         __nv_bfloat16* __restrict__ tabV,
-                                                         __nv_bfloat16* __restrict__ kcT,
-                                                         __nv_bfloat16* __restrict__ vcT) {
-  __shared__ __nv_bfloat16 ct[128][D + 2];  // one block's centred values, keys then values
+__global__ void __launch_bounds__(kMomThreads) tail_moments_kernel(const __nv_bfloat16* __restrict__ k,
+                                                                   const __nv_bfloat16* __restrict__ v, int L,
+                                                                   int blk, int NB, int Lp, float* __restrict__ kbar,
+                                                                   float* __restrict__ s2, float* __restrict__ vbar,
+                                                                   __nv_bfloat16* __restrict__ tabK,
+                                                                   __nv_bfloat16* __restrict__ tabS,
+                                                                   __nv_bfloat16* __restrict__ tabV,
+                                                                   __nv_bfloat16* __restrict__ kcT,
+                                                                   __nv_bfloat16* __restrict__ vcT) {
+  constexpr int VPR = D / 8;                // 16-byte vectors per token row
+  constexpr int PARTS = kMomThreads / D;    // token parts per dimension
+  __shared__ __align__(16) __nv_bfloat16 buf[128 * D];  // one block of keys or values, [t][d]
+  __shared__ float part[PARTS][D];
+  __shared__ float mean_s[D];
   const int j = blockIdx.x;
   const long long bh = blockIdx.y;
-  const int d = threadIdx.x;
+  const int tid = threadIdx.x;
+  const int d = tid % D, h = tid / D;
   const int lo = j * blk;
-  const int n = min(L, lo + blk) - lo;
-  const __nv_bfloat16* kb = k + (bh * L + lo) * D;
-  const __nv_bfloat16* vb = v + (bh * L + lo) * D;
-  float sk = 0.f, sv = 0.f;
-  for (int t = 0; t < n; ++t) {
-    sk += __bfloat162float(kb[static_cast<size_t>(t) * D + d]);
-    sv += __bfloat162float(vb[static_cast<size_t>(t) * D + d]);
-  }
-  const float mk = sk / static_cast<float>(n);
-  const float mv = sv / static_cast<float>(n);
-  float q2 = 0.f;
-  for (int t = 0; t < n; ++t) {
-    const float xk = __bfloat162float(kb[static_cast<size_t>(t) * D + d]) - mk;
-    q2 += xk * xk;
-    ct[t][d] = __float2bfloat16_rn(xk);
-  }
-  const float var = q2 / static_cast<float>(n);
+  const int n = min(L, lo + blk) - lo;      // <= blk <= 128
   const size_t o = (static_cast<size_t>(bh) * NB + j) * D + d;
-  kbar[o] = mk;
-  s2[o] = var;
-  vbar[o] = mv;
-  tabK[o] = __float2bfloat16_rn(mk);
-  tabS[o] = __float2bfloat16_rn(var * (0.5f * rsqrtf(static_cast<float>(D))));
-  tabV[o] = __float2bfloat16_rn(mv);
-  // transposed, coalesced along the tokens: the keys, then the values
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < D * n; idx += blockDim.x) {
-    const int dd = idx / n, t = idx - dd * n;
-    kcT[(static_cast<size_t>(bh) * D + dd) * Lp + lo + t] = ct[t][dd];
-  }
-  __syncthreads();
-  for (int t = 0; t < n; ++t)
-    ct[t][d] = __float2bfloat16_rn(__bfloat162float(vb[static_cast<size_t>(t) * D + d]) - mv);
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < D * n; idx += blockDim.x) {
-    const int dd = idx / n, t = idx - dd * n;
-    vcT[(static_cast<size_t>(bh) * D + dd) * Lp + lo + t] = ct[t][dd];
+#pragma unroll 1
+  for (int which = 0; which < 2; ++which) {
+    const __nv_bfloat16* src = (which ? v : k) + (bh * L + lo) * D;
+    __syncthreads();  // the previous pass has finished with buf
+    {
+      const uint4* s4 = reinterpret_cast<const uint4*>(src);
+      uint4* b4 = reinterpret_cast<uint4*>(buf);
+#pragma unroll
+      for (int r = 0; r < 128 * VPR / kMomThreads; ++r) {
+        const int e = tid + r * kMomThreads;
+        if (e < n * VPR) b4[e] = __ldg(s4 + e);
+      }
+    }
+    __syncthreads();
+    // mean over the block's tokens
+    float acc = 0.f;
+    for (int t = h; t < n; t += PARTS) acc += __bfloat162float(buf[t * D + d]);
+    part[h][d] = acc;
+    __syncthreads();
+    if (h == 0) {
+      float sum = 0.f;
+#pragma unroll
+      for (int q = 0; q < PARTS; ++q) sum += part[q][d];
+      mean_s[d] = sum / static_cast<float>(n);
+    }
+    __syncthreads();
+    const float mu = mean_s[d];
+    if (which == 0) {
+      // population variance of the keys
+      float q2 = 0.f;
+      for (int t = h; t < n; t += PARTS) {
+        const float x = __bfloat162float(buf[t * D + d]) - mu;
+        q2 += x * x;
+      }
+      __syncthreads();  // every part[] read of the mean is done
+      part[h][d] = q2;
+      __syncthreads();
+      if (h == 0) {
+        float sq = 0.f;
+#pragma unroll
+        for (int q = 0; q < PARTS; ++q) sq += part[q][d];
+        const float var = sq / static_cast<float>(n);
+        kbar[o] = mu;
+        s2[o] = var;
+        tabK[o] = __float2bfloat16_rn(mu);
+        tabS[o] = __float2bfloat16_rn(var * (0.5f * rsqrtf(static_cast<float>(D))));
+      }
+    } else if (h == 0) {
+      vbar[o] = mu;
+      tabV[o] = __float2bfloat16_rn(mu);
+    }
+    // centred values, transposed: thread item (t8, dd) writes tokens
+    // 8*t8 .. 8*t8+7 of dimension dd (consecutive threads: consecutive dd, so
+    // the shared-memory reads of a token row are conflict-free)
+    __nv_bfloat16* dstT = (which ? vcT : kcT) + static_cast<size_t>(bh) * D * Lp + lo;
+    const int n8 = (n + 7) / 8;
+    for (int item = tid; item < n8 * D; item += kMomThreads) {
+      const int t8 = item / D, dd = item % D;
+      const float m = mean_s[dd];
+      __nv_bfloat16* row = dstT + static_cast<size_t>(dd) * Lp + t8 * 8;
+      if (t8 * 8 + 8 <= n) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = __bfloat162float(buf[(t8 * 8 + 2 * e) * D + dd]) - m;
+          const float x1 = __bfloat162float(buf[(t8 * 8 + 2 * e + 1) * D + dd]) - m;
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(x0, x1);
+          w[e] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        *reinterpret_cast<uint4*>(row) = make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+        for (int t = t8 * 8; t < n; ++t)
+          row[t - t8 * 8] = __float2bfloat16_rn(__bfloat162float(buf[t * D + dd]) - m);
+      }
+    }
   }
 }
 
@@ -261,7 +312,7 @@ __global__ void cov_reduce_kernel(const float* __restrict__ part, int splits, in
 
 // ------------------------------------------------------------ coarse tail
 struct TailShared {
-  uint64_t q_full, c_full, q2_ready, kv_full, kv_empty, s_full, p_full, pv_done, cq_done, drain;
+  uint64_t q_full, c_full, q2_ready, b_full, b_empty, v_full, v_empty, s_full, p_full, pv_done, cq_done, drain;
   uint32_t tmem_base;
 };
 
@@ -294,8 +345,10 @@ __global__ void __launch_bounds__(160, 1)
     mbar_init(&sh->q_full, 1);
     mbar_init(&sh->c_full, 1);
     mbar_init(&sh->q2_ready, 128);
-    mbar_init(&sh->kv_full, 1);
-    mbar_init(&sh->kv_empty, 1);
+    mbar_init(&sh->b_full, 1);
+    mbar_init(&sh->b_empty, 1);
+    mbar_init(&sh->v_full, 1);
+    mbar_init(&sh->v_empty, 1);
     mbar_init(&sh->s_full, 1);
     mbar_init(&sh->p_full, 128);
     mbar_init(&sh->pv_done, 1);
@@ -323,11 +376,12 @@ __global__ void __launch_bounds__(160, 1)
       for (int p = 0; p < 2; ++p) tma_load_3d(sQ + p * kPanel, &tmQ, &sh->q_full, p * 64, qi * kRows, bh);
       mbar_arrive_expect_tx(&sh->c_full, kTileBytes);
       for (int p = 0; p < 2; ++p) tma_load_3d(sC + p * kPanel, &tmC, &sh->c_full, p * 64, 0, bh);
-      mbar_arrive_expect_tx(&sh->kv_full, 3 * kTileBytes);
+      mbar_arrive_expect_tx(&sh->b_full, 2 * kTileBytes);
+      mbar_arrive_expect_tx(&sh->v_full, kTileBytes);
       for (int p = 0; p < 2; ++p) {
-        tma_load_3d(sB1 + p * kPanel, &tmB1, &sh->kv_full, p * 64, 0, bh);
-        tma_load_3d(sB2 + p * kPanel, &tmB2, &sh->kv_full, p * 64, 0, bh);
-        tma_load_3d(sV + p * kPanel, &tmVb, &sh->kv_full, p * 64, 0, bh);
+        tma_load_3d(sB1 + p * kPanel, &tmB1, &sh->b_full, p * 64, 0, bh);
+        tma_load_3d(sB2 + p * kPanel, &tmB2, &sh->b_full, p * 64, 0, bh);
+        tma_load_3d(sV + p * kPanel, &tmVb, &sh->v_full, p * 64, 0, bh);
       }
     }
     __syncwarp();
@@ -347,21 +401,15 @@ __global__ void __launch_bounds__(160, 1)
     }
     __syncwarp();
     if (ok) ok = warp_wait_for(&sh->q2_ready, 0, status);
+    // Tile t's pseudo-key operands B1, B2 are reloaded for tile t+1 as soon as
+    // S(t) has read them (during the softmax of tile t), its values Vbar as
+    // soon as PV(t) has (during S(t+1) and its softmax).  S(t+1) overwrites
+    // the TMEM columns holding P(t), so it waits for PV(t).
+    int b_loads = 1, v_loads = 1, b_seen = 0, v_seen = 0;  // tile loads issued / waited for
     for (int t = 0; t < NT && ok; ++t) {
-      if (t > 0) {
-        // the previous tile's S and PV have read B1, B2 and Vbar
-        if (!(ok = warp_wait_for(&sh->kv_empty, (t - 1) & 1, status))) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&sh->kv_full, 3 * kTileBytes);
-          for (int p = 0; p < 2; ++p) {
-            tma_load_3d(sB1 + p * kPanel, &tmB1, &sh->kv_full, p * 64, t * kRows, bh);
-            tma_load_3d(sB2 + p * kPanel, &tmB2, &sh->kv_full, p * 64, t * kRows, bh);
-            tma_load_3d(sV + p * kPanel, &tmVb, &sh->kv_full, p * 64, t * kRows, bh);
-          }
-        }
-        __syncwarp();
-      }
-      if (!(ok = warp_wait_for(&sh->kv_full, t & 1, status))) break;
+      if (!(ok = warp_wait_for(&sh->b_full, t & 1, status))) break;
+      ++b_seen;
+      if (t > 0 && !(ok = warp_wait_for(&sh->pv_done, (t - 1) & 1, status))) break;
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
@@ -376,9 +424,24 @@ __global__ void __launch_bounds__(160, 1)
           mma_ss(tmem + COL_S, sdesc_sw128(aQ2 + off, 16, 1024), sdesc_sw128(aB2 + off, 16, 1024), idS, 1u);
         }
         tc_commit(&sh->s_full);
+        tc_commit(&sh->b_empty);
       }
       __syncwarp();
+      if (t + 1 < NT) {
+        if (!(ok = warp_wait_for(&sh->b_empty, t & 1, status))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sh->b_full, 2 * kTileBytes);
+          for (int p = 0; p < 2; ++p) {
+            tma_load_3d(sB1 + p * kPanel, &tmB1, &sh->b_full, p * 64, (t + 1) * kRows, bh);
+            tma_load_3d(sB2 + p * kPanel, &tmB2, &sh->b_full, p * 64, (t + 1) * kRows, bh);
+          }
+        }
+        ++b_loads;
+        __syncwarp();
+      }
       if (!(ok = warp_wait_for(&sh->p_full, t & 1, status))) break;
+      if (!(ok = warp_wait_for(&sh->v_full, t & 1, status))) break;
+      ++v_seen;
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
@@ -386,14 +449,27 @@ __global__ void __launch_bounds__(160, 1)
           mma_ts(tmem + COL_O, tmem + COL_S + kk * 8, sdesc_sw128(aV + kk * 2048, kRows * 128, 1024), idPV,
                  (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&sh->pv_done);
-        tc_commit(&sh->kv_empty);
+        tc_commit(&sh->v_empty);
       }
       __syncwarp();
+      if (t + 1 < NT) {
+        if (!(ok = warp_wait_for(&sh->v_empty, t & 1, status))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sh->v_full, kTileBytes);
+          for (int p = 0; p < 2; ++p)
+            tma_load_3d(sV + p * kPanel, &tmVb, &sh->v_full, p * 64, (t + 1) * kRows, bh);
+        }
+        ++v_loads;
+        __syncwarp();
+      }
     }
     if (!ok && lane == 0) {
-      // let every MMA this thread issued finish before TMEM is released
+      // let every MMA this thread issued finish before TMEM is released, and
+      // every tile load land before the shared memory is (bounded waits)
       tc_commit(&sh->drain);
       wait_for(&sh->drain, 0, nullptr);
+      if (b_loads > b_seen) wait_for(&sh->b_full, (b_loads - 1) & 1, nullptr);
+      if (v_loads > v_seen) wait_for(&sh->v_full, (v_loads - 1) & 1, nullptr);
     }
     __syncwarp();
   } else {
@@ -699,7 +775,7 @@ int launch_tail_stats(const bsa_shape& s, const __nv_bfloat16* k, const __nv_bfl
   uint8_t* base = static_cast<uint8_t*>(ws);
   auto* kcT = reinterpret_cast<__nv_bfloat16*>(base + w.kcT);
   auto* vcT = reinterpret_cast<__nv_bfloat16*>(base + w.vcT);
-  tail::tail_moments_kernel<128><<<dim3(NB, BH), 128, 0, st>>>(
+  tail::tail_moments_kernel<128><<<dim3(NB, BH), tail::kMomThreads, 0, st>>>(
       k, v, s.L, s.blk, NB, w.Lp, kbar, s2, vbar, reinterpret_cast<__nv_bfloat16*>(base + w.tabK),
       reinterpret_cast<__nv_bfloat16*>(base + w.tabS), reinterpret_cast<__nv_bfloat16*>(base + w.tabV), kcT, vcT);
   if (cudaGetLastError() != cudaSuccess) return BSA_ECUDA;
