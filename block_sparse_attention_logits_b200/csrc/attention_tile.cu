@@ -32,7 +32,8 @@
 //   warp 0       item queue; TMA: Q of every item (kQBuffers buffers), K ring
 //   warp 1       TMA: V ring; TMEM allocation
 //   warp 2       S issuer:  S_n = Q K_n^T into S[n%3] (S[n%2] when fused)
-//   warp 3       PV issuer: O[item%2] += P_n V_n, P read from TMEM
+//   warp 3       PV issuer: O[item%OB] += P_n V_n, P read from TMEM (OB = 1
+//                at D = 128, 2 at D = 64)
 //   warps 4-7    softmax of rows 32q+0..15 of every TMEM quarter q
 //   warps 8-11   softmax of rows 32q+16..31
 //   warps 12-15  epilogue: O/l (+ alpha*R) -> bf16, LSE
@@ -41,6 +42,17 @@
 // pair of one P column; 4 threads share a row and combine maxima and sums with
 // two shuffles.  The two softmax warpgroups own disjoint rows and never wait
 // for each other, so one can exponentiate while the other loads.
+//
+// FP8 Q.K^T (kF8, D = 128): the Q and K tiles are E4M3 codes (128-byte
+// swizzled rows of 128 codes), S = Q K^T runs as kind::f8f6f4 MMAs (32 codes of
+// K per instruction), and the softmax scales a block's logits by s_q * s_k,
+// the dequantization scales of the query and key blocks (the key block's scale
+// is loaded one block ahead).  V, P and O are as in the bf16 path.
+//
+// Row gathers (kGather, D = 128): token t of the attention's order is row
+// in_rows[t] of the grid-order Q, K and V; each 128-row tile arrives as 64
+// four-row TMA gathers (2 per lane of the producer warp), and the epilogue
+// writes O, LSE and reads R through the same rows.
 //
 // Online softmax in the log2 domain in fp32.  The reference max is only
 // raised when a block max exceeds it by more than 8 (so P <= 2^8); O is then
