@@ -295,3 +295,27 @@ def test_tail_validation(lib):
     assert lib.bsa_tail_reconstruct(Shape(1, 2, 100, 16, 0), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, NULL, FAKE,
                                     NULL) == _lib.BSA_EINVAL
     assert lib.bsa_complement_lists(s, FAKE, NULL, FAKE, NULL) == _lib.BSA_EINVAL
+
+
+def test_fp8_validation(lib):
+    s = Shape(1, 2, 1000, 128, 128)
+    x, codes, scales = FAKE, ctypes.c_void_p(2 << 20), ctypes.c_void_p(3 << 20)
+    # quantize: every pointer required and 16-byte aligned; the block shapes of the other calls
+    assert lib.bsa_quantize_fp8(s, NULL, codes, scales, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_quantize_fp8(s, x, codes, NULL, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_quantize_fp8(s, x, ctypes.c_void_p(codes.value + 8), scales, NULL) == _lib.BSA_EINVAL
+    assert lib.bsa_quantize_fp8(Shape(1, 2, 1000, 96, 128), x, codes, scales, NULL) == _lib.BSA_ESHAPE
+    assert lib.bsa_quantize_fp8(Shape(1, 2, 1000, 128, 32), x, codes, scales, NULL) == _lib.BSA_ESHAPE
+    # attention: codes, scales, v and outputs required; D = 128 and 128-token blocks only
+    q8, qs, k8, ks, v = (ctypes.c_void_p(a << 20) for a in (4, 5, 6, 7, 8))
+    out = (ctypes.c_void_p(9 << 20), ctypes.c_void_p(10 << 20), NULL, NULL)  # o, lse, status, stream
+    none4 = (NULL, NULL, NULL, NULL)  # kept_idx, kept_cnt, R, alpha
+    assert lib.bsa_sparse_attn_fwd_fp8(s, q8, NULL, k8, ks, v, *none4, *out) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd_fp8(s, q8, qs, k8, ks, v, FAKE, NULL, NULL, NULL, *out) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd_fp8(s, q8, qs, k8, ks, v, NULL, NULL, FAKE, NULL, *out) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd_fp8(s, q8, ctypes.c_void_p(qs.value + 2), k8, ks, v, *none4,
+                                       *out) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd_fp8(Shape(1, 2, 1000, 64, 128), q8, qs, k8, ks, v, *none4,
+                                       *out) == _lib.BSA_ESHAPE
+    assert lib.bsa_sparse_attn_fwd_fp8(Shape(1, 2, 1000, 128, 64), q8, qs, k8, ks, v, *none4,
+                                       *out) == _lib.BSA_ESHAPE
