@@ -176,28 +176,28 @@ __global__ void __launch_bounds__(256, 3) block_softmax_kernel(const float* __re
         if (j < NB) row[j] = sum > 0.f ? x[e] / sum : 0.f;
       }
     }
-    return;
-  }
-  for (int rr = w; rr < kTile; rr += 8) {
-    const int i = i0 + rr;
-    if (i >= NB) break;
-    float* row = probs + (bh * NB + i) * NB;
-    const uint8_t* crow = cand ? cand + (bh * NB + i) * NB : nullptr;
-    float m = -INFINITY;
-    for (int j = lane; j < NB; j += 32)
-      if (!crow || crow[j]) m = fmaxf(m, row[j]);
+  } else {
+    for (int rr = w; rr < kTile; rr += 8) {
+      const int i = i0 + rr;
+      if (i >= NB) break;
+      float* row = probs + (bh * NB + i) * NB;
+      const uint8_t* crow = cand ? cand + (bh * NB + i) * NB : nullptr;
+      float m = -INFINITY;
+      for (int j = lane; j < NB; j += 32)
+        if (!crow || crow[j]) m = fmaxf(m, row[j]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float sum = 0.f;
-    for (int j = lane; j < NB; j += 32) {
-      const float e = (!crow || crow[j]) ? expf(row[j] - m) : 0.f;
-      row[j] = e;
-      sum += e;
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float sum = 0.f;
+      for (int j = lane; j < NB; j += 32) {
+        const float e = (!crow || crow[j]) ? expf(row[j] - m) : 0.f;
+        row[j] = e;
+        sum += e;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      // a row without candidates (sum 0) stays all zeros
+      for (int j = lane; j < NB; j += 32) row[j] = sum > 0.f ? row[j] / sum : 0.f;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    // a row without candidates (sum 0) stays all zeros
-    for (int j = lane; j < NB; j += 32) row[j] = sum > 0.f ? row[j] / sum : 0.f;
   }
 }
 

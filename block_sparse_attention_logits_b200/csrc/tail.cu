@@ -313,13 +313,21 @@ __global__ void cov_reduce_kernel(const float* __restrict__ part, int splits, in
 // ------------------------------------------------------------ coarse tail
 struct TailShared {
   uint64_t q_full, c_full, q2_ready, b_full, b_empty, v_full, v_empty, s_full, p_full, pv_done, cq_done, drain;
+  uint64_t pair[4];        // the two softmax warps of a lane quarter: per tile, then once for the sums
+  float xchg[2][2][128];   // [tile parity][column half][row]: a warp's row maxima (then its row sums)
   uint32_t tmem_base;
 };
+constexpr int kTailSoftmaxWarps = 8;   // two per TMEM lane quarter, one per 64-column half
+constexpr int kTailThreads = 32 * kTailSoftmaxWarps + 32;
 
-// grid (NB, B*H), 160 threads.  Shared memory: Q | Q o Q | C | B1 | B2 | Vbar
-// (32 KB each), the mask row (NB bytes) and the barriers.
+// grid (NB, B*H), 288 threads: warps 0-7 softmax and epilogue (warp w takes
+// the rows of TMEM lane quarter w % 4 and the 64-column half w / 4 of S and of
+// O; the two warps of a quarter exchange their row maxima every tile and
+// their row sums at the end), warp 8 loads tiles and issues the MMAs.
+// Shared memory: Q | Q o Q | C | B1 | B2 | Vbar (32 KB each), the mask row
+// (NT * 128 bytes) and the barriers.
 // TMEM columns: S [0, 128) | O [128, 256) | CQ [256, 384).
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(kTailThreads, 1)
     coarse_tail_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                        const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
                        const __grid_constant__ CUtensorMap tmVb, const uint8_t* __restrict__ mask, int L, int blk,
@@ -333,24 +341,25 @@ __global__ void __launch_bounds__(160, 1)
   uint8_t* sB1 = smem + 3 * kTileBytes;
   uint8_t* sB2 = smem + 4 * kTileBytes;
   uint8_t* sV = smem + 5 * kTileBytes;
-  uint8_t* sMask = smem + 6 * kTileBytes;  // NB bytes
-  TailShared* sh = reinterpret_cast<TailShared*>(sMask + ((NB + 15) & ~15));
+  uint8_t* sMask = smem + 6 * kTileBytes;  // NT * 128 bytes: the mask row, 1 past NB
+  TailShared* sh = reinterpret_cast<TailShared*>(sMask + ((NB + 127) & ~127));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qi = blockIdx.x;
   const int bh = blockIdx.y;
   const int NT = (NB + 127) / 128;  // pseudo-key tiles
   const uint8_t* mrow = mask + (static_cast<size_t>(bh) * NB + qi) * NB;
-  for (int j = threadIdx.x; j < NB; j += blockDim.x) sMask[j] = mrow[j];
+  for (int j = threadIdx.x; j < NT * kRows; j += blockDim.x) sMask[j] = j < NB ? mrow[j] : 1;
   if (threadIdx.x == 0) {
     mbar_init(&sh->q_full, 1);
     mbar_init(&sh->c_full, 1);
-    mbar_init(&sh->q2_ready, 128);
+    mbar_init(&sh->q2_ready, 32 * kTailSoftmaxWarps);
     mbar_init(&sh->b_full, 1);
     mbar_init(&sh->b_empty, 1);
     mbar_init(&sh->v_full, 1);
     mbar_init(&sh->v_empty, 1);
     mbar_init(&sh->s_full, 1);
-    mbar_init(&sh->p_full, 128);
+    mbar_init(&sh->p_full, 32 * kTailSoftmaxWarps);
+    for (int qq = 0; qq < 4; ++qq) mbar_init(&sh->pair[qq], 64);
     mbar_init(&sh->pv_done, 1);
     mbar_init(&sh->cq_done, 1);
     mbar_init(&sh->drain, 1);
@@ -366,7 +375,7 @@ __global__ void __launch_bounds__(160, 1)
   const uint32_t tmem = sh->tmem_base;
   constexpr uint32_t COL_S = 0, COL_O = 128, COL_CQ = 256;
 
-  if (warp == 4) {
+  if (warp == kTailSoftmaxWarps) {
     // ------------------------------------------------ loads and MMA issue
     constexpr uint32_t idS = idesc_bf16_f32(kRows, 128, false, false);
     constexpr uint32_t idPV = idesc_bf16_f32(kRows, 128, false, true);
@@ -473,15 +482,19 @@ __global__ void __launch_bounds__(160, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------- softmax and epilogue, row r
-    const int r = warp * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // ------------------------------------------- softmax and epilogue
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;  // the thread's row
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t colS = COL_S + half * 64;  // this warp's 64 columns of S ...
+    const uint32_t colO = COL_O + half * 64;  // ... of O ...
+    const uint32_t colC = COL_CQ + half * 64;  // ... and of C Q^T
     bool ok = warp_wait_for(&sh->q_full, 0, status);
     if (ok) {
       // Q o Q in the same swizzled positions (an elementwise map keeps the layout)
       const uint4* src = reinterpret_cast<const uint4*>(sQ);
       uint4* dst = reinterpret_cast<uint4*>(sQ2);
-      for (int c = threadIdx.x; c < kTileBytes / 16; c += 128) {
+      for (int c = threadIdx.x; c < kTileBytes / 16; c += 32 * kTailSoftmaxWarps) {
         uint4 x = src[c];
         uint32_t* w = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll
@@ -495,65 +508,93 @@ __global__ void __launch_bounds__(160, 1)
     }
     mbar_arrive(&sh->q2_ready);
     const float bias_last = log2f(static_cast<float>(L - (NB - 1) * blk) / static_cast<float>(blk));
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
+    int xp = 0;                    // completions of this quarter's pair barrier so far
     for (int t = 0; t < NT && ok; ++t) {
       if (!(ok = warp_wait_for(&sh->s_full, t & 1, status))) break;
       tc_fence_after();
-      uint32_t s[128];
+      uint32_t s[64];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_off + COL_S + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(s + cc * 32));
+      for (int cc = 0; cc < 2; ++cc) tmem_ld32(tmem + lane_off + colS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(s + cc * 32));
       tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 128; ++e) reg_fence(s[e]);
-      float mx = -INFINITY;
+      for (int e = 0; e < 64; ++e) reg_fence(s[e]);
+      // kept blocks and blocks past NB (mask byte 1) are not in the tail; the
+      // mask bytes come 16 at a time, the maxima in four chains
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      const uint4* mrow4 = reinterpret_cast<const uint4*>(sMask + t * kRows + half * 64);
 #pragma unroll
-      for (int e = 0; e < 128; ++e) {
-        const int j = t * kRows + e;
-        float x = __uint_as_float(s[e]) * scale_log2;
-        if (j == NB - 1) x += bias_last;
-        if (j >= NB || sMask[j]) x = -INFINITY;
-        s[e] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+      for (int c = 0; c < 4; ++c) {
+        const uint4 mw = mrow4[c];
+        const uint32_t mwd[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+          const int e = c * 16 + b;
+          float x = __uint_as_float(s[e]) * scale_log2;
+          if (t * kRows + half * 64 + e == NB - 1) x += bias_last;
+          if ((mwd[b >> 2] >> (8 * (b & 3))) & 0xFFu) x = -INFINITY;
+          s[e] = __float_as_uint(x);
+          mx4[e & 3] = fmaxf(mx4[e & 3], x);
+        }
       }
+      // the other half-row's maximum, through shared memory (buffer by tile
+      // parity: a warp can be at most one exchange ahead of its partner)
+      sh->xchg[t & 1][half][r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      mbar_arrive(&sh->pair[quarter]);
+      if (!(ok = warp_wait_for(&sh->pair[quarter], xp & 1, status))) break;
+      ++xp;
+      const float mx = fmaxf(sh->xchg[t & 1][0][r], sh->xchg[t & 1][1][r]);
       const float m_new = fmaxf(m, mx);
       const bool grow_m = t > 0 && m_new > m;
       if (__any_sync(0xffffffffu, grow_m)) {
-        // rescale O once the previous PV has completed; the whole warp takes
-        // part in the TMEM accesses, rows whose maximum did not grow with 1
+        // rescale this half of O once the previous PV has completed; the whole
+        // warp takes part in the TMEM accesses, rows whose maximum did not grow
+        // with 1
         if (!(ok = warp_wait_for(&sh->pv_done, (t - 1) & 1, status))) break;
         tc_fence_after();
         const float f = grow_m ? ex2_approx(m - m_new) : 1.f;  // 0 while m is -inf
         l *= f;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_off + COL_O + cc * 32, o);
+          tmem_ld32(tmem + lane_off + colO + cc * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int x = 0; x < 32; ++x) {
             reg_fence(o[x]);
             o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
           }
-          tmem_st32(tmem + lane_off + COL_O + cc * 32, o);
+          tmem_st32(tmem + lane_off + colO + cc * 32, o);
         }
         tmem_wait_st();
       }
       m = m_new;
-      uint32_t p[64];
+      uint32_t p[32];
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial sums
+      const float mm = m == -INFINITY ? 0.f : m;  // a row with no tail block so far: every x is -inf
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = m == -INFINITY ? 0.f : ex2_approx(__uint_as_float(s[2 * c]) - m);
-        const float p1 = m == -INFINITY ? 0.f : ex2_approx(__uint_as_float(s[2 * c + 1]) - m);
-        l += p0 + p1;
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = ex2_approx(__uint_as_float(s[2 * c]) - mm);
+        const float p1 = ex2_approx(__uint_as_float(s[2 * c + 1]) - mm);
+        l4[c & 3] += p0 + p1;
         p[c] = pack_bf16x2(p0, p1);
       }
-      tmem_st32(tmem + lane_off + COL_S, *reinterpret_cast<uint32_t(*)[32]>(p));
-      tmem_st32(tmem + lane_off + COL_S + 32, *reinterpret_cast<uint32_t(*)[32]>(p + 32));
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      // P columns 32*half .. 32*half+31 (both halves have loaded their S:
+      // the exchange above follows every load)
+      tmem_st32(tmem + lane_off + COL_S + half * 32, p);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sh->p_full);
     }
-    // epilogue
+    // the full row sum, through the same exchange
+    if (ok) {
+      sh->xchg[xp & 1][half][r] = l;
+      mbar_arrive(&sh->pair[quarter]);
+      ok = warp_wait_for(&sh->pair[quarter], xp & 1, status);
+      l = sh->xchg[xp & 1][0][r] + sh->xchg[xp & 1][1][r];
+    }
+    // epilogue: this half of the row's obar
     if (ok) ok = warp_wait_for(&sh->pv_done, (NT - 1) & 1, status) && warp_wait_for(&sh->cq_done, 0, status);
     tc_fence_after();
     const int grow = qi * kRows + r;
@@ -561,15 +602,15 @@ __global__ void __launch_bounds__(160, 1)
       const bool store = grow < L;
       const size_t row = static_cast<size_t>(bh) * L + (store ? grow : 0);
       const bool empty = !(l > 0.f);
-      if (store) lbar[row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f + log_blk;
+      if (store && half == 0) lbar[row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f + log_blk;
       const float inv_l = empty ? 0.f : 1.f / l;
       const float inv_sqrt_d = rsqrtf(128.f);
-      __nv_bfloat16* out = obar + row * 128;
+      __nv_bfloat16* out = obar + row * 128 + half * 64;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t o[32], cq[32];
-        tmem_ld32(tmem + lane_off + COL_O + cc * 32, o);
-        tmem_ld32(tmem + lane_off + COL_CQ + cc * 32, cq);
+        tmem_ld32(tmem + lane_off + colO + cc * 32, o);
+        tmem_ld32(tmem + lane_off + colC + cc * 32, cq);
         tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
@@ -804,10 +845,10 @@ int launch_coarse_tail(const bsa_shape& s, const __nv_bfloat16* q, const uint8_t
       !tail::map3(&mB1, base + w.tabK, 128, NB, BH, 128) || !tail::map3(&mB2, base + w.tabS, 128, NB, BH, 128) ||
       !tail::map3(&mV, base + w.tabV, 128, NB, BH, 128))
     return BSA_ECUDA;
-  const int smem = 6 * tail::kTileBytes + ((NB + 15) & ~15) + 256 + 1024;
+  const int smem = 6 * tail::kTileBytes + ((NB + 127) & ~127) + static_cast<int>(sizeof(tail::TailShared)) + 1024;
   if (smem_opt_in(reinterpret_cast<const void*>(tail::coarse_tail_kernel), smem) != cudaSuccess) return BSA_ECUDA;
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
-  tail::coarse_tail_kernel<<<dim3(NB, BH), 160, smem, st>>>(mQ, mC, mB1, mB2, mV, mask, s.L, s.blk, NB, scale_log2,
+  tail::coarse_tail_kernel<<<dim3(NB, BH), tail::kTailThreads, smem, st>>>(mQ, mC, mB1, mB2, mV, mask, s.L, s.blk, NB, scale_log2,
                                                              std::log(static_cast<float>(s.blk)), lbar, obar, status);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ECUDA;
 }
