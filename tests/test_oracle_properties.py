@@ -2,8 +2,9 @@
 hypothesis, each checked against what the definitions imply -- top-p
 selection is the shortest ordered prefix reaching the target, interval
 encoding decodes back and merging adds the fewest blocks, the drift does not
-depend on the scale of the means, and a refinement taken at the same step
-turns the coarse tail into the exact one."""
+depend on the scale of the means, a refinement taken at the same step
+turns the coarse tail into the exact one, and E4M3 encoding is the nearest
+value, monotone, and bounded in its block quantization error."""
 
 import itertools
 
@@ -12,6 +13,7 @@ from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
 
 from oracle import attention as oatt
+from oracle import fp8 as ofp8
 from oracle import intervals as oint
 from oracle import reuse as oreu
 from oracle import tail as otail
@@ -124,3 +126,35 @@ def test_refresh_kept_share_is_a_mixture_weight(seed, nblocks, ragged):
     Oc, Lc = oatt.masked_attention(q, k, v, ci, cc, blk)
     mix = mass[..., None] * np.nan_to_num(Os) + (1 - mass)[..., None] * np.nan_to_num(Oc)
     assert np.allclose(mix, Od, atol=1e-10)
+
+
+_E4M3_CODES = np.array([c for c in range(256) if not np.isnan(ofp8.e4m3_value(np.uint8(c)))], np.uint8)
+_E4M3_VALUES = ofp8.e4m3_value(_E4M3_CODES)
+
+
+@SETTINGS
+@given(st.lists(st.floats(-600.0, 600.0, width=32), min_size=1, max_size=64))
+def test_e4m3_is_the_nearest_value_and_monotone(xs):
+    x = np.asarray(xs, np.float32)
+    v = ofp8.e4m3_value(ofp8.e4m3_encode(x))
+    xc = np.clip(x.astype(np.float64), -448.0, 448.0)
+    best = np.abs(xc[:, None] - _E4M3_VALUES[None, :]).min(axis=1)
+    assert np.array_equal(np.abs(v - xc), best)          # no representable value is nearer
+    order = np.argsort(x, kind="stable")
+    assert np.all(np.diff(v[order]) >= 0)                 # encoding keeps the order
+
+
+@SETTINGS
+@given(st.integers(0, 2 ** 31 - 1), st.integers(1, 300), st.floats(1e-3, 1e3))
+def test_block_quantization_error_is_one_e4m3_rounding(seed, L, spread):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((1, 1, L, 8)) * spread).astype(np.float32)
+    codes, scales = ofp8.quantize_blocks(x, 128)
+    deq = ofp8.dequantize_blocks(codes, scales, 128)
+    s = np.broadcast_to(np.repeat(scales.astype(np.float64), 128, axis=2)[:, :, :L, None], x.shape)
+    err = np.abs(deq - x)
+    normal = np.abs(x) >= 2.0 ** -6 * s
+    # half a unit in the last place: 2^-4 relative for normal codes, 2^-10
+    # of the scale for subnormal ones, plus the float32 rounding of x * (448 / amax)
+    assert np.all(err[normal] <= (2.0 ** -4 + 2.0 ** -20) * np.abs(x[normal]))
+    assert np.all(err[~normal] <= (2.0 ** -10 + 2.0 ** -20) * s[~normal])
