@@ -312,7 +312,7 @@ __global__ void cov_reduce_kernel(const float* __restrict__ part, int splits, in
 
 // ------------------------------------------------------------ coarse tail
 struct TailShared {
-  uint64_t q_full, c_full, q2_ready, b_full, b_empty, v_full, v_empty, s_full, p_full, pv_done, cq_done, drain;
+  uint64_t q_full, c_full, q2_ready, b_full, b_empty, v_full, v_empty, s_full[2], p_full[2], pv_done, cq_done, drain;
   uint64_t pair[4];        // the two softmax warps of a lane quarter: per tile, then once for the sums
   float xchg[2][2][128];   // [tile parity][column half][row]: a warp's row maxima (then its row sums)
   uint32_t tmem_base;
@@ -326,7 +326,7 @@ constexpr int kTailThreads = 32 * kTailSoftmaxWarps + 32;
 // their row sums at the end), warp 8 loads tiles and issues the MMAs.
 // Shared memory: Q | Q o Q | C | B1 | B2 | Vbar (32 KB each), the mask row
 // (NT * 128 bytes) and the barriers.
-// TMEM columns: S [0, 128) | O [128, 256) | CQ [256, 384).
+// TMEM columns: S0 [0, 128) | S1 [128, 256) | O [256, 384) | CQ [384, 512).
 __global__ void __launch_bounds__(kTailThreads, 1)
     coarse_tail_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                        const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
@@ -357,8 +357,10 @@ __global__ void __launch_bounds__(kTailThreads, 1)
     mbar_init(&sh->b_empty, 1);
     mbar_init(&sh->v_full, 1);
     mbar_init(&sh->v_empty, 1);
-    mbar_init(&sh->s_full, 1);
-    mbar_init(&sh->p_full, 32 * kTailSoftmaxWarps);
+    mbar_init(&sh->s_full[0], 1);
+    mbar_init(&sh->s_full[1], 1);
+    mbar_init(&sh->p_full[0], 32 * kTailSoftmaxWarps);
+    mbar_init(&sh->p_full[1], 32 * kTailSoftmaxWarps);
     for (int qq = 0; qq < 4; ++qq) mbar_init(&sh->pair[qq], 64);
     mbar_init(&sh->pv_done, 1);
     mbar_init(&sh->cq_done, 1);
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(kTailThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
-  constexpr uint32_t COL_S = 0, COL_O = 128, COL_CQ = 256;
+  constexpr uint32_t COL_S = 0, COL_O = 256, COL_CQ = 384;
 
   if (warp == kTailSoftmaxWarps) {
     // ------------------------------------------------ loads and MMA issue
@@ -410,34 +412,38 @@ __global__ void __launch_bounds__(kTailThreads, 1)
     }
     __syncwarp();
     if (ok) ok = warp_wait_for(&sh->q2_ready, 0, status);
-    // Tile t's pseudo-key operands B1, B2 are reloaded for tile t+1 as soon as
-    // S(t) has read them (during the softmax of tile t), its values Vbar as
-    // soon as PV(t) has (during S(t+1) and its softmax).  S(t+1) overwrites
-    // the TMEM columns holding P(t), so it waits for PV(t).
+    // S runs one tile ahead in two TMEM buffers (S, then P of tile t in
+    // buffer t % 2): S(t+1) is computed while the softmax works on tile t.
+    // The pseudo-key operands B1, B2 of the next tile are loaded as soon as S
+    // has read this tile's, the values Vbar as soon as PV has.  S(t+1)
+    // overwrites the buffer that held P(t-1), so it waits for PV(t-1).  Every
+    // barrier a waiter could otherwise see two phases ahead is kept per
+    // buffer (s_full, p_full).
     int b_loads = 1, v_loads = 1, b_seen = 0, v_seen = 0;  // tile loads issued / waited for
-    for (int t = 0; t < NT && ok; ++t) {
-      if (!(ok = warp_wait_for(&sh->b_full, t & 1, status))) break;
+    auto issue_s = [&](int t) -> bool {                     // S(t) into buffer t % 2
+      if (!warp_wait_for(&sh->b_full, t & 1, status)) return false;
       ++b_seen;
-      if (t > 0 && !(ok = warp_wait_for(&sh->pv_done, (t - 1) & 1, status))) break;
+      if (t >= 2 && !warp_wait_for(&sh->pv_done, (t - 2) & 1, status)) return false;
       tc_fence_after();
       if (lane == 0) {
+        const uint32_t dS = tmem + COL_S + (t & 1) * kRows;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-          mma_ss(tmem + COL_S, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aB1 + off, 16, 1024), idS,
-                 kk > 0 ? 1u : 0u);
+          mma_ss(dS, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aB1 + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-          mma_ss(tmem + COL_S, sdesc_sw128(aQ2 + off, 16, 1024), sdesc_sw128(aB2 + off, 16, 1024), idS, 1u);
+          mma_ss(dS, sdesc_sw128(aQ2 + off, 16, 1024), sdesc_sw128(aB2 + off, 16, 1024), idS, 1u);
         }
-        tc_commit(&sh->s_full);
+        tc_commit(&sh->s_full[t & 1]);
         tc_commit(&sh->b_empty);
       }
       __syncwarp();
       if (t + 1 < NT) {
-        if (!(ok = warp_wait_for(&sh->b_empty, t & 1, status))) break;
+        // the next tile's B1, B2 once S(t) has read this tile's
+        if (!warp_wait_for(&sh->b_empty, t & 1, status)) return false;
         if (lane == 0) {
           mbar_arrive_expect_tx(&sh->b_full, 2 * kTileBytes);
           for (int p = 0; p < 2; ++p) {
@@ -448,14 +454,20 @@ __global__ void __launch_bounds__(kTailThreads, 1)
         ++b_loads;
         __syncwarp();
       }
-      if (!(ok = warp_wait_for(&sh->p_full, t & 1, status))) break;
+      return true;
+    };
+    if (ok) ok = issue_s(0);
+    for (int t = 0; t < NT && ok; ++t) {
+      if (t + 1 < NT && !(ok = issue_s(t + 1))) break;
+      if (!(ok = warp_wait_for(&sh->p_full[t & 1], (t >> 1) & 1, status))) break;
       if (!(ok = warp_wait_for(&sh->v_full, t & 1, status))) break;
       ++v_seen;
       tc_fence_after();
       if (lane == 0) {
+        const uint32_t aP = tmem + COL_S + (t & 1) * kRows;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + COL_O, tmem + COL_S + kk * 8, sdesc_sw128(aV + kk * 2048, kRows * 128, 1024), idPV,
+          mma_ts(tmem + COL_O, aP + kk * 8, sdesc_sw128(aV + kk * 2048, kRows * 128, 1024), idPV,
                  (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&sh->pv_done);
         tc_commit(&sh->v_empty);
@@ -511,11 +523,13 @@ __global__ void __launch_bounds__(kTailThreads, 1)
     float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
     int xp = 0;                    // completions of this quarter's pair barrier so far
     for (int t = 0; t < NT && ok; ++t) {
-      if (!(ok = warp_wait_for(&sh->s_full, t & 1, status))) break;
+      if (!(ok = warp_wait_for(&sh->s_full[t & 1], (t >> 1) & 1, status))) break;
       tc_fence_after();
+      const uint32_t bufS = (t & 1) * kRows;  // this tile's S buffer
       uint32_t s[64];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) tmem_ld32(tmem + lane_off + colS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(s + cc * 32));
+      for (int cc = 0; cc < 2; ++cc)
+        tmem_ld32(tmem + lane_off + bufS + colS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(s + cc * 32));
       tmem_wait_ld();
 #pragma unroll
       for (int e = 0; e < 64; ++e) reg_fence(s[e]);
@@ -523,6 +537,7 @@ __global__ void __launch_bounds__(kTailThreads, 1)
       // mask bytes come 16 at a time, the maxima in four chains
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       const uint4* mrow4 = reinterpret_cast<const uint4*>(sMask + t * kRows + half * 64);
+      const int e_last = NB - 1 - t * kRows - half * 64;  // the ragged last block, if in this half
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const uint4 mw = mrow4[c];
@@ -531,7 +546,7 @@ __global__ void __launch_bounds__(kTailThreads, 1)
         for (int b = 0; b < 16; ++b) {
           const int e = c * 16 + b;
           float x = __uint_as_float(s[e]) * scale_log2;
-          if (t * kRows + half * 64 + e == NB - 1) x += bias_last;
+          if (e == e_last) x += bias_last;
           if ((mwd[b >> 2] >> (8 * (b & 3))) & 0xFFu) x = -INFINITY;
           s[e] = __float_as_uint(x);
           mx4[e & 3] = fmaxf(mx4[e & 3], x);
@@ -582,10 +597,10 @@ __global__ void __launch_bounds__(kTailThreads, 1)
       l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       // P columns 32*half .. 32*half+31 (both halves have loaded their S:
       // the exchange above follows every load)
-      tmem_st32(tmem + lane_off + COL_S + half * 32, p);
+      tmem_st32(tmem + lane_off + COL_S + bufS + half * 32, p);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sh->p_full);
+      mbar_arrive(&sh->p_full[t & 1]);
     }
     // the full row sum, through the same exchange
     if (ok) {
