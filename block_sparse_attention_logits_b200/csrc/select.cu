@@ -26,6 +26,10 @@ namespace bsa {
 namespace {
 
 constexpr uint32_t kSelected = 0xFFFFFFFFu;  // marker: above every real key
+// With T > 0 the threshold is the key of a block with mass, P >= 2^-40
+// (key >= 0x2B800000), and no key exceeds 1.0f (0x3F800000): bit 30 of tau is
+// 0 and bit 29 is 1, so the search starts at bit 28
+constexpr uint32_t kTopBits = 0x20000000u;
 
 __device__ __forceinline__ uint32_t prob_key(float p) {
   // NaN and p <= 0 (incl. -0) -> 0; p > 1 (incl. inf) -> bits of 1.0f
@@ -134,9 +138,9 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ p
     if (lane == 0 && best_j < NB) keys[best_j] = kSelected;
     tau = kSelected - 1u;
   } else {
-    // largest tau with sum_{key >= tau} u >= T (bit 31 is never set in a key)
-    tau = 0;
-    for (int b = 30; b >= 0; --b) {
+    // largest tau with sum_{key >= tau} u >= T; its top two bits are known
+    tau = kTopBits;
+    for (int b = 28; b >= 0; --b) {
       const uint32_t cand = tau | (1u << b);
       uint64_t g = 0;
       for (int j = lane; j < NB; j += 32) g += keys[j] >= cand ? us[j] : 0ull;
@@ -255,9 +259,9 @@ __global__ void __launch_bounds__(256) select_reg_kernel(const float* __restrict
       if (32 * r + lane == best_j) key[r] = kSelected;
     tau = kSelected - 1u;
   } else {
-    tau = 0;
+    tau = kTopBits;  // largest tau with sum_{key >= tau} u >= T; its top two bits are known
 #pragma unroll 1
-    for (int b = 30; b >= 0; --b) {
+    for (int b = 28; b >= 0; --b) {
       const uint32_t c = tau | (1u << b);
       uint64_t g[4] = {0ull, 0ull, 0ull, 0ull};  // independent partial sums
 #pragma unroll
