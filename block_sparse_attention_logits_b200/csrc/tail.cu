@@ -17,13 +17,14 @@
 // Kernels:
 //   tail_moments_kernel   one CTA per (head, block): means and variances, the
 //                         bf16 operand tables of the tail kernel, and the
-//                         block-centred keys and values written transposed
-//                         ([D, L] per head) for the covariance contraction.
+//                         block-centred keys and values ([L, D] per head, the
+//                         layout of K and V) for the covariance contraction.
 //   cov_kernel            C as a tensor-core contraction over the tokens:
-//                         A = centred V^T, B = centred K^T (both K-major
-//                         128-byte-swizzled tiles of 128 rows x 128 tokens),
-//                         accumulated in TMEM; the tokens of a head are split
-//                         over several CTAs whose partial sums cov_reduce adds.
+//                         A = centred V^T, B = centred K^T, both read as
+//                         MN-major 128-byte-swizzled tiles of 128 tokens x 128
+//                         dimensions, accumulated in TMEM; the tokens of a head
+//                         are split over several CTAs whose partial sums
+//                         cov_reduce adds.
 //   coarse_tail_kernel    one CTA per query block: S = Q kbar^T + (Q o Q) s2h^T
 //                         over tiles of 128 pseudo-keys (one per key block),
 //                         kept blocks masked out, online softmax, O += P vbar,
@@ -81,25 +82,27 @@ __device__ __forceinline__ bool warp_wait_for(uint64_t* bar, uint32_t parity, in
 // grid (NB, B*H), 256 threads.  Writes (all per head bh, block j):
 //   kbar, s2, vbar       float32 [bh][j][d]
 //   tabK = bf16(kbar), tabS = bf16(s2 / (2 sqrt(D))), tabV = bf16(vbar)   [bh][j][d]
-//   kcT, vcT             bf16 [bh][d][t] (row length Lp): the block-centred values
+//   kc, vc               bf16 [bh][t][d]: the block-centred keys and values
 // The block's keys, then its values, are read once from HBM with 16-byte
 // loads into shared memory; each (dimension, token part) thread sums its part
-// and the parts are combined; the centred values go out transposed, 8 tokens
-// (16 bytes) per store.  HBM-bound: K and V read once, kcT and vcT written.
+// and the parts are combined; the centred values go back out 16 bytes per
+// store in the input's layout.  HBM-bound: K and V read once, kc and vc
+// written once.
 constexpr int kMomThreads = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kMomThreads) tail_moments_kernel(const __nv_bfloat16* __restrict__ k,
                                                                    const __nv_bfloat16* __restrict__ v, int L,
-                                                                   int blk, int NB, int Lp, float* __restrict__ kbar,
+                                                                   int blk, int NB, float* __restrict__ kbar,
                                                                    float* __restrict__ s2, float* __restrict__ vbar,
                                                                    __nv_bfloat16* __restrict__ tabK,
                                                                    __nv_bfloat16* __restrict__ tabS,
                                                                    __nv_bfloat16* __restrict__ tabV,
-                                                                   __nv_bfloat16* __restrict__ kcT,
-                                                                   __nv_bfloat16* __restrict__ vcT) {
+                                                                   __nv_bfloat16* __restrict__ kc,
+                                                                   __nv_bfloat16* __restrict__ vc) {
   constexpr int VPR = D / 8;                // 16-byte vectors per token row
   constexpr int PARTS = kMomThreads / D;    // token parts per dimension
+  constexpr int PER = 128 * VPR / kMomThreads;  // vectors per thread (a full block)
   __shared__ __align__(16) __nv_bfloat16 buf[128 * D];  // one block of keys or values, [t][d]
   __shared__ float part[PARTS][D];
   __shared__ float mean_s[D];
@@ -112,16 +115,15 @@ __global__ void __launch_bounds__(kMomThreads) tail_moments_kernel(const __nv_bf
   const size_t o = (static_cast<size_t>(bh) * NB + j) * D + d;
 #pragma unroll 1
   for (int which = 0; which < 2; ++which) {
-    const __nv_bfloat16* src = (which ? v : k) + (bh * L + lo) * D;
+    const size_t base = (bh * L + lo) * D;
+    const uint4* src = reinterpret_cast<const uint4*>((which ? v : k) + base);
+    uint4* dst = reinterpret_cast<uint4*>((which ? vc : kc) + base);
+    uint4* b4 = reinterpret_cast<uint4*>(buf);
     __syncthreads();  // the previous pass has finished with buf
-    {
-      const uint4* s4 = reinterpret_cast<const uint4*>(src);
-      uint4* b4 = reinterpret_cast<uint4*>(buf);
 #pragma unroll
-      for (int r = 0; r < 128 * VPR / kMomThreads; ++r) {
-        const int e = tid + r * kMomThreads;
-        if (e < n * VPR) b4[e] = __ldg(s4 + e);
-      }
+    for (int r = 0; r < PER; ++r) {
+      const int e = tid + r * kMomThreads;
+      if (e < n * VPR) b4[e] = __ldg(src + e);
     }
     __syncthreads();
     // mean over the block's tokens
@@ -161,29 +163,23 @@ __global__ void __launch_bounds__(kMomThreads) tail_moments_kernel(const __nv_bf
       vbar[o] = mu;
       tabV[o] = __float2bfloat16_rn(mu);
     }
-    // centred values, transposed: thread item (t8, dd) writes tokens
-    // 8*t8 .. 8*t8+7 of dimension dd (consecutive threads: consecutive dd, so
-    // the shared-memory reads of a token row are conflict-free)
-    __nv_bfloat16* dstT = (which ? vcT : kcT) + static_cast<size_t>(bh) * D * Lp + lo;
-    const int n8 = (n + 7) / 8;
-    for (int item = tid; item < n8 * D; item += kMomThreads) {
-      const int t8 = item / D, dd = item % D;
-      const float m = mean_s[dd];
-      __nv_bfloat16* row = dstT + static_cast<size_t>(dd) * Lp + t8 * 8;
-      if (t8 * 8 + 8 <= n) {
-        uint32_t w[4];
+    // centred values in the input's layout: each thread its own vectors
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = __bfloat162float(buf[(t8 * 8 + 2 * e) * D + dd]) - m;
-          const float x1 = __bfloat162float(buf[(t8 * 8 + 2 * e + 1) * D + dd]) - m;
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(x0, x1);
-          w[e] = *reinterpret_cast<const uint32_t*>(&pr);
-        }
-        *reinterpret_cast<uint4*>(row) = make_uint4(w[0], w[1], w[2], w[3]);
-      } else {
-        for (int t = t8 * 8; t < n; ++t)
-          row[t - t8 * 8] = __float2bfloat16_rn(__bfloat162float(buf[t * D + dd]) - m);
+    for (int r = 0; r < PER; ++r) {
+      const int e = tid + r * kMomThreads;
+      if (e >= n * VPR) continue;
+      const uint4 x = b4[e];
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      const int d0 = (e % VPR) * 8;
+      uint32_t c[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float x0 = __uint_as_float(w[q] << 16) - mean_s[d0 + 2 * q];
+        const float x1 = __uint_as_float(w[q] & 0xFFFF0000u) - mean_s[d0 + 2 * q + 1];
+        const __nv_bfloat162 pr = __floats2bfloat162_rn(x0, x1);
+        c[q] = *reinterpret_cast<const uint32_t*>(&pr);
       }
+      dst[e] = make_uint4(c[0], c[1], c[2], c[3]);
     }
   }
 }
@@ -229,7 +225,10 @@ __global__ void __launch_bounds__(160, 1) cov_kernel(const __grid_constant__ CUt
   bool ok = true;
   if (warp == 4) {
     if (c0 < c1) {
-      constexpr uint32_t idC = idesc_bf16_f32(kRows, 128, false, false);
+      // A = centred V^T (M = value dimension), B = centred K^T (N = key
+      // dimension), K = tokens: both tiles are [128 tokens][128 dims], i.e.
+      // MN-major
+      constexpr uint32_t idC = idesc_bf16_f32(kRows, 128, true, true);
       // two stages: the load of chunk c overlaps the MMA of chunk c-1
       for (int c = c0; c < c1 && ok; ++c) {
         const int u = c - c0;
@@ -242,8 +241,8 @@ __global__ void __launch_bounds__(160, 1) cov_kernel(const __grid_constant__ CUt
           uint8_t* b = a + kTileBytes;
           mbar_arrive_expect_tx(&sh->full[st], 2 * kTileBytes);
           for (int p = 0; p < 2; ++p) {
-            tma_load_3d(a + p * kPanel, &tmVc, &sh->full[st], c * 128 + p * 64, 0, bh);
-            tma_load_3d(b + p * kPanel, &tmKc, &sh->full[st], c * 128 + p * 64, 0, bh);
+            tma_load_3d(a + p * kPanel, &tmVc, &sh->full[st], p * 64, c * 128, bh);
+            tma_load_3d(b + p * kPanel, &tmKc, &sh->full[st], p * 64, c * 128, bh);
           }
         }
         __syncwarp();
@@ -254,11 +253,9 @@ __global__ void __launch_bounds__(160, 1) cov_kernel(const __grid_constant__ CUt
           const uint32_t a = smem_u32(tiles + st * 2 * kTileBytes);
           const uint32_t b = a + kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-            mma_ss(tmem, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(b + off, 16, 1024), idC,
+          for (int kk = 0; kk < 8; ++kk)  // 16 tokens per step: 16 rows of 128 bytes
+            mma_ss(tmem, sdesc_sw128(a + kk * 2048, kPanel, 1024), sdesc_sw128(b + kk * 2048, kPanel, 1024), idC,
                    (u > 0 || kk > 0) ? 1u : 0u);
-          }
           tc_commit(&sh->empty[st]);
         }
         __syncwarp();
@@ -791,13 +788,13 @@ int splits_for(int BH) {
 }  // namespace tail
 
 // Workspace layout (bytes, each part 1024-aligned):
-//   kcT, vcT   bf16 [BH][D][Lp]           Lp = L rounded up to 64
+//   kc, vc     bf16 [BH][L][D]
 //   tabK, tabS, tabV  bf16 [BH][NB][D]
 //   tabC       bf16 [BH][D][D]
 //   part       f32  [splits][BH][D][D]
 struct TailWs {
-  size_t kcT, vcT, tabK, tabS, tabV, tabC, part, total;
-  int Lp, splits;
+  size_t kc, vc, tabK, tabS, tabV, tabC, part, total;
+  int splits;
 };
 
 static TailWs tail_ws_layout(const bsa_shape& s, int splits) {
@@ -805,11 +802,10 @@ static TailWs tail_ws_layout(const bsa_shape& s, int splits) {
   TailWs w;
   const size_t BH = static_cast<size_t>(s.B) * s.H;
   const int NB = n_blocks(s.L, s.blk);
-  w.Lp = (s.L + 63) & ~63;
   w.splits = splits;
   size_t o = 0;
-  w.kcT = o; o += up(BH * s.D * w.Lp * 2);
-  w.vcT = o; o += up(BH * s.D * w.Lp * 2);
+  w.kc = o; o += up(BH * s.L * s.D * 2);
+  w.vc = o; o += up(BH * s.L * s.D * 2);
   w.tabK = o; o += up(BH * NB * s.D * 2);
   w.tabS = o; o += up(BH * NB * s.D * 2);
   w.tabV = o; o += up(BH * NB * s.D * 2);
@@ -829,14 +825,14 @@ int launch_tail_stats(const bsa_shape& s, const __nv_bfloat16* k, const __nv_bfl
   const int splits = tail::splits_for(BH);
   const TailWs w = tail_ws_layout(s, splits);
   uint8_t* base = static_cast<uint8_t*>(ws);
-  auto* kcT = reinterpret_cast<__nv_bfloat16*>(base + w.kcT);
-  auto* vcT = reinterpret_cast<__nv_bfloat16*>(base + w.vcT);
+  auto* kc = reinterpret_cast<__nv_bfloat16*>(base + w.kc);
+  auto* vc = reinterpret_cast<__nv_bfloat16*>(base + w.vc);
   tail::tail_moments_kernel<128><<<dim3(NB, BH), tail::kMomThreads, 0, st>>>(
-      k, v, s.L, s.blk, NB, w.Lp, kbar, s2, vbar, reinterpret_cast<__nv_bfloat16*>(base + w.tabK),
-      reinterpret_cast<__nv_bfloat16*>(base + w.tabS), reinterpret_cast<__nv_bfloat16*>(base + w.tabV), kcT, vcT);
+      k, v, s.L, s.blk, NB, kbar, s2, vbar, reinterpret_cast<__nv_bfloat16*>(base + w.tabK),
+      reinterpret_cast<__nv_bfloat16*>(base + w.tabS), reinterpret_cast<__nv_bfloat16*>(base + w.tabV), kc, vc);
   if (cudaGetLastError() != cudaSuccess) return BSA_ECUDA;
   CUtensorMap mVc, mKc;
-  if (!tail::map3(&mVc, vcT, s.L, 128, BH, w.Lp) || !tail::map3(&mKc, kcT, s.L, 128, BH, w.Lp)) return BSA_ECUDA;
+  if (!tail::map3(&mVc, vc, 128, s.L, BH, 128) || !tail::map3(&mKc, kc, 128, s.L, BH, 128)) return BSA_ECUDA;
   constexpr int kCovSmem = 4 * tail::kTileBytes + 1024 + 1024;
   if (smem_opt_in(reinterpret_cast<const void*>(tail::cov_kernel), kCovSmem) != cudaSuccess) return BSA_ECUDA;
   float* part = reinterpret_cast<float*>(base + w.part);
