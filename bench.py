@@ -270,10 +270,12 @@ def oracle_sample(w, p, seconds, max_blocks=None):
 
 # ------------------------------------------------------------------- ours
 
-def interval_timings(idx, cnt, L, blk, D, barrier, q=0.95):
+def interval_timings(idx, cnt, L, blk, D, barrier, q=0.95, qkv=None):
     """The interval (skip-list) form of a step's kept lists: per-row runs and
     their histogram, the width for merge percentage q, encode and decode
-    (decode writes kept lists only); times in ms per call, sizes in bytes."""
+    (decode writes kept lists only); with qkv (the attention's inputs, blk
+    128) also the attention walking the merged pairs against the attention
+    over the lists they decode to; times in ms per call, sizes in bytes."""
     from block_sparse_attention_logits_b200 import api
     B, H, nb = cnt.shape
     dev = cnt.device
@@ -287,10 +289,17 @@ def interval_timings(idx, cnt, L, blk, D, barrier, q=0.95):
     n_int, nr2 = torch.empty_like(cnt), torch.empty_like(cnt)
     kidx, kcnt = torch.empty_like(idx), torch.empty_like(cnt)
     scratch = torch.zeros_like(hist)
-    calls = (("runs", lambda: api.interval_runs(idx, cnt, L, blk, D, n_runs=nr2, hist=scratch, status=st)),
+    calls = [("runs", lambda: api.interval_runs(idx, cnt, L, blk, D, n_runs=nr2, hist=scratch, status=st)),
              ("encode", lambda: api.kept_to_intervals(idx, cnt, Wq, L, blk, D, iv, n_int, nr2, st)),
              ("decode", lambda: api.intervals_to_kept(iv, n_int, L, blk, D, kept_idx=kidx, kept_cnt=kcnt,
-                                                      want_mask=False, status=st)))
+                                                      want_mask=False, status=st))]
+    if qkv is not None and blk == 128:
+        qa, ka, va = qkv
+        oa, la = torch.empty_like(qa), torch.empty(qa.shape[:3], dtype=torch.float32, device=dev)
+        calls += [("attention_walking_intervals",
+                   lambda: api.sparse_attn_fwd_intervals(qa, ka, va, blk, iv, n_int, o=oa, lse=la, status=st)),
+                  ("attention_on_decoded_lists",
+                   lambda: api.sparse_attn_fwd(qa, ka, va, blk, kidx, kcnt, o=oa, lse=la, status=st))]
     ms = {}
     for name, fn in calls:
         fn()
@@ -304,7 +313,11 @@ def interval_timings(idx, cnt, L, blk, D, barrier, q=0.95):
         ms[name] = round(a0.elapsed_time(a1) / 10, 4)
     rows = B * H * nb
     before = cnt.double().sum().item()
-    return {"runs_ms": ms["runs"], "encode_ms": ms["encode"], "decode_ms": ms["decode"],
+    extra = {}
+    if "attention_walking_intervals" in ms:
+        extra = {"attention_walking_intervals_ms": ms["attention_walking_intervals"],
+                 "attention_on_decoded_lists_ms": ms["attention_on_decoded_lists"]}
+    return {"runs_ms": ms["runs"], "encode_ms": ms["encode"], "decode_ms": ms["decode"], **extra,
             "merge_q": q, "width_at_q": Wq, "width_max": Wmax, "max_possible": api.max_intervals(nb),
             "runs_per_row_mean": round(n_runs.double().mean().item(), 2),
             "rows_merged_frac": round((n_runs > Wq).double().mean().item(), 4),
@@ -610,7 +623,8 @@ def run_ours(args, w, world, rank, local):
     intervals = None
     if not args.no_refresh:
         try:
-            intervals = interval_timings(bufs["idx"], bufs["cnt"], L, blk, D, barrier)
+            qkv_ = (bufs["qh"], bufs["kh"], bufs["vh"]) if w.hilbert else (q, k, v)
+            intervals = interval_timings(bufs["idx"], bufs["cnt"], L, blk, D, barrier, qkv=qkv_)
         except Exception as e:  # noqa: BLE001
             intervals = {"error": f"{type(e).__name__}: {e}"}
 

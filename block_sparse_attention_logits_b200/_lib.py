@@ -19,7 +19,7 @@ EXPORTS = (
     "bsa_complement_lists", "bsa_quantize_fp8", "bsa_sparse_attn_fwd_fp8",
     "bsa_wait_selftest",
     "bsa_reorder_workspace_bytes", "bsa_reorder_tokens", "bsa_reorder_tokens_noalloc", "bsa_permute_tokens",
-    "bsa_sparse_attn_fwd", "bsa_sparse_attn_fwd_scatter", "bsa_sparse_attn_fwd_gather", "bsa_sparse_attn_refresh", "bsa_refresh_refinement", "bsa_apply_correction",
+    "bsa_sparse_attn_fwd", "bsa_sparse_attn_fwd_scatter", "bsa_sparse_attn_fwd_gather", "bsa_sparse_attn_fwd_intervals", "bsa_sparse_attn_refresh", "bsa_refresh_refinement", "bsa_apply_correction",
 )
 
 BSA_OK, BSA_EINVAL, BSA_ESHAPE, BSA_ENODEV, BSA_ECUDA, BSA_EWORKSPACE = range(6)
@@ -85,6 +85,7 @@ def load():
         "bsa_sparse_attn_fwd": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_sparse_attn_fwd_scatter": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_sparse_attn_fwd_gather": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "bsa_sparse_attn_fwd_intervals": (_I, [Shape, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P]),
         "bsa_sparse_attn_refresh": (_I, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "bsa_refresh_refinement": (_I, [Shape, _P, _P, _P, _P]),
         "bsa_apply_correction": (_I, [Shape, _P, _P, _P, _P, _P]),

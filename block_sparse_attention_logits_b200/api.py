@@ -486,6 +486,35 @@ def sparse_attn_fwd(q, k, v, blk, kept_idx=None, kept_cnt=None, R=None, alpha=No
     return o, lse
 
 
+def sparse_attn_fwd_intervals(q, k, v, blk, intervals, n_int, R=None, alpha=None, o=None, lse=None, status=None):
+    """Block-sparse attention with the kept blocks given as interval pairs
+    (int32 [B,H,NB,W,2] and int32 [B,H,NB], as kept_to_intervals returns
+    them), walked by the kernel itself; blk 128.  Same result as
+    sparse_attn_fwd on intervals_to_kept of the same pairs."""
+    B, H, L, D = q.shape
+    nb = n_blocks(L, blk)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, torch.bfloat16, (B, H, L, D), name)
+    if intervals.dim() != 5:
+        raise ValueError("intervals must be int32 [B,H,NB,W,2]")
+    W = intervals.shape[3]
+    _need(intervals, torch.int32, (B, H, nb, W, 2), "intervals")
+    _need(n_int, torch.int32, (B, H, nb), "n_int")
+    if R is not None:
+        _need(R, torch.bfloat16, (B, H, L, D), "R")
+        _need(alpha, torch.float32, (H,), "alpha")
+    o = o if o is not None else torch.empty_like(q)
+    lse = lse if lse is not None else torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    _need(o, torch.bfloat16, (B, H, L, D), "o")
+    _need(lse, torch.float32, (B, H, L), "lse")
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
+    check("bsa_sparse_attn_fwd_intervals", _lib.load().bsa_sparse_attn_fwd_intervals(
+        Shape(B, H, L, D, blk), _ptr(q), _ptr(k), _ptr(v), _ptr(intervals), _ptr(n_int), W,
+        _ptr(R), _ptr(alpha), _ptr(o), _ptr(lse), _ptr(status), _stream()))
+    return o, lse
+
+
 def sparse_attn_refresh(q, k, v, blk, kept_idx, kept_cnt, want_r=True, want_mass=True, out=None, status=None):
     """Dense refresh in one pass over every key block.
 

@@ -390,6 +390,35 @@ int bsa_sparse_attn_fwd_gather(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k
   return bsa::launch_sparse_attn(s, a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int bsa_sparse_attn_fwd_intervals(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
+                                  const int32_t* intervals, const int32_t* n_int, int W, const bsa_bf16* R,
+                                  const float* alpha, bsa_bf16* o, float* lse, int32_t* status, bsa_stream stream) {
+  if (!q || !k || !v || !intervals || !n_int || !o || !lse) return BSA_EINVAL;
+  if ((R == nullptr) != (alpha == nullptr)) return BSA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return BSA_EINVAL;
+  if (!word_ok(intervals) || !word_ok(n_int) || (R && !aligned16(R))) return BSA_EINVAL;
+  if (!word_ok(status) || !word_ok(alpha)) return BSA_EINVAL;
+  if (int r = check_block_shape(s)) return r;
+  if (s.blk != 128) return BSA_ESHAPE;
+  if (W < 1 || W > n_blocks(s.L, s.blk)) return BSA_EINVAL;
+  if (int r = check_device()) return r;
+  bsa::AttnArgs a;
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  a.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  a.kept_idx = nullptr;
+  a.kept_cnt = nullptr;
+  a.intervals = intervals;
+  a.n_int = n_int;
+  a.W = W;
+  a.R = reinterpret_cast<const __nv_bfloat16*>(R);
+  a.alpha = alpha;
+  a.o = reinterpret_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.status = status;
+  return bsa::launch_sparse_attn(s, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int bsa_quantize_fp8(bsa_shape s, const bsa_bf16* x, uint8_t* codes, float* scales, bsa_stream stream) {
   if (!x || !codes || !scales) return BSA_EINVAL;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return BSA_EINVAL;

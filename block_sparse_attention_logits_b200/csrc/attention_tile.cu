@@ -151,6 +151,10 @@ struct Params {
   float scale_log2;
   int dense;
   int sched_slot;
+  // interval mode: the kept blocks as pairs [B,H,NB,W,2] and pairs per row [B,H,NB]
+  const int32_t* intervals;
+  const int32_t* n_int;
+  int W;
 };
 
 // kF8: Q and K are E4M3 (one byte per element), S = Q.K^T runs as a
@@ -328,7 +332,7 @@ __device__ __forceinline__ int next_item(int i, Shared* sh, const Params& prm) {
 struct Item {
   int bh, qb, cnt;
   const int32_t* list;   // null in dense mode
-  bool bad_cnt;          // the count was outside [0, NB] and was clamped
+  bool bad_cnt;          // the count was outside [0, NB] and was clamped (interval mode: malformed pairs)
   const int32_t* klist;  // fused refresh: the kept list (ascending) ...
   int kcnt;              // ... and its length
 };
@@ -366,6 +370,67 @@ __device__ __forceinline__ Item item_of(int w, const Params& prm) {
 __device__ __forceinline__ int entry_kb(const Item& it, int n, int NB) {
   const int kb = it.list ? __ldg(it.list + n) : n;
   return static_cast<unsigned>(kb) < static_cast<unsigned>(NB) ? kb : -1;
+}
+
+// Interval mode (CalibAtt appendix, Fig. S10: the kernel walks the skip
+// lists): the item carries its row's (start, end) pairs, checked as the decode
+// checks them (ascending, within [0, NB], non-empty; a malformed row is empty
+// and flagged), and every role walks them in order with its own cursor.
+struct ItemIv : Item {
+  const int32_t* pairs;
+};
+struct Walk {
+  int p = -1, kb = 0, end = 0;
+};
+
+__device__ __forceinline__ ItemIv item_iv_of(int w, const Params& prm) {
+  ItemIv it;
+  it.bh = w / prm.NT;
+  it.qb = w - it.bh * prm.NT;
+  it.klist = nullptr;
+  it.kcnt = 0;
+  it.list = nullptr;
+  const size_t r = static_cast<size_t>(it.bh) * prm.NB + it.qb;
+  const int ni = __ldg(prm.n_int + r);
+  it.pairs = prm.intervals + r * prm.W * 2;
+  bool bad = ni < 0 || ni > prm.W;
+  int cnt = 0, prev = 0;
+  for (int p = 0; !bad && p < ni; ++p) {
+    const int a = __ldg(it.pairs + 2 * p), b = __ldg(it.pairs + 2 * p + 1);
+    bad = a < prev || a >= b || b > prm.NB;
+    cnt += b - a;
+    prev = b;
+  }
+  it.bad_cnt = bad;
+  it.cnt = bad ? 0 : cnt;
+  return it;
+}
+
+// The next key block of a validated row (entries visited in order).
+__device__ __forceinline__ int entry_kb(const ItemIv& it, int, int, Walk& w) {
+  while (w.kb >= w.end) {
+    ++w.p;
+    w.kb = __ldg(it.pairs + 2 * w.p);
+    w.end = __ldg(it.pairs + 2 * w.p + 1);
+  }
+  return w.kb++;
+}
+
+template <bool kFused, bool kIntervals>
+__device__ __forceinline__ auto item_at(int w, const Params& prm) {
+  if constexpr (kIntervals)
+    return item_iv_of(w, prm);
+  else
+    return item_of<kFused>(w, prm);
+}
+
+// Key block of entry n in either mode (the cursor is used by interval mode only).
+template <bool kIntervals, class It>
+__device__ __forceinline__ int next_kb(const It& it, int n, int NB, Walk& w) {
+  if constexpr (kIntervals)
+    return entry_kb(it, n, NB, w);
+  else
+    return entry_kb(it, n, NB);
 }
 
 // Fused refresh: is key block j (visited in ascending order) in the kept list?
@@ -413,12 +478,13 @@ __device__ __forceinline__ void gather_tile(uint8_t* dst, const CUtensorMap* map
     tma_gather4(dst + pnl * (BM * 128) + lane * 512, map, bar, pnl * 64, g[0], g[1], g[2], g[3]);
 }
 
-template <int D, bool kFused, bool kF8, bool kGather>
+template <int D, bool kFused, bool kF8, bool kGather, bool kIntervals>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const Params prm) {
   using C = Cfg<D, kF8>;
   static_assert(!kGather || (D == 128 && !kFused && !kF8), "row gathers: bf16, D = 128, not the fused refresh");
+  static_assert(!kIntervals || (!kFused && !kF8 && !kGather), "interval pairs: bf16, not the fused refresh");
   // TMEM (512 columns): NS buffers of S (128 columns each) then OB buffers of
   // the accumulator(s) of an item (D columns each; the fused refresh keeps two
   // per item, OK and OR).  D = 128: S0|S1|S2|O, fused S0|S1|OK|OR.
@@ -510,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         w = __shfl_sync(0xffffffffu, w, 0);
         if (w < 0) break;
-        const Item it = item_of<kFused>(w, prm);
+        const auto it = item_at<kFused, kIntervals>(w, prm);
         if (it.bad_cnt && lane == 0) flag_status(prm, BSA_DEV_BAD_INDEX);
         const int qb = i % C::NQ;
         if (i >= C::NQ && !(ok = warp_wait(&sh->q_empty[qb], ((i - C::NQ) / C::NQ) & 1, sh, prm))) break;
@@ -526,8 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         it.bh);
         }
         __syncwarp();
+        Walk wk;
         for (int n = 0; ok && n < it.cnt; ++n) {
-          const int kb = entry_kb(it, n, NB);
+          const int kb = next_kb<kIntervals>(it, n, NB, wk);
           if (kb < 0) {
             if (lane == 0) flag_status(prm, BSA_DEV_BAD_INDEX);
             continue;
@@ -561,9 +628,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; ok; ++i) {
         const int w = next_item(i, sh, prm);
         if (w < 0) break;
-        const Item it = item_of<kFused>(w, prm);
+        const auto it = item_at<kFused, kIntervals>(w, prm);
+        Walk wk;
         for (int n = 0; n < it.cnt; ++n) {
-          const int kb = entry_kb(it, n, NB);
+          const int kb = next_kb<kIntervals>(it, n, NB, wk);
           if (kb < 0) continue;
           const int slot = u % NSV;
           if (u >= NSV && !(ok = warp_wait(&sh->empty_v[slot], ((u / NSV) - 1) & 1, sh, prm))) break;
@@ -594,12 +662,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; ok; ++i) {
         const int w = next_item(i, sh, prm);
         if (w < 0) break;
-        const Item it = item_of<kFused>(w, prm);
+        const auto it = item_at<kFused, kIntervals>(w, prm);
         const int qb = i % C::NQ;
         if (!(ok = warp_wait(&sh->q_full[qb], (i / C::NQ) & 1, sh, prm))) break;
         const uint32_t qa = q_base + qb * C::Q_BYTES;
+        Walk wk;
         for (int n = 0; n < it.cnt; ++n) {
-          if (entry_kb(it, n, NB) < 0) continue;
+          if (next_kb<kIntervals>(it, n, NB, wk) < 0) continue;
           const int sk = u % NSK;
           const int b = u % NS;
           if (!(ok = warp_wait(&sh->full_k[sk], (u / NSK) & 1, sh, prm))) break;
@@ -643,14 +712,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; ok; ++i) {
         const int w = next_item(i, sh, prm);
         if (w < 0) break;
-        const Item it = item_of<kFused>(w, prm);
+        const auto it = item_at<kFused, kIntervals>(w, prm);
         const int ob = i % OB;
         if (i >= OB && !(ok = warp_wait(&sh->o_empty[ob], ((i - OB) / OB) & 1, sh, prm))) break;
         bool first = true, first_rest = true;
         int kp = 0;
         bool bad = false;
+        Walk wk;
         for (int n = 0; n < it.cnt; ++n) {
-          const int kb = entry_kb(it, n, NB);
+          const int kb = next_kb<kIntervals>(it, n, NB, wk);
           if (kb < 0) continue;
           const bool kept = !kFused || kept_at(it, kb, kp, bad);
           const int sv = u % NSV;
@@ -701,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; ok; ++i) {
       const int w = next_item(i, sh, prm);
       if (w < 0) break;
-      const Item it = item_of<kFused>(w, prm);
+      const auto it = item_at<kFused, kIntervals>(w, prm);
       const int ob = i % OB;
       const int sb = i & 1;  // statistics buffer
       const uint32_t tO = tmem + lane_off + COL_O + ob * D;
@@ -716,13 +786,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool bad = false;
       // FP8: the K block scale of list entry n, loaded one block ahead
       const float* ks_row = kF8 ? prm.k_scale + static_cast<size_t>(it.bh) * prm.NB : nullptr;
-      auto k_scale_at = [&](int n) {
-        const int kb = entry_kb(it, n, NB);
+      auto k_scale_at = [&](int n) {  // list mode only (the FP8 path takes no intervals)
+        const int kb = entry_kb(static_cast<const Item&>(it), n, NB);
         return kb >= 0 ? __ldg(ks_row + kb) : 1.f;
       };
       float ks_next = kF8 && it.cnt > 0 ? k_scale_at(0) : 1.f;
+      Walk wk;
       for (int n = 0; n < it.cnt; ++n) {
-        const int kb = entry_kb(it, n, NB);
+        const int kb = next_kb<kIntervals>(it, n, NB, wk);
         float ks = 1.f;
         if constexpr (kF8) {
           ks = ks_next;
@@ -893,7 +964,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; ok; ++i) {
       const int w = next_item(i, sh, prm);
       if (w < 0) break;
-      const Item it = item_of<kFused>(w, prm);
+      const auto it = item_at<kFused, kIntervals>(w, prm);
       const int ob = i % OB;
       const int sb = i & 1;
       if (!(ok = warp_wait(&sh->o_full[ob], (i / OB) & 1, sh, prm))) break;
@@ -1098,10 +1169,11 @@ bool make_map8(CUtensorMap* m, const void* base, int D, int L, int BH, int box_r
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool kFused, bool kF8 = false, bool kGather = false>
+template <int D, bool kFused, bool kF8 = false, bool kGather = false, bool kIntervals = false>
 int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   using C = Cfg<D, kF8>;
-  if (smem_opt_in(reinterpret_cast<const void*>(sparse_attn_tile_kernel<D, kFused, kF8, kGather>), C::SMEM_BYTES) !=
+  if (smem_opt_in(reinterpret_cast<const void*>(sparse_attn_tile_kernel<D, kFused, kF8, kGather, kIntervals>),
+                  C::SMEM_BYTES) !=
       cudaSuccess)
     return BSA_ECUDA;
   const int BH = s.B * s.H;
@@ -1134,6 +1206,9 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   prm.q_scale = a.q_scale;
   prm.k_scale = a.k_scale;
   prm.in_rows = a.in_rows;
+  prm.intervals = a.intervals;
+  prm.n_int = a.n_int;
+  prm.W = a.W;
   prm.n_rows = static_cast<int>(n_rows < (1ll << 31) ? n_rows : 0);
   prm.H = s.H;
   prm.L = s.L;
@@ -1141,12 +1216,13 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   prm.NT = prm.NB;  // one work item per 128-token query block
   prm.n_work = BH * prm.NT;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  prm.dense = a.kept_idx == nullptr;
+  prm.dense = a.kept_idx == nullptr && a.intervals == nullptr;
   static std::atomic<unsigned int> launches{0};
   prm.sched_slot = static_cast<int>(launches.fetch_add(1u) % kSchedSlots);
   const int sms = sm_count();
   const int grid = prm.n_work < sms ? prm.n_work : sms;
-  sparse_attn_tile_kernel<D, kFused, kF8, kGather><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, prm);
+  sparse_attn_tile_kernel<D, kFused, kF8, kGather, kIntervals><<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv,
+                                                                                                      prm);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ECUDA;
 }
 
@@ -1154,6 +1230,12 @@ int run(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
 
 int launch_sparse_attn_tile(const bsa_shape& s, const AttnArgs& a, cudaStream_t st) {
   if (s.blk != 128) return BSA_ESHAPE;
+  if (a.intervals) {
+    if (a.o2 || a.q8 || a.in_rows) return BSA_ESHAPE;
+    if (s.D == 128) return tile_attn::run<128, false, false, false, true>(s, a, st);
+    if (s.D == 64) return tile_attn::run<64, false, false, false, true>(s, a, st);
+    return BSA_ESHAPE;
+  }
   if (a.in_rows) {
     if (s.D == 128 && !a.o2 && !a.q8) return tile_attn::run<128, false, false, true>(s, a, st);
     return BSA_ESHAPE;

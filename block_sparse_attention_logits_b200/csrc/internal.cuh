@@ -103,6 +103,11 @@ struct AttnArgs {
   // is row in_rows[t] of q, k and v (loaded by row gathers), and R is read in
   // the order of o (nullable = q, k, v already in the attention's order)
   const int32_t* in_rows = nullptr;
+  // blk = 128, bf16, not the fused refresh: the kept blocks as interval pairs
+  // (intervals [B,H,NB,W,2], n_int [B,H,NB]) instead of kept_idx / kept_cnt
+  const int32_t* intervals = nullptr;
+  const int32_t* n_int = nullptr;
+  int W = 0;
   // FP8 Q.K^T (blk = 128, D = 128): E4M3 codes of Q and K ([B,H,L,D] bytes) and
   // their dequantization scales per (b, h, 128-token block); non-null q8
   // selects it (q and k are then unused)

@@ -441,6 +441,25 @@ BSA_API int bsa_sparse_attn_fwd_gather(bsa_shape s, const bsa_bf16* q, const bsa
                                        int32_t* status, bsa_stream stream);
 
 /*
+ * bsa_sparse_attn_fwd_intervals -- bsa_sparse_attn_fwd with the kept blocks
+ * given as interval pairs, walked by the attention kernel itself (CalibAtt
+ * appendix, Fig. S10: the skip lists are what the kernel reads); no decode to
+ * padded lists.  intervals: device int32 [B,H,NB,W,2] and n_int: device int32
+ * [B,H,NB], as bsa_kept_to_intervals writes them (a row's first n_int pairs
+ * (start, end), end exclusive, ascending).  The result equals
+ * bsa_sparse_attn_fwd on the lists bsa_intervals_to_kept decodes from the
+ * same pairs, bit for bit.  A malformed row (n_int outside [0, W], or a pair
+ * with start < the previous end, start >= end or end > NB) is attended as
+ * empty (O = 0, LSE = -inf) and sets BSA_DEV_BAD_INDEX.
+ * Other arguments and errors as bsa_sparse_attn_fwd; 1 <= W <= NB (BSA_EINVAL
+ * otherwise); s.blk must be 128 (BSA_ESHAPE otherwise).
+ */
+BSA_API int bsa_sparse_attn_fwd_intervals(bsa_shape s, const bsa_bf16* q, const bsa_bf16* k, const bsa_bf16* v,
+                                          const int32_t* intervals, const int32_t* n_int, int W,
+                                          const bsa_bf16* R, const float* alpha, bsa_bf16* o, float* lse,
+                                          int32_t* status, bsa_stream stream);
+
+/*
  * FP8 Q.K^T.  Defines: the sparse attention of a distilled pipeline run in
  * FP8 with fused kernels (abstract on the page titled RECAP).  The page gives
  * no format or scaling rule; here Q and K are quantized to OCP E4M3 (max 448,

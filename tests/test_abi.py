@@ -319,3 +319,19 @@ def test_fp8_validation(lib):
                                        *out) == _lib.BSA_ESHAPE
     assert lib.bsa_sparse_attn_fwd_fp8(Shape(1, 2, 1000, 128, 64), q8, qs, k8, ks, v, *none4,
                                        *out) == _lib.BSA_ESHAPE
+
+
+def test_interval_attention_validation(lib):
+    s = Shape(1, 2, 1000, 128, 128)  # NB = 8
+    qkv = [FAKE, ctypes.c_void_p(2 << 20), ctypes.c_void_p(3 << 20)]
+    iv, ni = ctypes.c_void_p(4 << 20), ctypes.c_void_p(5 << 20)
+    tail = (NULL, NULL, ctypes.c_void_p(6 << 20), ctypes.c_void_p(7 << 20), NULL, NULL)  # R, alpha, o, lse, status, stream
+    assert lib.bsa_sparse_attn_fwd_intervals(s, *qkv, NULL, ni, 2, *tail) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd_intervals(s, *qkv, iv, NULL, 2, *tail) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd_intervals(s, *qkv, ctypes.c_void_p(iv.value + 2), ni, 2, *tail) == _lib.BSA_EINVAL
+    # the width: 1 <= W <= NB
+    assert lib.bsa_sparse_attn_fwd_intervals(s, *qkv, iv, ni, 0, *tail) == _lib.BSA_EINVAL
+    assert lib.bsa_sparse_attn_fwd_intervals(s, *qkv, iv, ni, 9, *tail) == _lib.BSA_EINVAL
+    # 128-token blocks only; R without alpha
+    assert lib.bsa_sparse_attn_fwd_intervals(Shape(1, 2, 1000, 128, 64), *qkv, iv, ni, 2, *tail) == _lib.BSA_ESHAPE
+    assert lib.bsa_sparse_attn_fwd_intervals(s, *qkv, iv, ni, 2, FAKE, NULL, *tail[2:]) == _lib.BSA_EINVAL

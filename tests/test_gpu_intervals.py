@@ -3,7 +3,8 @@ row and their histogram, the width for a merge percentage, encoding at several
 widths (rows with more runs are merged) and decoding back to the mask and kept
 lists -- all bit-exact; malformed rows are flagged and emptied; attention over
 decoded merged lists matches the oracle's masked attention over the merged
-blocks."""
+blocks; the attention walking the pairs itself equals the attention over the
+decoded lists bit for bit, and attends malformed rows as empty."""
 
 import numpy as np
 import pytest
@@ -151,3 +152,70 @@ def test_attention_over_decoded_merged_lists_matches_oracle():
     _, ki_ref, kc_ref = oint.intervals_to_kept(iv_ref, ni_ref, NB)
     O, LSE = oatt.masked_attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), ki_ref, kc_ref, blk)
     assert_attention_close(to_np(o), to_np(lse), O, LSE, "attention over merged intervals")
+
+
+@pytest.mark.parametrize("merge", [False, True], ids=["all-runs", "merged-W2"])
+def test_attention_walking_intervals_matches_lists_and_oracle(merge):
+    """bsa_sparse_attn_fwd_intervals walks the pairs itself: bit for bit the
+    attention over the lists the same pairs decode to, and within tolerance of
+    the oracle's masked attention over them.  6 x 40 rows over 148 SMs run
+    several items per CTA; random rows include empty and full ones."""
+    B, H, D, blk = 1, 6, 128, 128
+    L = 39 * blk + 40
+    NB = (L + blk - 1) // blk
+    q, k, v = (random_bf16((B, H, L, D), 120 + j) for j in range(3))
+    R = random_bf16((B, H, L, D), 124, scale=0.05)
+    alpha = torch.linspace(0.0, 1.0, H, dtype=torch.float32)
+    idx, cnt = random_kept_lists(B, H, NB, 125, 0.3, 2.0)
+    W = 2 if merge else oint.max_intervals(NB)
+    iv, n_int, _ = api.kept_to_intervals(_dev(idx), _dev(cnt), W, L, blk)
+    _, ki, kc = api.intervals_to_kept(iv, n_int, L, blk, want_mask=False)
+    qd, kd, vd, Rd, ad = q.to(DEV), k.to(DEV), v.to(DEV), R.to(DEV), alpha.to(DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o1, l1 = api.sparse_attn_fwd_intervals(qd, kd, vd, blk, iv, n_int, Rd, ad, status=st)
+    o2, l2 = api.sparse_attn_fwd(qd, kd, vd, blk, ki, kc, Rd, ad, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.equal(o1, o2)
+    assert torch.equal(l1, l2)
+    iv_ref, ni_ref, _ = oint.kept_to_intervals(idx, cnt, W)
+    _, ki_ref, kc_ref = oint.intervals_to_kept(iv_ref, ni_ref, NB)
+    O, LSE = oatt.masked_attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), ki_ref, kc_ref, blk)
+    O = O + alpha.numpy()[None, :, None, None] * R.float().numpy()
+    assert_attention_close(to_np(o1), to_np(l1), O, LSE, "attention walking intervals")
+
+
+def test_attention_walking_malformed_intervals_is_flagged_and_empty():
+    B, H, D, blk = 1, 2, 128, 128
+    L = 6 * blk
+    NB = L // blk
+    q, k, v = (random_bf16((B, H, L, D), 130 + j) for j in range(3))
+    idx, cnt = random_kept_lists(B, H, NB, 133, 0.4, 1.5)
+    W = oint.max_intervals(NB)
+    iv_ref, ni_ref, _ = oint.kept_to_intervals(idx, cnt, W)
+    bad = iv_ref.copy()
+    nb = ni_ref.copy()
+    nb[0, 0, 1] = W + 1                       # more pairs than the width
+    bad[0, 1, 2, 0] = [3, 3]                  # an empty pair
+    nb[0, 1, 2] = max(nb[0, 1, 2], 1)
+    bad[0, 1, 3, 0] = [0, NB + 1]             # past NB
+    nb[0, 1, 3] = max(nb[0, 1, 3], 1)
+    bad[0, 0, 4, :2] = [[2, 4], [1, 3]]       # out of order
+    nb[0, 0, 4] = 2
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, lse = api.sparse_attn_fwd_intervals(q.to(DEV), k.to(DEV), v.to(DEV), blk, _dev(bad), _dev(nb), status=st)
+    torch.cuda.synchronize()
+    assert st.item() & BSA_DEV_BAD_INDEX
+    on, ln = to_np(o), to_np(lse)
+    for (h, i) in ((0, 1), (1, 2), (1, 3), (0, 4)):
+        rows = slice(i * blk, (i + 1) * blk)
+        assert not on[0, h, rows].any() and np.all(np.isneginf(ln[0, h, rows]))
+    # the well-formed rows: the oracle over their decoded lists
+    good = np.ones((B, H, NB), bool)
+    for (h, i) in ((0, 1), (1, 2), (1, 3), (0, 4)):
+        good[0, h, i] = False
+    _, ki_ref, kc_ref = oint.intervals_to_kept(iv_ref, ni_ref, NB)
+    units = [(0, h, i) for h in range(H) for i in range(NB) if good[0, h, i]]
+    O, LSE = oatt.masked_attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), ki_ref, kc_ref, blk,
+                                   units=units)
+    assert_attention_close(on, ln, O, LSE, "well-formed rows")
