@@ -7,14 +7,16 @@
 // exponent and mantissa, T = ceil(p * sum u) in IEEE double.  The kept set is
 // the shortest prefix of the (P desc, index asc) order whose u-sum is >= T.
 //
-// No sort is needed.  One warp per row finds, by a 31-step bitwise search,
-// the largest key threshold tau with  sum_{key >= tau} u >= T.  Every block
-// with key > tau is kept; blocks with key == tau are kept in ascending index
-// order while the running mass is still below T (a warp prefix scan).  All
-// sums are exact uint64 integer sums, so the result does not depend on the
-// order of summation and equals the sequential definition bit for bit.
-// Rows of up to 1024 blocks keep their keys and masses in registers
-// (select_reg_kernel); longer rows stage them in shared memory.
+// No sort is needed.  One warp per row finds, by a bitwise search (at most
+// 29 steps: the top bits are known), the largest key threshold tau with
+// sum_{key >= tau} u >= T.  Every block with key > tau is kept; blocks with
+// key == tau are kept in ascending index order while the running mass is
+// still below T (a warp prefix scan).  Every decision rests on exact integer
+// sums, so the result does not depend on the order of summation and equals
+// the sequential definition bit for bit.  Rows of up to 1024 blocks keep
+// their keys in registers (select_reg_kernel), which also decides most search
+// steps on 32-bit coarse masses and stops the search as soon as a single key
+// value is left in play; longer rows stage keys and masses in shared memory.
 //
 // Restricted form (GSRS abstract: later searches restricted to an early
 // candidate set): with a candidate mask the search runs over the candidate
@@ -30,6 +32,10 @@ constexpr uint32_t kSelected = 0xFFFFFFFFu;  // marker: above every real key
 // (key >= 0x2B800000), and no key exceeds 1.0f (0x3F800000): bit 30 of tau is
 // 0 and bit 29 is 1, so the search starts at bit 28
 constexpr uint32_t kTopBits = 0x20000000u;
+constexpr uint32_t kMinMassKey = 0x2B800000u;  // smallest key with u > 0 (P = 2^-40)
+// coarse mass a = floor(P * 2^21) = u >> kCoarseShift: a row of at most 1024
+// blocks sums to below 2^31, one 32-bit redux
+constexpr int kCoarseShift = 19;
 
 __device__ __forceinline__ uint32_t prob_key(float p) {
   // NaN and p <= 0 (incl. -0) -> 0; p > 1 (incl. inf) -> bits of 1.0f
@@ -47,6 +53,16 @@ __device__ __forceinline__ uint64_t fixed_mass(uint32_t key) {
   const int sh = e - 110;
   if (sh >= 0) return m << sh;  // e <= 127 -> sh <= 17: fits
   return (-sh >= 24) ? 0ull : (m >> (-sh));
+}
+
+// floor(P * 2^21) = floor(floor(P * 2^40) / 2^19), from the same bits:
+// m * 2^(e - 129), at most 2^21 (P = 1).
+__device__ __forceinline__ uint32_t coarse_mass(uint32_t key) {
+  const int e = static_cast<int>(key >> 23);
+  if (e == 0) return 0u;
+  const uint32_t m = (key & 0x7FFFFFu) | 0x800000u;
+  const int sh = 129 - e;  // >= 2 for e <= 127
+  return sh >= 24 ? 0u : (m >> sh);
 }
 
 // Exact warp sum of per-lane masses below 2^53 (a row's total is at most
@@ -180,16 +196,26 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ p
 }
 
 // Register-resident form of select_kernel for NB <= 32 R: lane l holds the
-// key and the fixed-point mass of blocks j = 32 r + l (r < R), so the 31-step
-// search reads no shared memory (the shared-memory form re-reads the whole
-// row at every step).  Same arithmetic and the same result bit for bit.
+// key and the coarse mass of blocks j = 32 r + l (r < R), so the search reads
+// no shared memory (the shared-memory form re-reads the whole row at every
+// step), and the exact masses are recomputed from the keys where needed.
+// The same threshold and the same result bit for bit; fewer steps:
+//   * step c is first decided on coarse masses: with A = sum_{key >= c} a,
+//     the exact S(c) = sum_{key >= c} u lies in [A 2^19, (A + NB) 2^19), so
+//     A 2^19 >= T means S(c) >= T and (A + NB) 2^19 <= T means S(c) < T;
+//     only in between is the exact uint64 sum taken;
+//   * after every odd bit from bit 15 down, the search stops when the
+//     bracket [tau, tau + 2^b) holds a single key value k among the blocks
+//     with mass: then S(k) = S(tau) >= T and S(k + 1) = S(tau + 2^b) < T,
+//     so k is the threshold the remaining steps would reach;
+//   * the tie scan runs only over register slots that hold a block equal to
+//     tau.
+// Three CTAs per SM up to 640 blocks a row (71 registers at R = 20).
 template <int R>
-__global__ void __launch_bounds__(256) select_reg_kernel(const float* __restrict__ probs,
-                                                         const __grid_constant__ TopP tp,
-                                                         const uint8_t* __restrict__ cand,
-                                                         uint8_t* __restrict__ mask, int32_t* __restrict__ kept_idx,
-                                                         int32_t* __restrict__ kept_cnt, int H, int NB,
-                                                         long long rows) {
+__global__ void __launch_bounds__(256, R <= 20 ? 3 : 2)
+    select_reg_kernel(const float* __restrict__ probs, const __grid_constant__ TopP tp,
+                      const uint8_t* __restrict__ cand, uint8_t* __restrict__ mask, int32_t* __restrict__ kept_idx,
+                      int32_t* __restrict__ kept_cnt, int H, int NB, long long rows) {
   const int warps = blockDim.x >> 5;
   const int w = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -211,7 +237,6 @@ __global__ void __launch_bounds__(256) select_reg_kernel(const float* __restrict
   }
 
   uint32_t key[R];
-  uint64_t u[R];
   uint64_t total = 0;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
@@ -219,8 +244,7 @@ __global__ void __launch_bounds__(256) select_reg_kernel(const float* __restrict
     uint32_t kk = 0u;
     if (j < NB && (!crow || crow[j])) kk = prob_key(__ldg(P + j));
     key[r] = kk;
-    u[r] = fixed_mass(kk);
-    total += u[r];
+    total += fixed_mass(kk);
   }
   total = warp_sum(total);
   const uint64_t T = static_cast<uint64_t>(ceil(static_cast<double>(p) * static_cast<double>(total)));
@@ -259,18 +283,50 @@ __global__ void __launch_bounds__(256) select_reg_kernel(const float* __restrict
       if (32 * r + lane == best_j) key[r] = kSelected;
     tau = kSelected - 1u;
   } else {
-    tau = kTopBits;  // largest tau with sum_{key >= tau} u >= T; its top two bits are known
+    uint32_t a[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) a[r] = coarse_mass(key[r]);
+    // largest tau with S(tau) = sum_{key >= tau} u >= T; its top two bits are
+    // known.  Before bit b: S(tau) >= T > S(tau + 2^(b+1)).
+    tau = kTopBits;
 #pragma unroll 1
     for (int b = 28; b >= 0; --b) {
       const uint32_t c = tau | (1u << b);
-      uint64_t g[4] = {0ull, 0ull, 0ull, 0ull};  // independent partial sums
+      uint32_t g[4] = {0u, 0u, 0u, 0u};  // independent partial sums
 #pragma unroll
-      for (int r = 0; r < R; ++r) g[r & 3] += key[r] >= c ? u[r] : 0ull;
-      if (warp_sum((g[0] + g[1]) + (g[2] + g[3])) >= T) tau = c;
+      for (int r = 0; r < R; ++r) g[r & 3] += key[r] >= c ? a[r] : 0u;
+      const uint64_t A = __reduce_add_sync(0xffffffffu, (g[0] + g[1]) + (g[2] + g[3]));
+      bool ge = (A << kCoarseShift) >= T;
+      if (!ge && ((A + static_cast<uint64_t>(NB)) << kCoarseShift) > T) {
+        // undecided on coarse masses: the exact sum
+        uint64_t e[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int r = 0; r < R; ++r) e[r & 3] += key[r] >= c ? fixed_mass(key[r]) : 0ull;
+        ge = warp_sum((e[0] + e[1]) + (e[2] + e[3])) >= T;
+      }
+      if (ge) tau = c;
+      if ((b & 1) && b <= 15) {
+        // the bracket is now [tau, tau + 2^b); its keys with mass are >= kMinMassKey
+        const uint32_t lo = tau > kMinMassKey ? tau : kMinMassKey;
+        const uint32_t hi = tau + (1u << b);
+        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          if (key[r] >= lo && key[r] < hi) {
+            kmin = min(kmin, key[r]);
+            kmax = max(kmax, key[r]);
+          }
+        kmin = __reduce_min_sync(0xffffffffu, kmin);
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        if (kmin == kmax) {  // one key value left (an empty bracket gives kmin > kmax)
+          tau = kmin;
+          break;
+        }
+      }
     }
     uint64_t above = 0;
 #pragma unroll
-    for (int r = 0; r < R; ++r) above += key[r] > tau ? u[r] : 0ull;
+    for (int r = 0; r < R; ++r) above += key[r] > tau ? fixed_mass(key[r]) : 0ull;
     const uint64_t need = T - warp_sum(above);  // > 0 by maximality of tau
     // blocks equal to tau, in ascending index order, while mass is short
     uint64_t carry = 0;
@@ -278,7 +334,8 @@ __global__ void __launch_bounds__(256) select_reg_kernel(const float* __restrict
     for (int r = 0; r < R; ++r) {
       const int j = 32 * r + lane;
       const bool tie = j < NB && key[r] == tau;
-      const uint64_t val = tie ? u[r] : 0ull;
+      if (!__any_sync(0xffffffffu, tie)) continue;  // no block of this slot equals tau
+      const uint64_t val = tie ? fixed_mass(key[r]) : 0ull;
       uint64_t incl = val;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
