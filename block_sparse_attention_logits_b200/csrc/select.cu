@@ -236,15 +236,31 @@ __global__ void __launch_bounds__(256, R <= 20 ? 3 : 2)
     return;
   }
 
+  // every load of the row in flight before the first use: the loads are
+  // predicated on the bounds only, and the candidate bytes are applied after
+  float pv[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int j = 32 * r + lane;
+    pv[r] = j < NB ? __ldg(P + j) : 0.f;
+  }
+  if (crow) {
+    uint8_t cv[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int j = 32 * r + lane;
+      cv[r] = j < NB ? crow[j] : 0;
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (!cv[r]) pv[r] = 0.f;  // key 0, mass 0
+  }
   uint32_t key[R];
   uint64_t total = 0;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    const int j = 32 * r + lane;
-    uint32_t kk = 0u;
-    if (j < NB && (!crow || crow[j])) kk = prob_key(__ldg(P + j));
-    key[r] = kk;
-    total += fixed_mass(kk);
+    key[r] = prob_key(pv[r]);
+    total += fixed_mass(key[r]);
   }
   total = warp_sum(total);
   const uint64_t T = static_cast<uint64_t>(ceil(static_cast<double>(p) * static_cast<double>(total)));
