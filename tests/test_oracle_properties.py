@@ -3,8 +3,10 @@ hypothesis, each checked against what the definitions imply -- top-p
 selection is the shortest ordered prefix reaching the target, interval
 encoding decodes back and merging adds the fewest blocks, the drift does not
 depend on the scale of the means, a refinement taken at the same step
-turns the coarse tail into the exact one, and E4M3 encoding is the nearest
-value, monotone, and bounded in its block quantization error."""
+turns the coarse tail into the exact one, E4M3 encoding is the nearest
+value, monotone, and bounded in its block quantization error, and the masked
+attention depends on the kept set only (not its order), is affine in V and
+moves its LSE by exactly q.c/sqrt(D) when every key is shifted by c."""
 
 import itertools
 
@@ -158,3 +160,49 @@ def test_block_quantization_error_is_one_e4m3_rounding(seed, L, spread):
     # of the scale for subnormal ones, plus the float32 rounding of x * (448 / amax)
     assert np.all(err[normal] <= (2.0 ** -4 + 2.0 ** -20) * np.abs(x[normal]))
     assert np.all(err[~normal] <= (2.0 ** -10 + 2.0 ** -20) * s[~normal])
+
+
+def _attention_case(seed, nblocks, ragged, blk=8, D=8):
+    rng = np.random.default_rng(seed)
+    L = max(1, nblocks * blk - ragged)
+    nb = (L + blk - 1) // blk
+    q, k, v = (rng.standard_normal((1, 1, L, D)) for _ in range(3))
+    idx = np.full((1, 1, nb, nb), -1, np.int32)
+    cnt = np.zeros((1, 1, nb), np.int32)
+    for i in range(nb):
+        kept = np.flatnonzero(rng.uniform(size=nb) < 0.6)
+        idx[0, 0, i, :len(kept)] = kept
+        cnt[0, 0, i] = len(kept)
+    return q, k, v, idx, cnt, blk, rng
+
+
+@SETTINGS
+@given(st.integers(0, 2 ** 31 - 1), st.integers(1, 5), st.integers(0, 7))
+def test_masked_attention_depends_on_the_kept_set_not_its_order(seed, nblocks, ragged):
+    q, k, v, idx, cnt, blk, rng = _attention_case(seed, nblocks, ragged)
+    shuffled = idx.copy()
+    for i in range(idx.shape[2]):
+        c = cnt[0, 0, i]
+        shuffled[0, 0, i, :c] = rng.permutation(idx[0, 0, i, :c])
+    O1, L1 = oatt.masked_attention(q, k, v, idx, cnt, blk)
+    O2, L2 = oatt.masked_attention(q, k, v, shuffled, cnt, blk)
+    np.testing.assert_allclose(np.nan_to_num(O2), np.nan_to_num(O1), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(np.nan_to_num(L2, neginf=0), np.nan_to_num(L1, neginf=0), rtol=0, atol=1e-12)
+
+
+@SETTINGS
+@given(st.integers(0, 2 ** 31 - 1), st.integers(1, 5), st.integers(0, 7), st.floats(-3.0, 3.0), st.floats(-3.0, 3.0))
+def test_masked_attention_is_affine_in_v_and_shift_invariant_in_k(seed, nblocks, ragged, a, b):
+    """Softmax weights sum to one per row: O(a V + b) = a O + b.  Adding one
+    vector c to every key adds q.c / sqrt(D) to every logit of a query row:
+    O is unchanged and LSE moves by exactly that amount."""
+    q, k, v, idx, cnt, blk, rng = _attention_case(seed, nblocks, ragged)
+    O, LSE = oatt.masked_attention(q, k, v, idx, cnt, blk)
+    rows = np.isfinite(LSE)  # rows that keep at least one block
+    Oa, _ = oatt.masked_attention(q, k, a * v + b, idx, cnt, blk)
+    np.testing.assert_allclose(Oa[rows], (a * O + b)[rows], rtol=0, atol=1e-9)
+    c = rng.standard_normal(q.shape[-1])
+    Os, Ls = oatt.masked_attention(q, k + c, v, idx, cnt, blk)
+    np.testing.assert_allclose(Os[rows], O[rows], rtol=0, atol=1e-9)
+    shift = (q @ c)[..., :] / np.sqrt(q.shape[-1])
+    np.testing.assert_allclose(Ls[rows], (LSE + shift)[rows], rtol=0, atol=1e-9)
